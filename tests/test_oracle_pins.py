@@ -1,0 +1,358 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each test fixes a part of the oracle against a value printed on the pages
+(tests/golden/*.txt), a closed form, an invariant, a special case that reduces to
+a stock library routine, or brute force on a tiny input.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import dit_synth as S
+from oracle import dit_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(fname):
+    with open(os.path.join(GOLDEN, fname)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def small_image(**kw):
+    base = S.DIT_S8_F32.with_(depth=2, hidden=96, heads=4, mlp_hidden=384, num_classes=10,
+                              height=16, width=16, patch_h=4, patch_w=4, batch=2, index=-1)
+    return base.with_(**kw)
+
+
+def small_video(**kw):
+    base = S.VIDEO_RF.with_(depth=2, hidden=72, heads=2, mlp_hidden=288, in_channels=3, frames=3,
+                            height=8, width=6, patch_t=1, patch_h=2, patch_w=2, batch=2, index=-1)
+    return base.with_(**kw)
+
+
+# ----------------------------------------------------------------------------- shapes / FLOPs
+def test_token_count_and_decoder_width():
+    for side, ch, p, tokens, width in (map(int, r) for r in _rows("shapes.txt")):
+        cfg = S.DIT_XL2_CFG256.with_(height=side, width=side, in_channels=ch, patch_h=p, patch_w=p)
+        assert cfg.tokens == tokens
+        assert cfg.out_dim == width
+        x = np.zeros((1, ch, 1, side, side))
+        assert O.patchify(x, 1, p, p).shape == (1, tokens, ch * p * p)
+
+
+@pytest.mark.parametrize("row", _rows("gflops_table.txt"))
+def test_mac_counter_reproduces_printed_gflops(row):
+    size, depth, hidden, heads, patch, side, printed = row
+    cfg = S.DIT_XL2_CFG256.with_(depth=int(depth), hidden=int(hidden), heads=int(heads),
+                                 mlp_hidden=4 * int(hidden), patch_h=int(patch), patch_w=int(patch),
+                                 height=int(side), width=int(side))
+    g = O.count_forward_macs(cfg) / 1e9
+    assert abs(g - float(printed)) <= 0.1, (size, g, printed)
+
+
+def test_mac_counter_range_ends():
+    rng = dict((r[0], float(r[1])) for r in _rows("gflops_range.txt"))
+    low = O.count_forward_macs(S.DIT_S8_F32) / 1e9
+    high = O.count_forward_macs(S.DIT_XL2_CFG256) / 1e9
+    assert math.floor(low * 10) / 10 == rng["low"]
+    assert abs(high - rng["high"]) < 0.05
+
+
+def test_mac_counter_dry_equals_real():
+    cfg = small_image()
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg, batch=1)
+    O.reset_mac_counter()
+    O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    real = O.mac_count()
+    assert real == O.count_forward_macs(cfg)
+    assert real > 0
+
+
+# ----------------------------------------------------------------------------- elementwise
+def test_layernorm_moments_and_library():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((5, 7, 96)) * 3 + 1.5
+    y = O.layernorm(x)
+    assert np.allclose(y.mean(-1), 0, atol=1e-12)
+    assert np.allclose(y.var(-1), 1, atol=1e-5)  # eps 1e-6 shrinks var by ~eps/var
+    ref = F.layer_norm(torch.from_numpy(x), (96,), eps=1e-6).numpy()
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+    # constant row -> zeros (eps keeps it finite)
+    assert np.all(O.layernorm(np.full((1, 8), 3.0)) == 0)
+
+
+def test_rmsnorm_unit_rms_and_library():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((4, 72)) * 5
+    g = rng.standard_normal(72)
+    assert np.allclose(np.sqrt((O.rmsnorm(x, np.ones(72)) ** 2).mean(-1)), 1, atol=1e-6)
+    ref = F.rms_norm(torch.from_numpy(x), (72,), torch.from_numpy(g), eps=1e-6).numpy()
+    assert np.allclose(O.rmsnorm(x, g), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_gelu_silu_library_and_special_values():
+    x = np.linspace(-8, 8, 1001)
+    assert np.allclose(O.gelu_tanh(x), F.gelu(torch.from_numpy(x), approximate="tanh").numpy(),
+                       rtol=1e-13, atol=1e-13)
+    assert np.allclose(O.silu(x), F.silu(torch.from_numpy(x)).numpy(), rtol=1e-13, atol=1e-13)
+    assert O.gelu_tanh(np.array([0.0]))[0] == 0.0
+    assert abs(O.gelu_tanh(np.array([20.0]))[0] - 20.0) < 1e-12
+    assert abs(O.gelu_tanh(np.array([-20.0]))[0]) < 1e-12
+
+
+def test_modulate_identity_at_zero():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((2, 3, 8))
+    z = np.zeros((2, 8))
+    assert np.array_equal(O.modulate(x, z, z), x)
+    sh = rng.standard_normal((2, 8))
+    out = O.modulate(x, sh, z)
+    assert np.allclose(out - x, np.broadcast_to(sh[:, None], x.shape))
+
+
+# ----------------------------------------------------------------------------- attention
+def test_attention_two_token_closed_form():
+    # q0 = (1,0) sees logits (1/sqrt2, 0): weight on key 0 is sigmoid(1/sqrt2);
+    # q1 = 0 sees equal logits: the mean of the values.
+    q = np.array([[1.0, 0.0], [0.0, 0.0]])
+    k = np.array([[1.0, 0.0], [0.0, 1.0]])
+    v = np.array([[1.0, 2.0], [3.0, 4.0]])
+    w0 = 1.0 / (1.0 + math.exp(-1.0 / math.sqrt(2.0)))
+    want = np.array([w0 * v[0] + (1 - w0) * v[1], (v[0] + v[1]) / 2])
+    assert np.allclose(O.attention(q, k, v), want, rtol=1e-14, atol=1e-14)
+
+
+def test_attention_zero_query_is_mean_and_library():
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((9, 6)) for _ in range(3))
+    assert np.allclose(O.attention(np.zeros_like(q), k, v), np.broadcast_to(v.mean(0), v.shape))
+    ref = F.scaled_dot_product_attention(*(torch.from_numpy(a)[None] for a in (q, k, v)))[0].numpy()
+    assert np.allclose(O.attention(q, k, v), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_brute_force_tiny():
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.standard_normal((3, 4)) for _ in range(3))
+    out = np.zeros((3, 4))
+    for i in range(3):
+        e = [math.exp(sum(q[i, a] * k[j, a] for a in range(4)) / 2.0) for j in range(3)]
+        z = sum(e)
+        for a in range(4):
+            out[i, a] = sum(e[j] / z * v[j, a] for j in range(3))
+    assert np.allclose(O.attention(q, k, v), out, rtol=1e-13, atol=1e-13)
+
+
+def test_attention_permutation():
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.standard_normal((7, 5)) for _ in range(3))
+    p = rng.permutation(7)
+    base = O.attention(q, k, v)
+    assert np.allclose(O.attention(q, k[p], v[p]), base)   # keys/values: invariant
+    assert np.allclose(O.attention(q[p], k, v), base[p])   # queries: equivariant
+
+
+# ----------------------------------------------------------------------------- embeddings
+def test_timestep_embedding_invariants():
+    e = O.timestep_embedding(np.array([0.0, 1.0, 999.0]), 256)
+    assert e.shape == (3, 256)
+    assert np.all(e[0, :128] == 1) and np.all(e[0, 128:] == 0)      # t = 0
+    assert np.allclose(e[:, :128] ** 2 + e[:, 128:] ** 2, 1)         # cos^2 + sin^2
+    assert np.allclose((e ** 2).sum(1), 128)                         # |e|^2 = dim/2
+    assert abs(e[1, 0] - math.cos(1.0)) < 1e-15 and abs(e[1, 128] - math.sin(1.0)) < 1e-15  # f_0 = 1
+    assert abs(math.acos(e[1, 127]) - 10000 ** (-127 / 128)) < 1e-12  # slowest frequency
+    e2 = O.timestep_embedding(np.array([0.5]), 256, t_scale=1000.0)
+    assert np.allclose(e2, O.timestep_embedding(np.array([500.0]), 256))
+
+
+def test_sincos_2d_invariants():
+    d, gh, gw = 96, 3, 5
+    pe = O.pos_embed_sincos_2d(gh, gw, d)
+    assert pe.shape == (gh * gw, d)
+    q = d // 4
+    first = pe[0]
+    assert np.all(first[:q] == 0) and np.all(first[q:2 * q] == 1)
+    assert np.all(first[2 * q:3 * q] == 0) and np.all(first[3 * q:] == 1)
+    assert np.allclose((pe ** 2).sum(1), d / 2)
+    tok = lambda r, c: r * gw + c
+    assert np.array_equal(pe[tok(2, 1), :d // 2], pe[tok(2, 4), :d // 2])   # same row
+    assert np.array_equal(pe[tok(0, 3), d // 2:], pe[tok(2, 3), d // 2:])   # same column
+    assert abs(pe[tok(0, 1), d // 2] - math.sin(1.0)) < 1e-15               # w_0 = 1
+
+
+def test_rope_invariants():
+    rng = np.random.default_rng(6)
+    coords = O.token_coords((2, 3, 4))
+    q = rng.standard_normal((24, 72))
+    k = rng.standard_normal((24, 72))
+    rq = O.rope_3d(q, coords)
+    assert np.allclose(np.linalg.norm(rq, axis=1), np.linalg.norm(q, axis=1))
+    assert np.array_equal(O.rope_3d(q, np.zeros_like(coords)), q)
+    shifted = coords + np.array([3, -2, 5])
+    assert np.allclose(O.rope_3d(q, coords) @ O.rope_3d(k, coords).T,
+                       O.rope_3d(q, shifted) @ O.rope_3d(k, shifted).T)
+    # first pair of the time slice turns by exactly the frame index (theta_0 = 1)
+    ang = math.atan2(rq[12, 1], rq[12, 0]) - math.atan2(q[12, 1], q[12, 0])
+    assert abs(math.remainder(ang - coords[12, 0], 2 * math.pi)) < 1e-12
+
+
+def test_patchify_is_conv_and_unpatchify_is_rearrange():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((2, 3, 4, 8, 6))
+    w = rng.standard_normal((5, 3 * 2 * 2 * 3))
+    tok = O.patchify(x, 2, 2, 3) @ w.T
+    ref = F.conv3d(torch.from_numpy(x), torch.from_numpy(w).view(5, 3, 2, 2, 3), stride=(2, 2, 3))
+    assert np.allclose(tok, ref.flatten(2).transpose(1, 2).numpy(), rtol=1e-12, atol=1e-12)
+    grid = (2, 4, 2)
+    z = rng.standard_normal((2, 16, 2 * 2 * 3 * 3))
+    img = O.unpatchify(z, 3, grid, 2, 2, 3)
+    import einops
+    ref = einops.rearrange(z, "n (f h w) (a p q c) -> n c (f a) (h p) (w q)", f=2, h=4, w=2, a=2, p=2, q=3, c=3)
+    assert np.array_equal(img, ref)
+
+
+def test_unpatchify_inverts_channel_last_patchify():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((2, 4, 1, 8, 8))
+    v = O.patchify(x, 1, 2, 2).reshape(2, 16, 4, 1, 2, 2).transpose(0, 1, 3, 4, 5, 2).reshape(2, 16, 16)
+    assert np.array_equal(O.unpatchify(v, 4, (1, 4, 4), 1, 2, 2), x)
+
+
+def test_one_hot_embedding_picks_input_element():
+    cfg = small_image(depth=0)
+    W = S.weight_dict(cfg, S.make_weights(cfg))
+    x = np.random.default_rng(9).standard_normal(cfg.x_shape(1))
+    W = dict(W)
+    w = np.zeros_like(W["pe.w"])
+    c, ih, iw = 2, 1, 3
+    w[0, c * 16 + ih * 4 + iw] = 1.0
+    W["pe.w"] = w
+    W["pe.b"] = np.zeros_like(W["pe.b"])
+    h = O.linear(O.patchify(x[:, :, None], 1, 4, 4), W["pe.w"], W["pe.b"])
+    for i in range(4):
+        for j in range(4):
+            assert h[0, i * 4 + j, 0] == x[0, c, 4 * i + ih, 4 * j + iw]
+
+
+# ----------------------------------------------------------------------------- blocks / forward
+def test_zero_adaln_block_is_identity_bit_exact():
+    cfg = small_image()
+    W = S.weight_dict(cfg, S.set_adaln(cfg, S.make_weights(cfg), zero=True))
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((3, cfg.tokens, cfg.hidden))
+    sc = O.silu(rng.standard_normal((3, cfg.hidden)))
+    assert np.array_equal(O.dit_block(x, sc, W, "blocks.0.", cfg.heads), x)
+
+
+def test_zero_adaln_forward_skips_blocks():
+    cfg = small_image()
+    W = S.weight_dict(cfg, S.set_adaln(cfg, S.make_weights(cfg), zero=True))
+    inp = S.make_inputs(cfg)
+    out = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    h = O.embed(cfg, W, inp["x"][:, :, None])
+    sc = O.silu(O.condition(cfg, W, inp["t"], inp["y"]))
+    z = O.final_layer(h, sc, W)
+    want = O.unpatchify(z, cfg.out_channels, cfg.grid, 1, 4, 4)[:, :, 0]
+    assert np.array_equal(out, want)
+    assert np.array_equal(O.forward(cfg, W, inp["x"], inp["t"], inp["y"], stop_after_block=2), h)
+
+
+def test_block_is_token_permutation_equivariant():
+    cfg = small_image()
+    W = S.weight_dict(cfg, S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0))
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((2, cfg.tokens, cfg.hidden))
+    sc = O.silu(rng.standard_normal((2, cfg.hidden)))
+    p = rng.permutation(cfg.tokens)
+    a = O.dit_block(x, sc, W, "blocks.0.", cfg.heads)[:, p]
+    b = O.dit_block(x[:, p], sc, W, "blocks.0.", cfg.heads)
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_batch_rows_independent():
+    cfg = small_image(batch=3)
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    full = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    for i in range(3):
+        one = O.forward(cfg, W, inp["x"][i:i + 1], inp["t"][i:i + 1], inp["y"][i:i + 1])
+        assert np.allclose(one[0], full[i], rtol=1e-12, atol=1e-12)
+
+
+def test_guidance_special_cases():
+    cfg = small_image(cfg_scale=1.5)
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    x, t, y = inp["x"], inp["t"], inp["y"]
+    cond = O.forward(cfg, W, x, t, y, cfg_scale=1.0)
+    uncond = O.forward(cfg, W, x, t, np.full_like(y, cfg.num_classes), cfg_scale=1.0)
+    s1 = O.forward(cfg, W, x, t, y, cfg_scale=1.0, force_guidance=True)
+    s0 = O.forward(cfg, W, x, t, y, cfg_scale=0.0)
+    s15 = O.forward(cfg, W, x, t, y)
+    s3 = O.forward(cfg, W, x, t, y, cfg_scale=3.0)
+    assert np.allclose(s1, cond, rtol=1e-12, atol=1e-12)
+    assert np.allclose(s0, uncond, rtol=1e-12, atol=1e-12)
+    assert np.array_equal(O.cfg_combine(cond, uncond, 0.0), uncond)
+    assert np.allclose(s15, uncond + 1.5 * (cond - uncond), rtol=1e-12, atol=1e-12)
+    assert np.allclose(s3 - s15, (3.0 - 1.5) * (cond - uncond), rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("kind", ["image", "image_guided", "video"])
+def test_forward_matches_torch_layers(kind):
+    from torch_reference import reference_forward
+    if kind == "video":
+        cfg = small_video()
+    else:
+        cfg = small_image(cfg_scale=1.5 if kind == "image_guided" else 1.0)
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    got = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    want = reference_forward(cfg, S.weight_dict(cfg, W), inp["x"], inp["t"], inp["y"])
+    assert got.shape == want.shape == cfg.out_shape()
+    assert np.allclose(got, want, rtol=1e-9, atol=1e-10), np.abs(got - want).max()
+
+
+_PLANTS = {
+    "erf_gelu": ("gelu_tanh", lambda x: 0.5 * np.asarray(x) * (1 + np.vectorize(math.erf)(np.asarray(x) / math.sqrt(2)))),
+    "chunk_order": ("adaln_chunks", None),
+    "no_gate": ("dit_block", None),
+    "ln_eps": ("layernorm", lambda x, eps=1e-6: O.__dict__["_orig_layernorm"](x, eps=1e-2)),
+    "attn_scale": ("attention", None),
+}
+
+
+@pytest.mark.parametrize("plant", sorted(_PLANTS))
+def test_oracle_catches_planted_mistakes(plant, monkeypatch):
+    """A plausible slip planted in the oracle (wrong GELU, swapped modulation
+    chunks, a dropped gate, a wrong LN eps, a wrong attention scale) makes the
+    torch-layer cross-check fail by far more than its tolerance."""
+    from torch_reference import reference_forward
+    cfg = small_image()
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    Wd = S.weight_dict(cfg, W)
+    inp = S.make_inputs(cfg)
+    want = reference_forward(cfg, Wd, inp["x"], inp["t"], inp["y"])
+    name, fn = _PLANTS[plant]
+    orig = getattr(O, name)
+    monkeypatch.setitem(O.__dict__, "_orig_layernorm", O.layernorm)
+    if plant == "chunk_order":
+        fn = lambda sc, w, b, n: orig(sc, w, b, n)[::-1]
+    elif plant == "no_gate":
+        def fn(x, sc, W_, prefix, heads, coords=None):
+            W2 = dict(W_)
+            W2[prefix + "ada.b"] = W_[prefix + "ada.b"].copy()
+            W2[prefix + "ada.b"][2 * cfg.hidden:3 * cfg.hidden] = 0.0
+            W2[prefix + "ada.w"] = W_[prefix + "ada.w"].copy()
+            W2[prefix + "ada.w"][2 * cfg.hidden:3 * cfg.hidden] = 0.0
+            return orig(x, sc, W2, prefix, heads, coords)
+    elif plant == "attn_scale":
+        fn = lambda q, k, v: orig(q * math.sqrt(q.shape[1]) ** 0.5, k, v)
+    monkeypatch.setattr(O, name, fn)
+    got = O.forward(cfg, Wd, inp["x"], inp["t"], inp["y"])
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    assert rel > 1e-7, rel  # the cross-check above holds the oracle to ~1e-9
