@@ -1,0 +1,228 @@
+"""ctypes binding of libdit_b200.so (include/dit.h).
+
+Argument marshalling only: every step of the forward runs in the library's CUDA
+kernels.  torch provides device memory and streams.  If the library is missing or
+cannot be loaded, every call raises; there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_float, c_int, c_uint16, c_void_p
+from typing import Optional, Sequence
+
+import numpy as np
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdit_b200.so")
+
+DIT_OK, DIT_ERR_INVALID_ARG, DIT_ERR_UNSUPPORTED, DIT_ERR_OOM, DIT_ERR_CUDA = 0, 1, 2, 3, 4
+DIT_ERR_DEVICE_TIMEOUT, DIT_ERR_BAD_LABEL, DIT_ERR_NO_DEVICE = 5, 6, 7
+DIT_OPT_FORCE_GUIDANCE, DIT_OPT_USE_GRAPH = 1, 2
+
+# every exported symbol declared in include/dit.h
+EXPORTS = [
+    "dit_create", "dit_weight_count", "dit_forward", "dit_forward_host", "dit_sync_status", "dit_last_error",
+    "dit_status_string", "dit_destroy", "dit_set_option", "dit_debug_residual", "dit_debug_condition",
+    "dit_debug_wait_probe", "dit_op_linear_bf16", "dit_forward_launch_count", "dit_profile_enable",
+    "dit_profile_read",
+]
+
+KERNEL_KINDS = ["cond", "adaln", "patch", "ln", "qkv", "attn", "proj", "fc1", "fc2", "decode"]
+
+
+class DitConfig(ctypes.Structure):
+    _fields_ = [("dtype", c_int), ("in_channels", c_int), ("frames", c_int), ("height", c_int), ("width", c_int),
+                ("patch_t", c_int), ("patch_h", c_int), ("patch_w", c_int), ("hidden", c_int), ("depth", c_int),
+                ("heads", c_int), ("mlp_hidden", c_int), ("learn_sigma", c_int), ("pos_kind", c_int),
+                ("qk_norm", c_int), ("cond_kind", c_int), ("num_classes", c_int), ("freq_dim", c_int),
+                ("max_batch", c_int), ("t_scale", c_float)]
+
+
+class DitError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(msg)
+        self.code = code
+
+
+_LIB = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the library (raises if it was not built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with python -m diffusion_transformer_denoiser_dit_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = c_void_p
+    sig = {
+        "dit_create": (c_int, [POINTER(DitConfig), POINTER(c_void_p), c_int, POINTER(c_void_p)]),
+        "dit_weight_count": (c_int, [POINTER(DitConfig)]),
+        "dit_forward": (c_int, [P, P, P, P, c_int, c_float, P, P]),
+        "dit_forward_host": (c_int, [P, P, P, P, c_int, c_float, P, P]),
+        "dit_sync_status": (c_int, [P]),
+        "dit_last_error": (ctypes.c_char_p, [P]),
+        "dit_status_string": (ctypes.c_char_p, [c_int]),
+        "dit_destroy": (None, [P]),
+        "dit_set_option": (c_int, [P, c_int, c_int]),
+        "dit_debug_residual": (c_int, [P, P, P, P, c_int, c_float, c_int, P, P]),
+        "dit_debug_condition": (c_int, [P, P, P, c_int, c_float, P, P]),
+        "dit_debug_wait_probe": (c_int, [P, c_int, P]),
+        "dit_op_linear_bf16": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, P]),
+        "dit_forward_launch_count": (c_int, [P, c_int, c_float]),
+        "dit_profile_enable": (c_int, [P, c_int]),
+        "dit_profile_read": (c_int, [P, POINTER(c_float), POINTER(c_int)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = lib
+    return lib
+
+
+def make_config(cfg, max_batch: Optional[int] = None) -> DitConfig:
+    """dit_config from any object with the same field names (e.g. dit_synth.DiTConfig)."""
+    mb = max_batch if max_batch is not None else cfg.batch
+    return DitConfig(cfg.dtype, cfg.in_channels, cfg.frames, cfg.height, cfg.width, cfg.patch_t, cfg.patch_h,
+                     cfg.patch_w, cfg.hidden, cfg.depth, cfg.heads, cfg.mlp_hidden, cfg.learn_sigma, cfg.pos_kind,
+                     cfg.qk_norm, cfg.cond_kind, cfg.num_classes, cfg.freq_dim, mb, float(cfg.t_scale))
+
+
+def status_string(code: int) -> str:
+    return load().dit_status_string(code).decode()
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+class DiT:
+    """A created model: device weights + workspace owned by the library."""
+
+    def __init__(self, cfg, weights: Sequence[np.ndarray], max_batch: Optional[int] = None):
+        self.lib = load()
+        self.cfg = cfg
+        self._c = make_config(cfg, max_batch)
+        arrs = [np.ascontiguousarray(w, dtype=np.float32) for w in weights]
+        ptrs = (c_void_p * len(arrs))(*[a.ctypes.data for a in arrs])
+        h = c_void_p()
+        rc = self.lib.dit_create(ctypes.byref(self._c), ptrs, len(arrs), ctypes.byref(h))
+        if rc != DIT_OK:
+            raise DitError(rc, f"dit_create failed: {status_string(rc)}")
+        self.h = h
+
+    # ---- helpers
+    def _check(self, rc: int, what: str):
+        if rc != DIT_OK:
+            msg = self.lib.dit_last_error(self.h).decode() if self.h else ""
+            raise DitError(rc, f"{what}: {status_string(rc)} {msg}")
+
+    def rows(self, B: int, cfg_scale: float) -> int:
+        return 2 * B if (self.cfg.cond_kind == 0 and cfg_scale != 1.0) else B
+
+    def out_shape(self, B: int):
+        return self.cfg.out_shape(B)
+
+    # ---- calls
+    def forward(self, x, t, y, cfg_scale: float, out=None, stream=None):
+        import torch
+        B = x.shape[0]
+        if out is None:
+            out = torch.empty(self.out_shape(B), dtype=torch.float32, device=x.device)
+        rc = self.lib.dit_forward(self.h, _ptr(x), _ptr(t), _ptr(y), B, float(cfg_scale), _ptr(out), _stream(stream))
+        self._check(rc, "dit_forward")
+        return out
+
+    def forward_host(self, x: np.ndarray, t: np.ndarray, y: np.ndarray, cfg_scale: float, out: np.ndarray = None,
+                     stream=None):
+        B = x.shape[0]
+        if out is None:
+            out = np.empty(self.out_shape(B), dtype=np.float32)
+        rc = self.lib.dit_forward_host(self.h, x.ctypes.data, t.ctypes.data, y.ctypes.data, B, float(cfg_scale),
+                                       out.ctypes.data, _stream(stream))
+        self._check(rc, "dit_forward_host")
+        return out
+
+    def forward_host_ptr(self, x_ptr: int, t_ptr: int, y_ptr: int, B: int, cfg_scale: float, out_ptr: int,
+                         stream=None):
+        rc = self.lib.dit_forward_host(self.h, x_ptr, t_ptr, y_ptr, B, float(cfg_scale), out_ptr, _stream(stream))
+        self._check(rc, "dit_forward_host")
+
+    def debug_residual(self, x, t, y, cfg_scale: float, after_block: int, stream=None):
+        import torch
+        B = x.shape[0]
+        R = self.rows(B, cfg_scale) if not getattr(self, "_force", False) else 2 * B
+        h = torch.empty((R, self.cfg.tokens, self.cfg.hidden), dtype=torch.float32, device=x.device)
+        rc = self.lib.dit_debug_residual(self.h, _ptr(x), _ptr(t), _ptr(y), B, float(cfg_scale), after_block, _ptr(h),
+                                         _stream(stream))
+        self._check(rc, "dit_debug_residual")
+        return h
+
+    def debug_condition(self, t, y, cfg_scale: float, stream=None):
+        import torch
+        B = t.shape[0]
+        R = self.rows(B, cfg_scale) if not getattr(self, "_force", False) else 2 * B
+        c = torch.empty((R, self.cfg.hidden), dtype=torch.float32, device=t.device)
+        rc = self.lib.dit_debug_condition(self.h, _ptr(t), _ptr(y), B, float(cfg_scale), _ptr(c), _stream(stream))
+        self._check(rc, "dit_debug_condition")
+        return c
+
+    def set_option(self, option: int, value: int):
+        self._check(self.lib.dit_set_option(self.h, option, value), "dit_set_option")
+        if option == DIT_OPT_FORCE_GUIDANCE:
+            self._force = bool(value)
+
+    def sync_status(self) -> int:
+        return self.lib.dit_sync_status(self.h)
+
+    def wait_probe(self, timeout_us: int, stream=None):
+        self._check(self.lib.dit_debug_wait_probe(self.h, timeout_us, _stream(stream)), "dit_debug_wait_probe")
+
+    def launch_count(self, B: int, cfg_scale: float) -> int:
+        return self.lib.dit_forward_launch_count(self.h, B, float(cfg_scale))
+
+    def profile(self, enable: bool):
+        self._check(self.lib.dit_profile_enable(self.h, int(enable)), "dit_profile_enable")
+
+    def profile_read(self):
+        """{kind: (total_ms, launches)} of the launches recorded since the last read."""
+        n = len(KERNEL_KINDS)
+        ms = (c_float * n)()
+        cnt = (c_int * n)()
+        self._check(self.lib.dit_profile_read(self.h, ms, cnt), "dit_profile_read")
+        return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
+
+    def close(self):
+        if getattr(self, "h", None):
+            self.lib.dit_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def linear_bf16(x, w, b, block_n: int = 128, stream=None):
+    """y = x W^T + b on the tensor-core GEMM (x, w: torch bf16 CUDA tensors)."""
+    import torch
+    lib = load()
+    M, K = x.shape
+    N = w.shape[0]
+    y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    rc = lib.dit_op_linear_bf16(_ptr(x), _ptr(w), _ptr(b), _ptr(y), M, N, K, block_n, _stream(stream))
+    if rc != DIT_OK:
+        raise DitError(rc, f"dit_op_linear_bf16: {status_string(rc)}")
+    return y

@@ -1,0 +1,814 @@
+// C-ABI layer: configuration checks, device weights and workspace, tensor maps,
+// and the kernel sequence of one DiT denoiser forward.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace dit;
+
+namespace {
+
+struct BlockW {
+  void *qkv_w = nullptr, *proj_w = nullptr, *fc1_w = nullptr, *fc2_w = nullptr;  // bf16 or f32
+  float *qkv_b = nullptr, *proj_b = nullptr, *fc1_b = nullptr, *fc2_b = nullptr;
+  float *qn = nullptr, *kn = nullptr;
+  CUtensorMap tm_qkv, tm_proj, tm_fc1, tm_fc2;
+};
+
+struct Geometry {
+  int gf, gh, gw, T, Kp, P, Cout, dh, DP, Tpad, Rmax, RPalloc, Mmax, nmod;
+  int bn_qkv, bn_proj, bn_fc1, bn_fc2;
+};
+
+bool validate(const dit_config* c, std::string& err) {
+  auto bad = [&](const char* m) {
+    err = m;
+    return false;
+  };
+  if (c == nullptr) return bad("config is NULL");
+  if (c->dtype != DIT_DTYPE_F32 && c->dtype != DIT_DTYPE_BF16) return bad("dtype must be DIT_DTYPE_F32 or DIT_DTYPE_BF16");
+  if (c->in_channels <= 0 || c->frames <= 0 || c->height <= 0 || c->width <= 0) return bad("latent extent must be positive");
+  if (c->patch_t <= 0 || c->patch_h <= 0 || c->patch_w <= 0) return bad("patch extent must be positive");
+  if (c->frames % c->patch_t || c->height % c->patch_h || c->width % c->patch_w)
+    return bad("patch extent must divide the latent extent");
+  if (c->hidden <= 0 || c->depth < 0 || c->heads <= 0 || c->mlp_hidden <= 0) return bad("model sizes must be positive");
+  if (c->hidden % c->heads) return bad("hidden must be a multiple of heads");
+  if (c->learn_sigma != 0 && c->learn_sigma != 1) return bad("learn_sigma must be 0 or 1");
+  if (c->pos_kind != DIT_POS_SINCOS2D && c->pos_kind != DIT_POS_ROPE3D) return bad("unknown pos_kind");
+  if (c->qk_norm != 0 && c->qk_norm != 1) return bad("qk_norm must be 0 or 1");
+  if (c->cond_kind != DIT_COND_CLASS && c->cond_kind != DIT_COND_VECTOR) return bad("unknown cond_kind");
+  if (c->cond_kind == DIT_COND_CLASS && c->num_classes <= 0) return bad("num_classes must be positive");
+  if (c->freq_dim <= 0 || (c->freq_dim & 1)) return bad("freq_dim must be positive and even");
+  if (c->max_batch <= 0) return bad("max_batch must be positive");
+  if (!isfinite(c->t_scale)) return bad("t_scale must be finite");
+  return true;
+}
+
+// Shapes the kernels cover (DIT_ERR_UNSUPPORTED otherwise).
+bool supported(const dit_config* c, std::string& err) {
+  const int dh = c->hidden / c->heads;
+  if (dh != 64 && dh != 72) {
+    err = "head dim (hidden / heads) must be 64 or 72";
+    return false;
+  }
+  if (c->hidden % 4 || c->hidden > 1536) {
+    err = "hidden must be a multiple of 4 and at most 1536";
+    return false;
+  }
+  if (c->pos_kind == DIT_POS_SINCOS2D && (c->frames / c->patch_t != 1 || c->hidden % 4)) {
+    err = "2D sin-cos positions need one frame of patches and hidden % 4 == 0";
+    return false;
+  }
+  if (c->pos_kind == DIT_POS_ROPE3D && dh % 6) {
+    err = "3D RoPE needs head dim % 6 == 0";
+    return false;
+  }
+  if (c->dtype == DIT_DTYPE_BF16) {
+    if (c->hidden % (2 * dh) || c->mlp_hidden % 8) {
+      err = "bf16 path needs an even number of heads and mlp_hidden % 8 == 0";
+      return false;
+    }
+  }
+  const long long kp = 1LL * c->in_channels * c->patch_t * c->patch_h * c->patch_w;
+  if (kp * 16 * 4 > 200 * 1024) {
+    err = "patch vector too long";
+    return false;
+  }
+  return true;
+}
+
+Geometry geometry(const dit_config* c) {
+  Geometry g;
+  g.gf = c->frames / c->patch_t;
+  g.gh = c->height / c->patch_h;
+  g.gw = c->width / c->patch_w;
+  g.T = g.gf * g.gh * g.gw;
+  g.Kp = c->in_channels * c->patch_t * c->patch_h * c->patch_w;
+  g.Cout = c->learn_sigma ? 2 * c->in_channels : c->in_channels;
+  g.P = c->patch_t * c->patch_h * c->patch_w * g.Cout;
+  g.dh = c->hidden / c->heads;
+  g.DP = (g.dh + 15) / 16 * 16;
+  g.Tpad = (g.T + 127) / 128 * 128;
+  g.Rmax = c->cond_kind == DIT_COND_CLASS ? 2 * c->max_batch : c->max_batch;
+  g.RPalloc = (g.Rmax + 255) / 256 * 256;
+  g.Mmax = g.Rmax * g.T;
+  g.nmod = (6 * c->depth + 2) * c->hidden;
+  g.bn_qkv = 2 * g.dh;
+  g.bn_proj = 2 * g.dh;
+  g.bn_fc1 = 2 * g.dh;
+  g.bn_fc2 = 2 * g.dh;
+  return g;
+}
+
+int weight_count(const dit_config* c) {
+  const int per_block = 10 + (c->qk_norm ? 2 : 0);
+  return 6 + (c->cond_kind == DIT_COND_CLASS ? 1 : 0) + c->depth * per_block + 4;
+}
+
+int adaln_bn(int R) {
+  if (R <= 16) return 16;
+  if (R <= 32) return 32;
+  if (R <= 64) return 64;
+  if (R <= 128) return 128;
+  return 256;
+}
+
+}  // namespace
+
+struct dit_handle {
+  dit_config cfg;
+  Geometry g;
+  bool bf16 = false;
+  int device = 0, num_sms = 148;
+  std::string err;
+  std::vector<void*> allocs;
+  // weights
+  float *pe_w = nullptr, *pe_b = nullptr, *t_w1 = nullptr, *t_b1 = nullptr, *t_w2 = nullptr, *t_b2 = nullptr;
+  float* table = nullptr;
+  void* ada_w = nullptr;
+  float* ada_b = nullptr;
+  std::vector<BlockW> blk;
+  float *dec_w = nullptr, *dec_b = nullptr;
+  float *pos = nullptr, *rope = nullptr;
+  // workspace
+  float *E = nullptr, *hid = nullptr, *c = nullptr, *mod = nullptr, *h = nullptr;
+  void *sc = nullptr, *u = nullptr, *q = nullptr, *k = nullptr, *v = nullptr, *o = nullptr, *gbuf = nullptr;
+  int *status = nullptr, *probe_flag = nullptr;
+  float *x_stage = nullptr, *t_stage = nullptr, *out_stage = nullptr;
+  void* y_stage = nullptr;
+  CUtensorMap tm_ada, tm_sc[5], tm_u, tm_o, tm_g;
+  int force_guidance = 0;
+  int use_graph = 0;
+  // per-launch event timing (dit_profile_enable)
+  bool prof = false;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<std::pair<int, int>> prof_recs;  // (kind, index of the start event in ev_pool)
+
+  template <typename T>
+  T* alloc(size_t bytes, bool zero = true) {
+    void* p = nullptr;
+    if (bytes == 0) bytes = 16;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
+    allocs.push_back(p);
+    if (zero) cudaMemset(p, 0, bytes);
+    return static_cast<T*>(p);
+  }
+};
+
+static dit_status fail(dit_handle* h, dit_status s, const std::string& m) {
+  if (h) h->err = m;
+  return s;
+}
+
+static dit_status cuda_fail(dit_handle* h, cudaError_t e, const char* where) {
+  std::string m = std::string(where) + ": " + cudaGetErrorString(e);
+  return fail(h, DIT_ERR_CUDA, m);
+}
+
+#define DIT_CK(h, call, where)                       \
+  do {                                               \
+    cudaError_t e_ = (call);                         \
+    if (e_ != cudaSuccess) return cuda_fail(h, e_, where); \
+  } while (0)
+
+extern "C" {
+
+int dit_weight_count(const dit_config* cfg) {
+  std::string e;
+  if (!validate(cfg, e)) return 0;
+  return weight_count(cfg);
+}
+
+const char* dit_status_string(dit_status s) {
+  switch (s) {
+    case DIT_OK: return "DIT_OK";
+    case DIT_ERR_INVALID_ARG: return "DIT_ERR_INVALID_ARG";
+    case DIT_ERR_UNSUPPORTED: return "DIT_ERR_UNSUPPORTED";
+    case DIT_ERR_OOM: return "DIT_ERR_OOM";
+    case DIT_ERR_CUDA: return "DIT_ERR_CUDA";
+    case DIT_ERR_DEVICE_TIMEOUT: return "DIT_ERR_DEVICE_TIMEOUT";
+    case DIT_ERR_BAD_LABEL: return "DIT_ERR_BAD_LABEL";
+    case DIT_ERR_NO_DEVICE: return "DIT_ERR_NO_DEVICE";
+  }
+  return "DIT_ERR_UNKNOWN";
+}
+
+const char* dit_last_error(const dit_handle* h) { return h ? h->err.c_str() : "null handle"; }
+
+void dit_destroy(dit_handle* h) {
+  if (h == nullptr) return;
+  cudaDeviceSynchronize();
+  for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
+  for (void* p : h->allocs) cudaFree(p);
+  delete h;
+}
+
+// Upload one host float32 tensor to a float32 device buffer, or convert it to bf16
+// through a float32 staging buffer.
+static dit_status upload(dit_handle* H, const float* src, size_t n, void* dst, bool to_bf16, float* staging) {
+  if (!to_bf16) {
+    DIT_CK(H, cudaMemcpy(dst, src, n * 4, cudaMemcpyHostToDevice), "weight upload");
+    return DIT_OK;
+  }
+  DIT_CK(H, cudaMemcpy(staging, src, n * 4, cudaMemcpyHostToDevice), "weight upload");
+  DIT_CK(H, launch_f32_to_bf16(staging, static_cast<uint16_t*>(dst), n, 0), "bf16 convert");
+  DIT_CK(H, cudaDeviceSynchronize(), "bf16 convert");
+  return DIT_OK;
+}
+
+dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_weights, dit_handle** out) {
+  std::string err;
+  if (out == nullptr) return DIT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!validate(cfg, err)) return DIT_ERR_INVALID_ARG;
+  if (weights == nullptr || n_weights != weight_count(cfg)) return DIT_ERR_INVALID_ARG;
+  for (int i = 0; i < n_weights; ++i)
+    if (weights[i] == nullptr) return DIT_ERR_INVALID_ARG;
+  if (!supported(cfg, err)) return DIT_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DIT_ERR_NO_DEVICE;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major != 10) return DIT_ERR_NO_DEVICE;
+
+  dit_handle* H = new dit_handle();
+  H->cfg = *cfg;
+  H->g = geometry(cfg);
+  H->bf16 = cfg->dtype == DIT_DTYPE_BF16;
+  H->device = dev;
+  H->num_sms = prop.multiProcessorCount;
+  const Geometry& g = H->g;
+  const int d = cfg->hidden, mlp = cfg->mlp_hidden, N = cfg->depth;
+  const size_t es = H->bf16 ? 2 : 4;
+
+#define ALLOC(ptr, T, bytes)                                      \
+  do {                                                            \
+    ptr = H->alloc<T>(bytes);                                     \
+    if (ptr == nullptr) {                                         \
+      dit_destroy(H);                                             \
+      return DIT_ERR_OOM;                                         \
+    }                                                             \
+  } while (0)
+
+  // ---------------- weights
+  ALLOC(H->pe_w, float, (size_t)d * g.Kp * 4);
+  ALLOC(H->pe_b, float, (size_t)d * 4);
+  ALLOC(H->t_w1, float, (size_t)d * cfg->freq_dim * 4);
+  ALLOC(H->t_b1, float, (size_t)d * 4);
+  ALLOC(H->t_w2, float, (size_t)d * d * 4);
+  ALLOC(H->t_b2, float, (size_t)d * 4);
+  if (cfg->cond_kind == DIT_COND_CLASS) ALLOC(H->table, float, (size_t)(cfg->num_classes + 1) * d * 4);
+  ALLOC(H->ada_w, void, (size_t)g.nmod * d * es);
+  ALLOC(H->ada_b, float, (size_t)g.nmod * 4);
+  H->blk.resize(N);
+  for (int i = 0; i < N; ++i) {
+    BlockW& b = H->blk[i];
+    ALLOC(b.qkv_w, void, (size_t)3 * d * d * es);
+    ALLOC(b.qkv_b, float, (size_t)3 * d * 4);
+    ALLOC(b.proj_w, void, (size_t)d * d * es);
+    ALLOC(b.proj_b, float, (size_t)d * 4);
+    ALLOC(b.fc1_w, void, (size_t)mlp * d * es);
+    ALLOC(b.fc1_b, float, (size_t)mlp * 4);
+    ALLOC(b.fc2_w, void, (size_t)d * mlp * es);
+    ALLOC(b.fc2_b, float, (size_t)d * 4);
+    if (cfg->qk_norm) {
+      ALLOC(b.qn, float, (size_t)g.dh * 4);
+      ALLOC(b.kn, float, (size_t)g.dh * 4);
+    }
+  }
+  ALLOC(H->dec_w, float, (size_t)g.P * d * 4);
+  ALLOC(H->dec_b, float, (size_t)g.P * 4);
+  if (cfg->pos_kind == DIT_POS_SINCOS2D) ALLOC(H->pos, float, (size_t)g.T * d * 4);
+  else ALLOC(H->rope, float, (size_t)g.T * g.dh * 4);
+
+  // ---------------- workspace
+  const size_t R = g.Rmax, M = g.Mmax;
+  ALLOC(H->E, float, R * cfg->freq_dim * 4);
+  ALLOC(H->hid, float, R * d * 4);
+  ALLOC(H->c, float, R * d * 4);
+  ALLOC(H->sc, void, (size_t)g.RPalloc * d * es);
+  ALLOC(H->mod, float, R * g.nmod * 4);
+  ALLOC(H->h, float, M * d * 4);
+  ALLOC(H->u, void, M * d * es);
+  if (H->bf16) {
+    const size_t qk = R * cfg->heads * (size_t)g.Tpad * g.DP * 2;
+    ALLOC(H->q, void, qk);
+    ALLOC(H->k, void, qk);
+    ALLOC(H->v, void, qk);
+  } else {
+    const size_t qk = R * cfg->heads * (size_t)g.T * g.dh * 4;
+    ALLOC(H->q, void, qk);
+    ALLOC(H->k, void, qk);
+    ALLOC(H->v, void, qk);
+  }
+  ALLOC(H->o, void, M * d * es);
+  ALLOC(H->gbuf, void, M * mlp * es);
+  ALLOC(H->status, int, 64);
+  ALLOC(H->probe_flag, int, 64);
+  const size_t xin = (size_t)cfg->max_batch * cfg->in_channels * cfg->frames * cfg->height * cfg->width;
+  const size_t xout = (size_t)cfg->max_batch * g.Cout * cfg->frames * cfg->height * cfg->width;
+  ALLOC(H->x_stage, float, xin * 4);
+  ALLOC(H->t_stage, float, (size_t)cfg->max_batch * 4);
+  ALLOC(H->y_stage, void, (size_t)cfg->max_batch * (cfg->cond_kind == DIT_COND_CLASS ? 4 : (size_t)d * 4));
+  ALLOC(H->out_stage, float, xout * 4);
+
+  // ---------------- upload
+  size_t maxn = 0;
+  {
+    const size_t cand[] = {(size_t)3 * d * d, (size_t)mlp * d, (size_t)6 * d * d};
+    for (size_t v : cand) maxn = v > maxn ? v : maxn;
+  }
+  float* staging = nullptr;
+  if (H->bf16) ALLOC(staging, float, maxn * 4);
+  int wi = 0;
+  dit_status st = DIT_OK;
+#define UP(dst, n, tobf)                                                 \
+  do {                                                                   \
+    st = upload(H, weights[wi++], (n), (dst), (tobf), staging);          \
+    if (st != DIT_OK) {                                                  \
+      dit_destroy(H);                                                    \
+      return st;                                                         \
+    }                                                                    \
+  } while (0)
+  UP(H->pe_w, (size_t)d * g.Kp, false);
+  UP(H->pe_b, (size_t)d, false);
+  UP(H->t_w1, (size_t)d * cfg->freq_dim, false);
+  UP(H->t_b1, (size_t)d, false);
+  UP(H->t_w2, (size_t)d * d, false);
+  UP(H->t_b2, (size_t)d, false);
+  if (cfg->cond_kind == DIT_COND_CLASS) UP(H->table, (size_t)(cfg->num_classes + 1) * d, false);
+  for (int i = 0; i < N; ++i) {
+    BlockW& b = H->blk[i];
+    UP(static_cast<char*>(H->ada_w) + (size_t)i * 6 * d * d * es, (size_t)6 * d * d, H->bf16);
+    UP(H->ada_b + (size_t)i * 6 * d, (size_t)6 * d, false);
+    UP(b.qkv_w, (size_t)3 * d * d, H->bf16);
+    UP(b.qkv_b, (size_t)3 * d, false);
+    if (cfg->qk_norm) {
+      UP(b.qn, (size_t)g.dh, false);
+      UP(b.kn, (size_t)g.dh, false);
+    }
+    UP(b.proj_w, (size_t)d * d, H->bf16);
+    UP(b.proj_b, (size_t)d, false);
+    UP(b.fc1_w, (size_t)mlp * d, H->bf16);
+    UP(b.fc1_b, (size_t)mlp, false);
+    UP(b.fc2_w, (size_t)d * mlp, H->bf16);
+    UP(b.fc2_b, (size_t)d, false);
+  }
+  UP(static_cast<char*>(H->ada_w) + (size_t)N * 6 * d * d * es, (size_t)2 * d * d, H->bf16);
+  UP(H->ada_b + (size_t)N * 6 * d, (size_t)2 * d, false);
+  UP(H->dec_w, (size_t)g.P * d, false);
+  UP(H->dec_b, (size_t)g.P, false);
+#undef UP
+#undef ALLOC
+
+  if (launch_pos_tables(H->pos, H->rope, g.gf, g.gh, g.gw, d, g.dh, 0) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    dit_destroy(H);
+    return DIT_ERR_CUDA;
+  }
+
+  // ---------------- tensor maps (bf16 path)
+  if (H->bf16) {
+    bool ok = make_tmap_bf16_kmajor(&H->tm_ada, H->ada_w, g.nmod, d, 128);
+    const int bns[5] = {16, 32, 64, 128, 256};
+    for (int i = 0; i < 5; ++i) ok = ok && make_tmap_bf16_kmajor(&H->tm_sc[i], H->sc, g.RPalloc, d, bns[i]);
+    ok = ok && make_tmap_bf16_kmajor(&H->tm_u, H->u, g.Mmax, d, 128);
+    ok = ok && make_tmap_bf16_kmajor(&H->tm_o, H->o, g.Mmax, d, 128);
+    ok = ok && make_tmap_bf16_kmajor(&H->tm_g, H->gbuf, g.Mmax, mlp, 128);
+    for (int i = 0; i < N && ok; ++i) {
+      BlockW& b = H->blk[i];
+      ok = make_tmap_bf16_kmajor(&b.tm_qkv, b.qkv_w, 3 * d, d, g.bn_qkv) &&
+           make_tmap_bf16_kmajor(&b.tm_proj, b.proj_w, d, d, g.bn_proj) &&
+           make_tmap_bf16_kmajor(&b.tm_fc1, b.fc1_w, mlp, d, g.bn_fc1) &&
+           make_tmap_bf16_kmajor(&b.tm_fc2, b.fc2_w, d, mlp, g.bn_fc2);
+    }
+    if (!ok) {
+      dit_destroy(H);
+      return DIT_ERR_CUDA;
+    }
+  }
+  *out = H;
+  return DIT_OK;
+}
+
+int dit_forward_launch_count(const dit_handle* H, int B, float cfg_scale) {
+  if (H == nullptr) return 0;
+  (void)B;
+  (void)cfg_scale;
+  const int per_block = 7 + ((!H->bf16 && (H->cfg.qk_norm || H->cfg.pos_kind == DIT_POS_ROPE3D)) ? 1 : 0);
+  return 3 + 1 + 1 + H->cfg.depth * per_block + 1 + 1;
+}
+
+}  // extern "C"
+
+// --------------------------------------------------------------------------- forward
+namespace {
+
+struct RunPlan {
+  int B, R, M;
+  bool guided;
+  float s;
+};
+
+dit_status check_run(dit_handle* H, const void* x, const void* t, const void* y, int B, float s, RunPlan& p) {
+  if (H == nullptr) return DIT_ERR_INVALID_ARG;
+  if (x == nullptr || t == nullptr || y == nullptr) return fail(H, DIT_ERR_INVALID_ARG, "null input pointer");
+  if (B < 1 || B > H->cfg.max_batch) return fail(H, DIT_ERR_INVALID_ARG, "batch outside [1, max_batch]");
+  if (!isfinite(s)) return fail(H, DIT_ERR_INVALID_ARG, "cfg_scale must be finite");
+  p.B = B;
+  p.guided = H->cfg.cond_kind == DIT_COND_CLASS && (s != 1.0f || H->force_guidance);
+  p.R = p.guided ? 2 * B : B;
+  p.M = p.R * H->g.T;
+  p.s = s;
+  return DIT_OK;
+}
+
+void prof_begin(dit_handle* H, int kind, cudaStream_t st) {
+  if (!H->prof) return;
+  const size_t i = H->prof_recs.size() * 2;
+  while (H->ev_pool.size() < i + 2) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return;
+    H->ev_pool.push_back(e);
+  }
+  H->prof_recs.push_back({kind, static_cast<int>(i)});
+  cudaEventRecord(H->ev_pool[i], st);
+}
+
+void prof_end(dit_handle* H, cudaStream_t st) {
+  if (!H->prof || H->prof_recs.empty()) return;
+  cudaEventRecord(H->ev_pool[H->prof_recs.back().second + 1], st);
+}
+
+#define DIT_LAUNCH(H, kind, st, call, where) \
+  do {                                      \
+    prof_begin(H, kind, st);                \
+    DIT_CK(H, call, where);                 \
+    prof_end(H, st);                        \
+  } while (0)
+
+dit_status run_condition(dit_handle* H, const float* t, const void* y, const RunPlan& p, cudaStream_t st) {
+  const dit_config& c = H->cfg;
+  CondArgs a;
+  a.t = t;
+  a.y = y;
+  a.B = p.B;
+  a.R = p.R;
+  a.d = c.hidden;
+  a.freq = c.freq_dim;
+  a.cond_kind = c.cond_kind;
+  a.num_classes = c.num_classes;
+  a.guided = p.guided;
+  a.t_scale = c.t_scale;
+  a.w1 = H->t_w1;
+  a.b1 = H->t_b1;
+  a.w2 = H->t_w2;
+  a.b2 = H->t_b2;
+  a.table = H->table;
+  a.E = H->E;
+  a.hid = H->hid;
+  a.c = H->c;
+  a.sc = H->sc;
+  a.sc_bf16 = H->bf16;
+  a.status = H->status;
+  DIT_LAUNCH(H, DIT_KERNEL_COND, st, launch_condition(a, st), "condition");
+  return DIT_OK;
+}
+
+// Runs the forward through `stop_after` blocks (depth => the whole network, with
+// the final layer when out != nullptr).
+dit_status run_forward(dit_handle* H, const float* x, const float* t, const void* y, const RunPlan& p, int stop_after,
+                       float* out, cudaStream_t st) {
+  const dit_config& c = H->cfg;
+  const Geometry& g = H->g;
+  const int d = c.hidden, mlp = c.mlp_hidden, T = g.T;
+  dit_status s = run_condition(H, t, y, p, st);
+  if (s != DIT_OK) return s;
+
+  // modulation vectors of every block and the final layer: mod[r, (6N+2) d]
+  {
+    EpiArgs ea = {};
+    ea.M = g.nmod;
+    ea.N = p.R;
+    ea.bias = H->ada_b;
+    ea.out = H->mod;
+    ea.ldo = g.nmod;
+    ea.status = H->status;
+    if (H->bf16) {
+      const int bn = adaln_bn(p.R);
+      const int idx = bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : bn == 128 ? 3 : 4;
+      DIT_LAUNCH(H, DIT_KERNEL_ADALN, st, launch_gemm_tc(EPI_ADALN, bn, &H->tm_ada, &H->tm_sc[idx], d, ea, H->num_sms, st), "adaLN gemm");
+    } else {
+      DIT_LAUNCH(H, DIT_KERNEL_ADALN, st, launch_gemm_simt(EPI_ADALN, static_cast<const float*>(H->ada_w), static_cast<const float*>(H->sc),
+                                 g.nmod, p.R, d, ea, st),
+             "adaLN gemm");
+    }
+  }
+  {
+    PatchArgs a;
+    a.x = x;
+    a.w = H->pe_w;
+    a.b = H->pe_b;
+    a.pos = H->pos;
+    a.h = H->h;
+    a.B = p.B;
+    a.R = p.R;
+    a.C = c.in_channels;
+    a.F = c.frames;
+    a.H = c.height;
+    a.W = c.width;
+    a.pt = c.patch_t;
+    a.ph = c.patch_h;
+    a.pw = c.patch_w;
+    a.d = d;
+    DIT_LAUNCH(H, DIT_KERNEL_PATCH, st, launch_patch_embed(a, st), "patch embed");
+  }
+  const int nblk = stop_after < c.depth ? stop_after : c.depth;
+  for (int i = 0; i < nblk; ++i) {
+    BlockW& b = H->blk[i];
+    const float* mb = H->mod + (size_t)i * 6 * d;
+    LnArgs ln;
+    ln.h = H->h;
+    ln.u = H->u;
+    ln.u_bf16 = H->bf16;
+    ln.ld_mod = g.nmod;
+    ln.M = p.M;
+    ln.T = T;
+    ln.d = d;
+    ln.shift = mb;
+    ln.scale = mb + d;
+    DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "ln1");
+
+    EpiArgs qa = {};
+    qa.M = p.M;
+    qa.N = 3 * d;
+    qa.bias = b.qkv_b;
+    qa.q = H->q;
+    qa.k = H->k;
+    qa.v = H->v;
+    qa.d = d;
+    qa.H = c.heads;
+    qa.dh = g.dh;
+    qa.DP = g.DP;
+    qa.Tpad = g.Tpad;
+    qa.T = T;
+    qa.qn = b.qn;
+    qa.kn = b.kn;
+    qa.rope = H->rope;
+    qa.status = H->status;
+    AttnArgs aa;
+    aa.q = H->q;
+    aa.k = H->k;
+    aa.v = H->v;
+    aa.o = H->o;
+    aa.R = p.R;
+    aa.H = c.heads;
+    aa.T = T;
+    aa.dh = g.dh;
+    aa.DP = g.DP;
+    aa.Tpad = g.Tpad;
+    aa.d = d;
+    aa.bf16 = H->bf16;
+    EpiArgs pa = {};
+    pa.M = p.M;
+    pa.N = d;
+    pa.bias = b.proj_b;
+    pa.h = H->h;
+    pa.ldh = d;
+    pa.gate = mb + 2 * d;
+    pa.ld_gate = g.nmod;
+    pa.T = T;
+    pa.status = H->status;
+    EpiArgs f1 = {};
+    f1.M = p.M;
+    f1.N = mlp;
+    f1.bias = b.fc1_b;
+    f1.out = H->gbuf;
+    f1.ldo = mlp;
+    f1.status = H->status;
+    EpiArgs f2 = pa;
+    f2.bias = b.fc2_b;
+    f2.gate = mb + 5 * d;
+
+    if (H->bf16) {
+      DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_tc(EPI_QKV, g.bn_qkv, &H->tm_u, &b.tm_qkv, d, qa, H->num_sms, st), "qkv gemm");
+      DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_simt(aa, st), "attention");
+      DIT_LAUNCH(H, DIT_KERNEL_PROJ, st, launch_gemm_tc(EPI_RESID, g.bn_proj, &H->tm_o, &b.tm_proj, d, pa, H->num_sms, st), "proj gemm");
+    } else {
+      DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_simt(EPI_QKV, static_cast<const float*>(H->u), static_cast<const float*>(b.qkv_w), p.M,
+                                 3 * d, d, qa, st),
+             "qkv gemm");
+      if (c.qk_norm || c.pos_kind == DIT_POS_ROPE3D) {
+        QkNormArgs qn;
+        qn.q = static_cast<float*>(H->q);
+        qn.k = static_cast<float*>(H->k);
+        qn.qn = b.qn;
+        qn.kn = b.kn;
+        qn.rope = H->rope;
+        qn.RH = p.R * c.heads;
+        qn.T = T;
+        qn.dh = g.dh;
+        DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_qknorm_rope_f32(qn, st), "qk norm");
+      }
+      DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_simt(aa, st), "attention");
+      DIT_LAUNCH(H, DIT_KERNEL_PROJ, st, launch_gemm_simt(EPI_RESID, static_cast<const float*>(H->o), static_cast<const float*>(b.proj_w), p.M, d,
+                                 d, pa, st),
+             "proj gemm");
+    }
+    ln.shift = mb + 3 * d;
+    ln.scale = mb + 4 * d;
+    DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "ln2");
+    if (H->bf16) {
+      DIT_LAUNCH(H, DIT_KERNEL_FC1, st, launch_gemm_tc(EPI_GELU, g.bn_fc1, &H->tm_u, &b.tm_fc1, d, f1, H->num_sms, st), "fc1 gemm");
+      DIT_LAUNCH(H, DIT_KERNEL_FC2, st, launch_gemm_tc(EPI_RESID, g.bn_fc2, &H->tm_g, &b.tm_fc2, mlp, f2, H->num_sms, st), "fc2 gemm");
+    } else {
+      DIT_LAUNCH(H, DIT_KERNEL_FC1, st, launch_gemm_simt(EPI_GELU, static_cast<const float*>(H->u), static_cast<const float*>(b.fc1_w), p.M,
+                                 mlp, d, f1, st),
+             "fc1 gemm");
+      DIT_LAUNCH(H, DIT_KERNEL_FC2, st, launch_gemm_simt(EPI_RESID, static_cast<const float*>(H->gbuf), static_cast<const float*>(b.fc2_w), p.M,
+                                 d, mlp, f2, st),
+             "fc2 gemm");
+    }
+  }
+  if (out == nullptr) return DIT_OK;
+
+  LnArgs ln;
+  ln.h = H->h;
+  ln.u = H->u;
+  ln.u_bf16 = H->bf16;
+  ln.ld_mod = g.nmod;
+  ln.M = p.M;
+  ln.T = T;
+  ln.d = d;
+  ln.shift = H->mod + (size_t)c.depth * 6 * d;
+  ln.scale = ln.shift + d;
+  DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "final ln");
+  DecodeArgs da;
+  da.u = H->u;
+  da.u_bf16 = H->bf16;
+  da.w = H->dec_w;
+  da.b = H->dec_b;
+  da.out = out;
+  da.B = p.B;
+  da.T = T;
+  da.d = d;
+  da.P = g.P;
+  da.Cout = g.Cout;
+  da.F = c.frames;
+  da.H = c.height;
+  da.W = c.width;
+  da.pt = c.patch_t;
+  da.ph = c.patch_h;
+  da.pw = c.patch_w;
+  da.guided = p.guided;
+  da.s = p.s;
+  DIT_LAUNCH(H, DIT_KERNEL_DECODE, st, launch_decode_cfg(da, st), "decode");
+  return DIT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dit_status dit_set_option(dit_handle* H, int option, int value) {
+  if (H == nullptr) return DIT_ERR_INVALID_ARG;
+  if (option == DIT_OPT_FORCE_GUIDANCE) {
+    H->force_guidance = value != 0;
+    return DIT_OK;
+  }
+  if (option == DIT_OPT_USE_GRAPH) {
+    H->use_graph = value != 0;
+    return DIT_OK;
+  }
+  return fail(H, DIT_ERR_INVALID_ARG, "unknown option");
+}
+
+dit_status dit_forward(dit_handle* H, const float* x, const float* t, const void* y, int B, float cfg_scale, float* out,
+                       dit_stream_t stream) {
+  RunPlan p;
+  dit_status s = check_run(H, x, t, y, B, cfg_scale, p);
+  if (s != DIT_OK) return s;
+  if (out == nullptr) return fail(H, DIT_ERR_INVALID_ARG, "null output pointer");
+  return run_forward(H, x, t, y, p, H->cfg.depth, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dit_status dit_forward_host(dit_handle* H, const float* x, const float* t, const void* y, int B, float cfg_scale,
+                            float* out, dit_stream_t stream) {
+  RunPlan p;
+  dit_status s = check_run(H, x, t, y, B, cfg_scale, p);
+  if (s != DIT_OK) return s;
+  if (out == nullptr) return fail(H, DIT_ERR_INVALID_ARG, "null output pointer");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const dit_config& c = H->cfg;
+  const size_t xin = (size_t)B * c.in_channels * c.frames * c.height * c.width;
+  const size_t xout = (size_t)B * H->g.Cout * c.frames * c.height * c.width;
+  const size_t ybytes = (size_t)B * (c.cond_kind == DIT_COND_CLASS ? 4 : (size_t)c.hidden * 4);
+  DIT_CK(H, cudaMemcpyAsync(H->x_stage, x, xin * 4, cudaMemcpyHostToDevice, st), "x upload");
+  DIT_CK(H, cudaMemcpyAsync(H->t_stage, t, (size_t)B * 4, cudaMemcpyHostToDevice, st), "t upload");
+  DIT_CK(H, cudaMemcpyAsync(H->y_stage, y, ybytes, cudaMemcpyHostToDevice, st), "y upload");
+  s = run_forward(H, H->x_stage, H->t_stage, H->y_stage, p, c.depth, H->out_stage, st);
+  if (s != DIT_OK) return s;
+  DIT_CK(H, cudaMemcpyAsync(out, H->out_stage, xout * 4, cudaMemcpyDeviceToHost, st), "out download");
+  DIT_CK(H, cudaStreamSynchronize(st), "stream sync");
+  return DIT_OK;
+}
+
+dit_status dit_debug_residual(dit_handle* H, const float* x, const float* t, const void* y, int B, float cfg_scale,
+                              int after_block, float* h_out, dit_stream_t stream) {
+  RunPlan p;
+  dit_status s = check_run(H, x, t, y, B, cfg_scale, p);
+  if (s != DIT_OK) return s;
+  if (h_out == nullptr || after_block < 0 || after_block > H->cfg.depth)
+    return fail(H, DIT_ERR_INVALID_ARG, "bad residual request");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = run_forward(H, x, t, y, p, after_block, nullptr, st);
+  if (s != DIT_OK) return s;
+  DIT_CK(H, cudaMemcpyAsync(h_out, H->h, (size_t)p.M * H->cfg.hidden * 4, cudaMemcpyDeviceToDevice, st), "copy h");
+  return DIT_OK;
+}
+
+dit_status dit_debug_condition(dit_handle* H, const float* t, const void* y, int B, float cfg_scale, float* c_out,
+                               dit_stream_t stream) {
+  RunPlan p;
+  dit_status s = check_run(H, t, t, y, B, cfg_scale, p);
+  if (s != DIT_OK) return s;
+  if (c_out == nullptr) return fail(H, DIT_ERR_INVALID_ARG, "null output pointer");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = run_condition(H, t, y, p, st);
+  if (s != DIT_OK) return s;
+  DIT_CK(H, cudaMemcpyAsync(c_out, H->c, (size_t)p.R * H->cfg.hidden * 4, cudaMemcpyDeviceToDevice, st), "copy c");
+  return DIT_OK;
+}
+
+dit_status dit_sync_status(dit_handle* H) {
+  if (H == nullptr) return DIT_ERR_INVALID_ARG;
+  DIT_CK(H, cudaDeviceSynchronize(), "sync");
+  int v = 0;
+  DIT_CK(H, cudaMemcpy(&v, H->status, 4, cudaMemcpyDeviceToHost), "status read");
+  DIT_CK(H, cudaMemset(H->status, 0, 4), "status clear");
+  return static_cast<dit_status>(v);
+}
+
+dit_status dit_debug_wait_probe(dit_handle* H, int timeout_us, dit_stream_t stream) {
+  if (H == nullptr || timeout_us < 0) return DIT_ERR_INVALID_ARG;
+  DIT_CK(H, launch_wait_probe(H->probe_flag, H->status, (long long)timeout_us * 1000LL,
+                              reinterpret_cast<cudaStream_t>(stream)),
+         "wait probe");
+  return DIT_OK;
+}
+
+dit_status dit_profile_enable(dit_handle* H, int enable) {
+  if (H == nullptr) return DIT_ERR_INVALID_ARG;
+  H->prof = enable != 0;
+  return DIT_OK;
+}
+
+dit_status dit_profile_read(dit_handle* H, float* total_ms, int* launches) {
+  if (H == nullptr || total_ms == nullptr || launches == nullptr) return DIT_ERR_INVALID_ARG;
+  DIT_CK(H, cudaDeviceSynchronize(), "sync");
+  for (int k = 0; k < DIT_KERNEL_COUNT; ++k) {
+    total_ms[k] = 0.f;
+    launches[k] = 0;
+  }
+  for (const auto& r : H->prof_recs) {
+    float ms = 0.f;
+    DIT_CK(H, cudaEventElapsedTime(&ms, H->ev_pool[r.second], H->ev_pool[r.second + 1]), "event time");
+    if (r.first >= 0 && r.first < DIT_KERNEL_COUNT) {
+      total_ms[r.first] += ms;
+      launches[r.first] += 1;
+    }
+  }
+  H->prof_recs.clear();
+  return DIT_OK;
+}
+
+dit_status dit_op_linear_bf16(const uint16_t* x, const uint16_t* w, const float* b, float* y, int M, int N, int K,
+                              int block_n, dit_stream_t stream) {
+  if (x == nullptr || w == nullptr || y == nullptr || M < 0 || N <= 0 || K <= 0 || (K % 8) != 0)
+    return DIT_ERR_INVALID_ARG;
+  if (!gemm_tc_supported_bn(block_n)) return DIT_ERR_INVALID_ARG;
+  if (M == 0) return DIT_OK;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return DIT_ERR_NO_DEVICE;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16_kmajor(&ta, x, M, K, 128) || !make_tmap_bf16_kmajor(&tb, w, N, K, block_n))
+    return DIT_ERR_INVALID_ARG;
+  EpiArgs ea = {};
+  ea.M = M;
+  ea.N = N;
+  ea.bias = b;
+  ea.out = y;
+  ea.ldo = N;
+  if (launch_gemm_tc(EPI_F32, block_n, &ta, &tb, K, ea, sms, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DIT_ERR_CUDA;
+  return DIT_OK;
+}
+
+}  // extern "C"

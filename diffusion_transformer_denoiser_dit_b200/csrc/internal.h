@@ -1,0 +1,124 @@
+// Internal launch interfaces between the C-ABI layer (dit_api.cu) and the kernel
+// translation units.  Plain structs of device pointers and sizes.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dit {
+
+// ------------------------------------------------------------------ GEMM epilogues
+enum Epi : int {
+  EPI_F32 = 0,    // out[m, n] = acc + bias[n]                              (float32)
+  EPI_ADALN = 1,  // out[n, m] = acc + bias[m]   (A = modulation weights, B = SiLU(c) rows)
+  EPI_GELU = 2,   // out[m, n] = gelu_tanh(acc + bias[n])                   (bf16 / f32)
+  EPI_RESID = 3,  // h[m, n]  += gate[row(m), n] * (acc + bias[n])          (float32 RMW)
+  EPI_QKV = 4,    // scatter to q, k, v head-major (+ QK-RMSNorm, 3D RoPE)
+};
+
+struct EpiArgs {
+  int M, N;             // logical output extent (rows of A, rows of B)
+  const float* bias;    // [N], or [M] for EPI_ADALN
+  void* out;            // EPI_F32 / EPI_ADALN / EPI_GELU destination
+  int ldo;              // its row stride in elements
+  // EPI_RESID
+  float* h;             // residual stream [M, ldh]
+  int ldh;
+  const float* gate;    // gate vector of row r at gate + r * ld_gate
+  int ld_gate;
+  int T;                // tokens per sample (row(m) = m / T)
+  // EPI_QKV
+  void* q;              // bf16 [R*H, Tpad, DP]  (f32 path: [R*H, T, dh])
+  void* k;
+  void* v;              // bf16 transposed [R*H, DP, Tpad] (f32 path: [R*H, T, dh])
+  int d, H, dh, DP, Tpad;
+  const float* qn;      // [dh] RMSNorm gains or nullptr
+  const float* kn;
+  const float* rope;    // [T, dh/2, 2] (cos, sin) or nullptr
+  int* status;
+};
+
+// tensor-core GEMM D[M, N] = A[M, K] B[N, K]^T with A, B bf16 K-major.
+// Returns cudaSuccess or the launch error.
+cudaError_t launch_gemm_tc(int epi, int block_n, const CUtensorMap* tmA, const CUtensorMap* tmB, int K,
+                           const EpiArgs& ea, int num_sms, cudaStream_t st);
+int gemm_tc_supported_bn(int block_n);
+// Build a 2-D bf16 K-major tensor map: rows x K, box = box_rows x 64, 128-byte swizzle.
+bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
+
+// float32 SIMT GEMM with the same epilogues (f32 outputs everywhere).
+cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, int M, int N, int K, const EpiArgs& ea,
+                             cudaStream_t st);
+
+// ------------------------------------------------------------------ small steps
+struct CondArgs {
+  const float* t;        // [B]
+  const void* y;         // int32 [B] or float32 [B, d]
+  int B, R, d, freq, cond_kind, num_classes, guided;
+  float t_scale;
+  const float *w1, *b1, *w2, *b2, *table;
+  float* E;              // scratch [R, freq]
+  float* hid;            // scratch [R, d]
+  float* c;              // [R, d]   (optional, may be null)
+  void* sc;              // SiLU(c): bf16 [*, d] or f32 [R, d]
+  int sc_bf16;
+  int* status;
+};
+cudaError_t launch_condition(const CondArgs& a, cudaStream_t st);
+
+struct PatchArgs {
+  const float* x;        // [B, C, F, H, W]
+  const float* w;        // [d, Kp]
+  const float* b;        // [d]
+  const float* pos;      // [T, d] or nullptr
+  float* h;              // [R*T, d]
+  int B, R, C, F, H, W, pt, ph, pw, d;
+};
+cudaError_t launch_patch_embed(const PatchArgs& a, cudaStream_t st);
+
+struct LnArgs {
+  const float* h;        // [M, d]
+  void* u;               // bf16 or f32 [M, d]
+  int u_bf16;
+  const float* shift;    // row r vector at shift + r * ld_mod
+  const float* scale;
+  int ld_mod;
+  int M, T, d;
+};
+cudaError_t launch_ln_modulate(const LnArgs& a, cudaStream_t st);
+
+struct AttnArgs {
+  const void *q, *k, *v;  // layouts as in EpiArgs (bf16 head-major padded or f32 head-major)
+  void* o;                // [R*T, d] bf16 or f32, token-major
+  int R, H, T, dh, DP, Tpad, d;
+  int bf16;               // 1: bf16 padded layouts, V transposed
+};
+cudaError_t launch_attention_simt(const AttnArgs& a, cudaStream_t st);
+cudaError_t launch_attention_tc(const AttnArgs& a, const CUtensorMap* tq_main, const CUtensorMap* tq_tail,
+                                const CUtensorMap* tk_main, const CUtensorMap* tk_tail, const CUtensorMap* tv,
+                                int* status, cudaStream_t st);
+
+struct QkNormArgs {   // f32 path: RMSNorm + RoPE applied in place to q, k [R*H, T, dh]
+  float *q, *k;
+  const float *qn, *kn, *rope;
+  int RH, T, dh;
+};
+cudaError_t launch_qknorm_rope_f32(const QkNormArgs& a, cudaStream_t st);
+
+struct DecodeArgs {
+  const void* u;         // [R*T, d] bf16 or f32
+  int u_bf16;
+  const float* w;        // [P, d]
+  const float* b;        // [P]
+  float* out;            // [B, Cout, F, H, W]
+  int B, T, d, P, Cout, F, H, W, pt, ph, pw, guided;
+  float s;
+};
+cudaError_t launch_decode_cfg(const DecodeArgs& a, cudaStream_t st);
+
+cudaError_t launch_pos_tables(float* pos, float* rope, int gf, int gh, int gw, int d, int dh, cudaStream_t st);
+cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaStream_t st);
+cudaError_t launch_wait_probe(int* flag, int* status, long long limit_ns, cudaStream_t st);
+
+}  // namespace dit

@@ -1,0 +1,217 @@
+/*
+ * dit.h — C ABI of the B200 (sm_100a) DiT denoiser forward library.
+ *
+ * The library computes one evaluation of the Diffusion Transformer denoiser
+ * (the noise / covariance or velocity predictor of a latent diffusion or
+ * rectified-flow model) on one GPU:
+ *
+ *   patchify + linear embed (+ 2D sin-cos positions)            "확산 트랜스포머"
+ *     (itwiki.kr), section "잠재 공간과 패치화": T = (I/p)^2 tokens of width d;
+ *   c = MLP(sinusoid(t)) + e(y)                                  same page, "adaLN-Zero":
+ *     c is the sum of the timestep and class embeddings (or a pooled text vector);
+ *   N blocks of  x += a1 * Attn(LN(x)(1+g1)+b1),  x += a2 * FFN(LN(x)(1+g2)+b2)
+ *     with (b1,g1,a1,b2,g2,a2) = Linear(SiLU(c))                 same page, "adaLN-Zero";
+ *   final modulated LN, linear decoder to p x p x 2C per token, unpatchify
+ *                                                                "Sora / DiT" (cv-learn.com),
+ *     "방법 및 아키텍처"; itwiki page, "잠재 공간과 패치화";
+ *   classifier-free guidance  e = e(null) + s (e(c) - e(null))   "Sora / DiT", guidance bullet;
+ *   video variant: spacetime patches, QK-RMSNorm and 3D RoPE, velocity head
+ *                                                                "GOKU : Flow Based Video
+ *     Generative Foundation Models" (blog.outta.ai), sections 2.2 and 2.3.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named "dev" are CUDA device pointers on the current device; "host"
+ *     pointers are ordinary (preferably pinned) host memory.
+ *   - All floating-point I/O is float32 (IEEE binary32); labels are int32.
+ *   - Work is enqueued on the given cudaStream_t (0 = legacy default stream) and
+ *     the call returns without waiting unless stated otherwise.
+ *   - A dit_status is returned; DIT_OK (0) means the work was enqueued.  Errors
+ *     found on the host return before anything is launched.  Errors found on
+ *     the device (a label outside [0, num_classes], a bounded wait that ran out)
+ *     are recorded in a per-handle device status word, read by dit_sync_status.
+ *   - No entry point traps, aborts or waits without a bound.
+ */
+#ifndef DIT_B200_H
+#define DIT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dit_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  DIT_OK = 0,
+  DIT_ERR_INVALID_ARG = 1,    /* null pointer, bad size, batch > max_batch, bad weight count */
+  DIT_ERR_UNSUPPORTED = 2,    /* shape the kernels do not cover (e.g. head dim not 64 or 72) */
+  DIT_ERR_OOM = 3,            /* device allocation failed in dit_create */
+  DIT_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed */
+  DIT_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait gave up (device status word) */
+  DIT_ERR_BAD_LABEL = 6,      /* a class label outside [0, num_classes]; it was clamped */
+  DIT_ERR_NO_DEVICE = 7       /* no sm_100 device is current */
+} dit_status;
+
+enum { DIT_DTYPE_F32 = 0, DIT_DTYPE_BF16 = 1 };
+enum { DIT_POS_SINCOS2D = 0, DIT_POS_ROPE3D = 1 };
+enum { DIT_COND_CLASS = 0, DIT_COND_VECTOR = 1 };
+
+/* Model and workload description.  Image models use frames = patch_t = 1. */
+typedef struct dit_config {
+  int dtype;          /* DIT_DTYPE_F32: float32 SIMT kernels; DIT_DTYPE_BF16: bf16 operands on
+                         tcgen05 tensor cores with float32 accumulation, statistics and residual */
+  int in_channels;    /* C of the latent (4 for the image models, 16 for the video model) */
+  int frames, height, width;       /* latent extent F, H, W */
+  int patch_t, patch_h, patch_w;   /* patch extent; each must divide the latent extent */
+  int hidden;         /* d */
+  int depth;          /* N blocks */
+  int heads;          /* attention heads; head dim d/heads must be 64 or 72 */
+  int mlp_hidden;     /* FFN width (4d in every DiT size) */
+  int learn_sigma;    /* 1: decoder emits 2C channels (noise + diagonal covariance); 0: C */
+  int pos_kind;       /* DIT_POS_SINCOS2D (added to tokens) or DIT_POS_ROPE3D (rotates q, k) */
+  int qk_norm;        /* 1: RMSNorm with learnable gain on q and k of each head */
+  int cond_kind;      /* DIT_COND_CLASS: label table of num_classes+1 rows (last = null);
+                         DIT_COND_VECTOR: caller passes a float32 vector of width d per sample */
+  int num_classes;    /* 1000 for ImageNet; the null label is num_classes */
+  int freq_dim;       /* width of the timestep sinusoid (256) */
+  int max_batch;      /* largest user batch B; device workspace is sized for 2*max_batch rows */
+  float t_scale;      /* the sinusoid sees t * t_scale (1 for integer steps, 1000 for t in [0,1)) */
+} dit_config;
+
+typedef struct dit_handle dit_handle;
+
+/*
+ * dit_create — validate the configuration, allocate device weights and workspace,
+ * upload and convert the weights.
+ *
+ * weights: n_weights host float32 arrays in this fixed order (linear weights are
+ * row-major [out, in]; K_p = C*patch_t*patch_h*patch_w; P = patch_t*patch_h*patch_w*C_out):
+ *   pe.w [d, K_p] (patch vector order c, i_t, i_h, i_w — a flattened Conv weight), pe.b [d],
+ *   t.w1 [d, freq_dim], t.b1 [d], t.w2 [d, d], t.b2 [d],
+ *   y.table [num_classes+1, d]                          (DIT_COND_CLASS only),
+ *   for each block: ada.w [6d, d], ada.b [6d], qkv.w [3d, d], qkv.b [3d],
+ *                   q_norm.g [d/heads], k_norm.g [d/heads]   (qk_norm only),
+ *                   proj.w [d, d], proj.b [d], fc1.w [mlp, d], fc1.b [mlp],
+ *                   fc2.w [d, mlp], fc2.b [d],
+ *   final.ada.w [2d, d], final.ada.b [2d], dec.w [P, d], dec.b [P].
+ * The ada.w output rows are ordered (shift1, scale1, gate1, shift2, scale2, gate2),
+ * the final ones (shift, scale); qkv.w rows are [q | k | v], heads contiguous.
+ * The library copies everything; the caller may free the host arrays on return.
+ * Blocks the calling thread until the upload is complete.
+ * Returns DIT_ERR_INVALID_ARG / DIT_ERR_UNSUPPORTED before any CUDA call when the
+ * configuration is rejected, DIT_ERR_NO_DEVICE without an sm_100 device, DIT_ERR_OOM
+ * when device memory runs out.  *out is set only on DIT_OK.
+ */
+dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_weights,
+                      dit_handle** out);
+
+/* Number of weight arrays dit_create expects for cfg (0 if cfg is invalid). */
+int dit_weight_count(const dit_config* cfg);
+
+/*
+ * dit_forward — one denoiser evaluation, enqueued on stream.
+ *   x   dev float32 [B, C, H, W] (images) or [B, C, F, H, W] (video), NC(F)HW
+ *   t   dev float32 [B] timesteps
+ *   y   dev int32 [B] class labels (DIT_COND_CLASS) or float32 [B, d] (DIT_COND_VECTOR)
+ *   out dev float32 [B, C_out, (F,) H, W]
+ * Guidance: with a class-conditional model and cfg_scale != 1 the library runs 2B
+ * rows, [x; x] with labels [y; num_classes], and writes e(null) + s (e(y) - e(null)).
+ * Otherwise it runs B rows and writes e(y).  1 <= B <= max_batch.
+ * One forward may be in flight per handle (the handle owns one workspace); the
+ * handle is not thread-safe.  Buffers must stay valid until the stream reaches
+ * the end of the call.
+ */
+dit_status dit_forward(dit_handle* h, const float* x, const float* t, const void* y, int B,
+                       float cfg_scale, float* out, dit_stream_t stream);
+
+/*
+ * dit_forward_host — dit_forward on host buffers: copies x, t, y into the handle's
+ * device staging area, runs the forward on stream, copies out back and waits for
+ * the stream.  Same layouts and rules as dit_forward.
+ */
+dit_status dit_forward_host(dit_handle* h, const float* x_host, const float* t_host,
+                            const void* y_host, int B, float cfg_scale, float* out_host,
+                            dit_stream_t stream);
+
+/* Reads and clears the handle's device status word (synchronises the device first).
+   Returns DIT_OK or the first device-side error recorded since the last call. */
+dit_status dit_sync_status(dit_handle* h);
+
+/* Text of the last host-side error on this handle (never NULL). */
+const char* dit_last_error(const dit_handle* h);
+
+/* Short name of a status code (never NULL). */
+const char* dit_status_string(dit_status s);
+
+/* Frees every device allocation of the handle.  Waits for outstanding work. */
+void dit_destroy(dit_handle* h);
+
+/* ------------------------------------------------------------------------------ */
+/* Diagnostics.  Same device-pointer and stream rules as dit_forward.             */
+/* ------------------------------------------------------------------------------ */
+
+/* Option switches (test use).  DIT_OPT_FORCE_GUIDANCE = 1 makes dit_forward run the
+   2B guided rows even at cfg_scale == 1 (so e(null) + 1*(e(y)-e(null)) is returned).
+   DIT_OPT_USE_GRAPH = 0/1 disables / enables CUDA-graph replay of the forward. */
+enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2 };
+dit_status dit_set_option(dit_handle* h, int option, int value);
+
+/*
+ * dit_debug_residual — run the forward up to and including block `after_block`
+ * (0 = right after patch embedding) and copy the float32 residual stream
+ * [rows, T, d] into h_out (dev), rows ordered [cond; uncond] when guided.
+ * The final layer is not run.  Same guidance rule as dit_forward.
+ */
+dit_status dit_debug_residual(dit_handle* h, const float* x, const float* t, const void* y, int B,
+                              float cfg_scale, int after_block, float* h_out, dit_stream_t stream);
+
+/*
+ * dit_debug_condition — compute the condition vector c [rows, d] (float32, dev)
+ * from t and y exactly as dit_forward does (rows = 2B when guided).
+ */
+dit_status dit_debug_condition(dit_handle* h, const float* t, const void* y, int B, float cfg_scale,
+                               float* c_out, dit_stream_t stream);
+
+/*
+ * dit_debug_wait_probe — launch one kernel that waits on a device flag nothing ever
+ * sets, with the library's bounded-wait routine and a limit of timeout_us
+ * microseconds.  When the limit runs out the kernel records DIT_ERR_DEVICE_TIMEOUT
+ * in the status word and returns, so dit_sync_status reports it and the context
+ * stays usable.  Exercises the device-side failure path without faulting a GPU.
+ */
+dit_status dit_debug_wait_probe(dit_handle* h, int timeout_us, dit_stream_t stream);
+
+/*
+ * dit_op_linear_bf16 — the tensor-core GEMM building block on its own:
+ *   y[M, N] = x[M, K] W[N, K]^T + b[N]
+ * x, W: dev bf16 (raw uint16 bit patterns), row-major, K % 8 == 0, 16-byte aligned;
+ * b: dev float32 [N] or NULL; y: dev float32 [M, N].  block_n selects the tile
+ * width (16, 32, 64, 128, 144 or 256).  Uses tcgen05.mma with TMA-fed shared
+ * memory and a TMEM accumulator; float32 accumulation.
+ */
+dit_status dit_op_linear_bf16(const uint16_t* x, const uint16_t* w, const float* b, float* y,
+                              int M, int N, int K, int block_n, dit_stream_t stream);
+
+/*
+ * Per-step kernel timing.  While enabled, dit_forward brackets each launch with a pair
+ * of CUDA events on its stream and files the pair under one of the DIT_KERNEL_* kinds.
+ * dit_profile_read synchronises the device, writes per-kind total milliseconds and
+ * launch counts (arrays of at least DIT_KERNEL_COUNT entries) and clears the record.
+ */
+enum { DIT_KERNEL_COND = 0, DIT_KERNEL_ADALN = 1, DIT_KERNEL_PATCH = 2, DIT_KERNEL_LN = 3, DIT_KERNEL_QKV = 4,
+       DIT_KERNEL_ATTN = 5, DIT_KERNEL_PROJ = 6, DIT_KERNEL_FC1 = 7, DIT_KERNEL_FC2 = 8, DIT_KERNEL_DECODE = 9,
+       DIT_KERNEL_COUNT = 10 };
+dit_status dit_profile_enable(dit_handle* h, int enable);
+dit_status dit_profile_read(dit_handle* h, float* total_ms, int* launches);
+
+/* Number of kernel launches one dit_forward enqueues for batch B (graph nodes if a
+   graph is replayed). */
+int dit_forward_launch_count(const dit_handle* h, int B, float cfg_scale);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT_B200_H */

@@ -1,0 +1,229 @@
+"""CUDA path vs the CPU oracle, through the C ABI (GPU only).
+
+Tolerances (from the workload definition): float32 path relative L2 <= 1e-4;
+bf16 path relative L2 <= 2e-2 and max|gpu - oracle| / std(oracle) <= 5e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dit_synth as S
+from diffusion_transformer_denoiser_dit_b200 import binding
+from diffusion_transformer_denoiser_dit_b200.binding import DiT
+from oracle import dit_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+F32_REL = 1e-4
+BF16_REL = 2e-2
+BF16_MAXN = 5e-2
+
+
+def metrics(got, want):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    maxn = np.abs(got - want).max() / want.std()
+    return rel, maxn
+
+
+def assert_parity(cfg, got, want, what=""):
+    assert got.shape == want.shape, (got.shape, want.shape)
+    assert np.all(np.isfinite(got)), what
+    rel, maxn = metrics(got, want)
+    if cfg.dtype == S.DTYPE_F32:
+        assert rel <= F32_REL, (what, rel, maxn)
+    else:
+        assert rel <= BF16_REL and maxn <= BF16_MAXN, (what, rel, maxn)
+    return rel, maxn
+
+
+def dev(inp):
+    return {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in inp.items()}
+
+
+# ----------------------------------------------------------------------------- configs
+def small_video_f32():
+    return S.VIDEO_RF.with_(dtype=S.DTYPE_F32, hidden=144, heads=2, mlp_hidden=576, depth=2, in_channels=4, frames=3,
+                            height=8, width=6, batch=2, index=-1)
+
+
+def small_image_bf16_dh72():   # T = 225 (ragged), 6 rows with guidance, M = 1350
+    return S.DIT_XL2_CFG256.with_(hidden=288, heads=4, mlp_hidden=1152, depth=2, height=30, width=30, batch=3,
+                                  index=-1)
+
+
+def small_image_bf16_dh64():   # T = 64, M = 320, no guidance
+    return S.DIT_B4_BF16.with_(hidden=256, heads=4, mlp_hidden=1024, depth=2, batch=5, index=-1)
+
+
+def small_video_bf16():        # T = 48, QK-RMSNorm + 3D RoPE
+    return S.VIDEO_RF.with_(hidden=288, heads=4, mlp_hidden=1152, depth=2, in_channels=4, frames=3, height=8, width=8,
+                            batch=2, index=-1)
+
+
+SMALL = {
+    "s8_f32": lambda: S.DIT_S8_F32,
+    "video_f32": small_video_f32,
+    "img_bf16_dh72": small_image_bf16_dh72,
+    "img_bf16_dh64": small_image_bf16_dh64,
+    "video_bf16": small_video_bf16,
+    "b4_bf16_full": lambda: S.DIT_B4_BF16,
+}
+
+
+# ----------------------------------------------------------------------------- GEMM building block
+@pytest.mark.parametrize("M,N,K,bn", [
+    (128, 128, 64, 128), (300, 144, 1152, 144), (77, 50, 72, 64), (1000, 192, 200, 192),
+    (513, 256, 4608, 256), (64, 16, 1152, 16), (200, 32, 1152, 32), (8192, 3456, 1152, 144),
+])
+def test_tcgen05_linear_matches_definition(M, N, K, bn):
+    g = torch.Generator(device="cuda").manual_seed(M * 7 + N)
+    x = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    w = torch.randn(N, K, device="cuda", generator=g).to(torch.bfloat16)
+    b = torch.randn(N, device="cuda", generator=g)
+    y = binding.linear_bf16(x, w, b, block_n=bn)
+    torch.cuda.synchronize()
+    ref = x.double().cpu().numpy() @ w.double().cpu().numpy().T + b.double().cpu().numpy()
+    err = np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, err
+
+
+# ----------------------------------------------------------------------------- end to end
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("gates", ["random", "strong"])
+def test_forward_parity(name, gates):
+    cfg = SMALL[name]()
+    W = S.make_weights(cfg)
+    if gates == "strong":
+        W = S.set_adaln(cfg, W, gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    want = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    m = DiT(cfg, W)
+    d = dev(inp)
+    got = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale)
+    assert m.sync_status() == binding.DIT_OK
+    assert_parity(cfg, got.cpu().numpy(), want, name)
+    m.close()
+
+
+@pytest.mark.parametrize("name", ["s8_f32", "img_bf16_dh72", "video_bf16", "video_f32"])
+def test_residual_stream_parity_per_block(name):
+    cfg = SMALL[name]()
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    for k in range(cfg.depth + 1):
+        got = m.debug_residual(d["x"], d["t"], d["y"], cfg.cfg_scale, k).cpu().numpy()
+        want = O.forward(cfg, W, inp["x"], inp["t"], inp["y"], stop_after_block=k)
+        assert_parity(cfg, got, want, f"{name} after block {k}")
+    m.close()
+
+
+def test_condition_vector_parity():
+    cfg = small_image_bf16_dh72()
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    c = m.debug_condition(d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    yy = np.concatenate([inp["y"], np.full(cfg.batch, cfg.num_classes)])
+    tt = np.concatenate([inp["t"], inp["t"]])
+    want = O.condition(cfg, S.weight_dict(cfg, W), tt, yy)
+    assert np.abs(c - want).max() / np.abs(want).max() < 1e-5
+    m.close()
+
+
+def test_zero_adaln_blocks_are_identity_on_gpu():
+    cfg = small_image_bf16_dh72()
+    W = S.set_adaln(cfg, S.make_weights(cfg), zero=True)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    h0 = m.debug_residual(d["x"], d["t"], d["y"], cfg.cfg_scale, 0).cpu()
+    hN = m.debug_residual(d["x"], d["t"], d["y"], cfg.cfg_scale, cfg.depth).cpu()
+    assert torch.equal(h0, hN)
+    m.close()
+
+
+def test_guidance_special_cases_on_gpu():
+    cfg = small_image_bf16_dh72()
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    null = torch.full_like(d["y"], cfg.num_classes)
+    cond = m.forward(d["x"], d["t"], d["y"], 1.0).cpu().numpy()
+    uncond = m.forward(d["x"], d["t"], null, 1.0).cpu().numpy()
+    s0 = m.forward(d["x"], d["t"], d["y"], 0.0).cpu().numpy()
+    s15 = m.forward(d["x"], d["t"], d["y"], 1.5).cpu().numpy()
+    assert metrics(s0, uncond)[0] < 1e-5
+    assert metrics(s15, uncond + 1.5 * (cond - uncond))[0] < 1e-4
+    m.set_option(binding.DIT_OPT_FORCE_GUIDANCE, 1)
+    s1 = m.forward(d["x"], d["t"], d["y"], 1.0).cpu().numpy()
+    assert metrics(s1, cond)[0] < 1e-5
+    m.close()
+
+
+def test_host_entry_point_matches_device_entry_point():
+    cfg = small_image_bf16_dh64()
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    a = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    b = m.forward_host(inp["x"], inp["t"], inp["y"], cfg.cfg_scale)
+    assert np.array_equal(a, b)
+    m.close()
+
+
+def test_batch_smaller_than_max_and_rows_independent():
+    cfg = small_image_bf16_dh72()
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W, max_batch=cfg.batch)
+    d = dev(inp)
+    full = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    one = m.forward(d["x"][1:2].contiguous(), d["t"][1:2].contiguous(), d["y"][1:2].contiguous(),
+                    cfg.cfg_scale).cpu().numpy()
+    assert metrics(one[0], full[1])[0] < 1e-5
+    m.close()
+
+
+def test_bad_label_is_reported_and_clamped():
+    cfg = small_image_bf16_dh64()
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    inp["y"][0] = 5000
+    m = DiT(cfg, W)
+    d = dev(inp)
+    out = m.forward(d["x"], d["t"], d["y"], 1.0)
+    assert m.sync_status() == binding.DIT_ERR_BAD_LABEL
+    assert torch.isfinite(out).all()
+    assert m.sync_status() == binding.DIT_OK   # cleared by the read
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    cfg = small_image_bf16_dh64()
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    m.wait_probe(2000)   # 2 ms on a flag nothing sets
+    assert m.sync_status() == binding.DIT_ERR_DEVICE_TIMEOUT
+    d = dev(inp)
+    out = m.forward(d["x"], d["t"], d["y"], 1.0)
+    assert m.sync_status() == binding.DIT_OK
+    want = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    assert_parity(cfg, out.cpu().numpy(), want, "after timeout")
+    m.close()
+
+
+def test_host_side_errors_launch_nothing():
+    cfg = small_image_bf16_dh64()
+    m = DiT(cfg, S.make_weights(cfg))
+    d = dev(S.make_inputs(cfg, batch=cfg.batch + 1))
+    with pytest.raises(binding.DitError) as e:
+        m.forward(d["x"], d["t"], d["y"], 1.0)
+    assert e.value.code == binding.DIT_ERR_INVALID_ARG
+    m.close()
