@@ -24,7 +24,7 @@ EXPORTS = [
     "dit_create", "dit_weight_count", "dit_forward", "dit_forward_host", "dit_sync_status", "dit_last_error",
     "dit_status_string", "dit_destroy", "dit_set_option", "dit_debug_residual", "dit_debug_condition",
     "dit_debug_wait_probe", "dit_op_linear_bf16", "dit_forward_launch_count", "dit_profile_enable",
-    "dit_profile_read",
+    "dit_profile_read", "dit_condition_static",
 ]
 
 KERNEL_KINDS = ["cond", "adaln", "patch", "ln", "qkv", "attn", "proj", "fc1", "fc2", "decode"]
@@ -73,6 +73,8 @@ def load() -> ctypes.CDLL:
         "dit_forward_launch_count": (c_int, [P, c_int, c_float]),
         "dit_profile_enable": (c_int, [P, c_int]),
         "dit_profile_read": (c_int, [P, POINTER(c_float), POINTER(c_int)]),
+        "dit_condition_static": (c_int, [P, P, c_int, c_int, P, P, P, P, P, c_int, c_int, c_int, c_int, c_float,
+                                         P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -206,6 +206,35 @@ enum { DIT_KERNEL_COND = 0, DIT_KERNEL_ADALN = 1, DIT_KERNEL_PATCH = 2, DIT_KERN
 dit_status dit_profile_enable(dit_handle* h, int enable);
 dit_status dit_profile_read(dit_handle* h, float* total_ms, int* launches);
 
+/*
+ * dit_condition_static — the condition vector c [rows, hidden] (rows = 2B when
+ * guided, else B), computed like dit_forward computes it, for callers that cannot
+ * allocate device memory (code that runs where cudaMalloc is forbidden or would
+ * deadlock, such as inside a caching allocator's own callbacks, or programs that
+ * must fix their whole device footprint before they start).  No handle is needed and
+ * nothing is allocated: every input, weight and output is the caller's, and the
+ * intermediate buffers live in one fixed device array inside the library.
+ * The pages have no counterpart of this entry point; it is a library service.
+ *   t [B] f32, y int32 [B] (cond_kind DIT_COND_CLASS) or f32 [B, hidden] (DIT_COND_VECTOR),
+ *   w1 [hidden, freq_dim], b1 [hidden], w2 [hidden, hidden], b2 [hidden],
+ *   table [num_classes+1, hidden] (class models; NULL otherwise), all dev float32;
+ *   guided = 1 appends B rows with the null label (class models only);
+ *   c_out dev f32 [rows, hidden]; status dev int32 (or NULL) receives DIT_ERR_BAD_LABEL
+ *   when a label lies outside [0, num_classes] (the label is clamped).
+ * Limits of the fixed scratch: rows <= 128, freq_dim <= 512, hidden <= 1536; larger
+ * requests return DIT_ERR_INVALID_ARG before anything is launched.  The array
+ * (1.75 MiB) stays resident on every GPU that loaded the library until the process
+ * exits.  The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents; every call
+ * rewrites what it reads, so nothing has to start at zero, but calls whose work
+ * overlaps on the GPU (different streams, or different threads) race on it.
+ */
+dit_status dit_condition_static(const float* t, const void* y, int B, int guided, const float* w1,
+                                const float* b1, const float* w2, const float* b2, const float* table,
+                                int cond_kind, int num_classes, int freq_dim, int hidden, float t_scale,
+                                float* c_out, int* status, dit_stream_t stream);
+
 /* Number of kernel launches one dit_forward enqueues for batch B (graph nodes if a
    graph is replayed). */
 int dit_forward_launch_count(const dit_handle* h, int B, float cfg_scale);
