@@ -143,6 +143,7 @@ struct dit_handle {
   float *x_stage = nullptr, *t_stage = nullptr, *out_stage = nullptr;
   void* y_stage = nullptr;
   CUtensorMap tm_ada, tm_sc[5], tm_u, tm_o, tm_g;
+  AttnMaps attn_maps;
   int force_guidance = 0;
   int use_graph = 0;
   // per-launch event timing (dit_profile_enable)
@@ -381,6 +382,7 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
     ok = ok && make_tmap_bf16_kmajor(&H->tm_u, H->u, g.Mmax, d, 128);
     ok = ok && make_tmap_bf16_kmajor(&H->tm_o, H->o, g.Mmax, d, 128);
     ok = ok && make_tmap_bf16_kmajor(&H->tm_g, H->gbuf, g.Mmax, mlp, 128);
+    ok = ok && make_attention_maps(&H->attn_maps, H->q, H->k, H->v, g.Rmax * cfg->heads, g.Tpad, g.DP);
     for (int i = 0; i < N && ok; ++i) {
       BlockW& b = H->blk[i];
       ok = make_tmap_bf16_kmajor(&b.tm_qkv, b.qkv_w, 3 * d, d, g.bn_qkv) &&
@@ -598,7 +600,7 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
 
     if (H->bf16) {
       DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_tc(EPI_QKV, g.bn_qkv, &H->tm_u, &b.tm_qkv, d, qa, H->num_sms, st), "qkv gemm");
-      DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_simt(aa, st), "attention");
+      DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_tc(aa, H->attn_maps, H->status, st), "attention");
       DIT_LAUNCH(H, DIT_KERNEL_PROJ, st, launch_gemm_tc(EPI_RESID, g.bn_proj, &H->tm_o, &b.tm_proj, d, pa, H->num_sms, st), "proj gemm");
     } else {
       DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_simt(EPI_QKV, static_cast<const float*>(H->u), static_cast<const float*>(b.qkv_w), p.M,

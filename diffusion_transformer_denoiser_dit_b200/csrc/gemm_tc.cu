@@ -304,18 +304,27 @@ static PFN_encodeTiled_t encode_fn() {
   return fn;
 }
 
-bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows) {
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                    uint32_t box_rows, int swizzle_bytes) {
   PFN_encodeTiled_t fn = encode_fn();
-  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (K * 2) % 16 != 0 || box_rows == 0 ||
-      box_rows > 256)
+  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (cols * 2) % 16 != 0 || box_rows == 0 ||
+      box_rows > 256 || box_cols == 0 || (box_cols * 2) % 16 != 0 || box_cols * 2 > (uint32_t)swizzle_bytes)
     return false;
-  cuuint64_t dims[2] = {K, rows};
-  cuuint64_t strides[1] = {K * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                : CU_TENSOR_MAP_SWIZZLE_NONE;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows) {
+  return make_tmap_bf16(map, base, rows, K, 64, box_rows, 128);
 }
 
 template <int BN, int EPI>

@@ -46,6 +46,11 @@ cudaError_t launch_gemm_tc(int epi, int block_n, const CUtensorMap* tmA, const C
 int gemm_tc_supported_bn(int block_n);
 // Build a 2-D bf16 K-major tensor map: rows x K, box = box_rows x 64, 128-byte swizzle.
 bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
+// General 2-D bf16 tensor map: rows x cols (cols contiguous), box box_rows x box_cols,
+// swizzle 128 / 64 / 32 bytes (0 = none).  The box row (box_cols * 2 bytes) must not
+// exceed the swizzle span.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                    uint32_t box_rows, int swizzle_bytes);
 
 // float32 SIMT GEMM with the same epilogues (f32 outputs everywhere).
 cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, int M, int N, int K, const EpiArgs& ea,
@@ -95,9 +100,14 @@ struct AttnArgs {
   int bf16;               // 1: bf16 padded layouts, V transposed
 };
 cudaError_t launch_attention_simt(const AttnArgs& a, cudaStream_t st);
-cudaError_t launch_attention_tc(const AttnArgs& a, const CUtensorMap* tq_main, const CUtensorMap* tq_tail,
-                                const CUtensorMap* tk_main, const CUtensorMap* tk_tail, const CUtensorMap* tv,
-                                int* status, cudaStream_t st);
+// Tensor maps of the tensor-core attention: q / k main (box 128 x 64, 128B swizzle),
+// q / k tail (head-dim columns 64..79, box 128 x 16, 32B swizzle; unused when dh = 64),
+// v (transposed, box DP x 64, 128B swizzle).
+struct AttnMaps {
+  CUtensorMap q, qt, k, kt, v;
+};
+bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* v, int RH, int Tpad, int DP);
+cudaError_t launch_attention_tc(const AttnArgs& a, const AttnMaps& maps, int* status, cudaStream_t st);
 
 struct QkNormArgs {   // f32 path: RMSNorm + RoPE applied in place to q, k [R*H, T, dh]
   float *q, *k;
