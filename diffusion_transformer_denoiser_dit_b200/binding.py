@@ -24,7 +24,7 @@ EXPORTS = [
     "dit_create", "dit_weight_count", "dit_forward", "dit_forward_host", "dit_sync_status", "dit_last_error",
     "dit_status_string", "dit_destroy", "dit_set_option", "dit_debug_residual", "dit_debug_condition",
     "dit_debug_wait_probe", "dit_op_linear_bf16", "dit_forward_launch_count", "dit_profile_enable",
-    "dit_profile_read", "dit_condition_static",
+    "dit_profile_read", "dit_condition_static", "dit_op_linear_bf16_pair",
 ]
 
 KERNEL_KINDS = ["cond", "adaln", "patch", "ln", "qkv", "attn", "proj", "fc1", "fc2", "decode"]
@@ -70,6 +70,7 @@ def load() -> ctypes.CDLL:
         "dit_debug_condition": (c_int, [P, P, P, c_int, c_float, P, P]),
         "dit_debug_wait_probe": (c_int, [P, c_int, P]),
         "dit_op_linear_bf16": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, P]),
+        "dit_op_linear_bf16_pair": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, P]),
         "dit_forward_launch_count": (c_int, [P, c_int, c_float]),
         "dit_profile_enable": (c_int, [P, c_int]),
         "dit_profile_read": (c_int, [P, POINTER(c_float), POINTER(c_int)]),
@@ -217,14 +218,16 @@ class DiT:
             pass
 
 
-def linear_bf16(x, w, b, block_n: int = 128, stream=None):
-    """y = x W^T + b on the tensor-core GEMM (x, w: torch bf16 CUDA tensors)."""
+def linear_bf16(x, w, b, block_n: int = 128, stream=None, pair: bool = False):
+    """y = x W^T + b on the tensor-core GEMM (x, w: torch bf16 CUDA tensors);
+    pair=True runs the SM-pair (cta_group::2) kernel."""
     import torch
     lib = load()
     M, K = x.shape
     N = w.shape[0]
     y = torch.empty((M, N), dtype=torch.float32, device=x.device)
-    rc = lib.dit_op_linear_bf16(_ptr(x), _ptr(w), _ptr(b), _ptr(y), M, N, K, block_n, _stream(stream))
+    fn = lib.dit_op_linear_bf16_pair if pair else lib.dit_op_linear_bf16
+    rc = fn(_ptr(x), _ptr(w), _ptr(b), _ptr(y), M, N, K, block_n, _stream(stream))
     if rc != DIT_OK:
         raise DitError(rc, f"dit_op_linear_bf16: {status_string(rc)}")
     return y

@@ -18,12 +18,14 @@ struct BlockW {
   void *qkv_w = nullptr, *proj_w = nullptr, *fc1_w = nullptr, *fc2_w = nullptr;  // bf16 or f32
   float *qkv_b = nullptr, *proj_b = nullptr, *fc1_b = nullptr, *fc2_b = nullptr;
   float *qn = nullptr, *kn = nullptr;
-  CUtensorMap tm_qkv, tm_proj, tm_fc1, tm_fc2;
+  CUtensorMap tm_qkv, tm_fc1;          // weights as the B operand (box = tile width rows)
+  CUtensorMap ta_qkv, ta_proj, ta_fc2;  // weights as the A operand of the swapped GEMMs (box 128 rows)
 };
 
 struct Geometry {
   int gf, gh, gw, T, Kp, P, Cout, dh, DP, Tpad, Rmax, RPalloc, Mmax, nmod;
-  int bn_qkv, bn_proj, bn_fc1, bn_fc2;
+  int bn_qkv, bn_fc1;
+  int headwise;  // 1: QK-RMSNorm / RoPE need whole heads -> two-head tiles for the QKV projection
 };
 
 bool validate(const dit_config* c, std::string& err) {
@@ -70,8 +72,8 @@ bool supported(const dit_config* c, std::string& err) {
     return false;
   }
   if (c->dtype == DIT_DTYPE_BF16) {
-    if (c->hidden % (2 * dh) || c->mlp_hidden % 8) {
-      err = "bf16 path needs an even number of heads and mlp_hidden % 8 == 0";
+    if (c->hidden % (2 * dh) || c->hidden % 32 || c->mlp_hidden % 32) {
+      err = "bf16 path needs an even number of heads and hidden, mlp_hidden multiples of 32";
       return false;
     }
   }
@@ -99,10 +101,13 @@ Geometry geometry(const dit_config* c) {
   g.RPalloc = (g.Rmax + 255) / 256 * 256;
   g.Mmax = g.Rmax * g.T;
   g.nmod = (6 * c->depth + 2) * c->hidden;
-  g.bn_qkv = 2 * g.dh;
-  g.bn_proj = 2 * g.dh;
-  g.bn_fc1 = 2 * g.dh;
-  g.bn_fc2 = 2 * g.dh;
+  // GEMM tiles.  The MMA reads its A and B tiles from shared memory every instruction,
+  // so wide (N = 256) tiles keep the tensor cores fed.  proj, fc2 and (without QK norm
+  // / RoPE) QKV run with swapped operands — A = weights (features), B = tokens — so the
+  // N = 256 tile runs over tokens and the tile count fills the SMs; fc1 runs directly.
+  g.headwise = (c->qk_norm || c->pos_kind == DIT_POS_ROPE3D) ? 1 : 0;
+  g.bn_qkv = g.headwise ? 2 * g.dh : 256;
+  g.bn_fc1 = 256;
   return g;
 }
 
@@ -143,6 +148,8 @@ struct dit_handle {
   float *x_stage = nullptr, *t_stage = nullptr, *out_stage = nullptr;
   void* y_stage = nullptr;
   CUtensorMap tm_ada, tm_sc[5], tm_u, tm_o, tm_g;
+  CUtensorMap tm_g_out, tm_h_red;  // TMA-store targets: GELU output, residual stream
+  CUtensorMap tb_u, tb_o, tb_g;     // activations as the B operand of the swapped GEMMs (box 256 rows)
   AttnMaps attn_maps;
   int force_guidance = 0;
   int use_graph = 0;
@@ -382,13 +389,19 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
     ok = ok && make_tmap_bf16_kmajor(&H->tm_u, H->u, g.Mmax, d, 128);
     ok = ok && make_tmap_bf16_kmajor(&H->tm_o, H->o, g.Mmax, d, 128);
     ok = ok && make_tmap_bf16_kmajor(&H->tm_g, H->gbuf, g.Mmax, mlp, 128);
+    ok = ok && make_tmap_bf16(&H->tm_g_out, H->gbuf, g.Mmax, mlp, 32, 32, 64);
+    ok = ok && make_tmap_f32(&H->tm_h_red, H->h, g.Mmax, d, 32, 16, 128);
+    ok = ok && make_tmap_bf16_kmajor(&H->tb_u, H->u, g.Mmax, d, 256);
+    ok = ok && make_tmap_bf16_kmajor(&H->tb_o, H->o, g.Mmax, d, 256);
+    ok = ok && make_tmap_bf16_kmajor(&H->tb_g, H->gbuf, g.Mmax, mlp, 256);
     ok = ok && make_attention_maps(&H->attn_maps, H->q, H->k, H->v, g.Rmax * cfg->heads, g.Tpad, g.DP);
     for (int i = 0; i < N && ok; ++i) {
       BlockW& b = H->blk[i];
-      ok = make_tmap_bf16_kmajor(&b.tm_qkv, b.qkv_w, 3 * d, d, g.bn_qkv) &&
-           make_tmap_bf16_kmajor(&b.tm_proj, b.proj_w, d, d, g.bn_proj) &&
+      ok = make_tmap_bf16_kmajor(&b.tm_qkv, b.qkv_w, 3 * d, d, g.headwise ? g.bn_qkv : 128) &&
            make_tmap_bf16_kmajor(&b.tm_fc1, b.fc1_w, mlp, d, g.bn_fc1) &&
-           make_tmap_bf16_kmajor(&b.tm_fc2, b.fc2_w, d, mlp, g.bn_fc2);
+           make_tmap_bf16_kmajor(&b.ta_qkv, b.qkv_w, 3 * d, d, 128) &&
+           make_tmap_bf16_kmajor(&b.ta_proj, b.proj_w, d, d, 128) &&
+           make_tmap_bf16_kmajor(&b.ta_fc2, b.fc2_w, d, mlp, 128);
     }
     if (!ok) {
       dit_destroy(H);
@@ -599,9 +612,23 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
     f2.gate = mb + 5 * d;
 
     if (H->bf16) {
-      DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_tc(EPI_QKV, g.bn_qkv, &H->tm_u, &b.tm_qkv, d, qa, H->num_sms, st), "qkv gemm");
+      if (g.headwise) {
+        DIT_LAUNCH(H, DIT_KERNEL_QKV, st,
+                   launch_gemm_tc(EPI_QKV_HEAD, g.bn_qkv, &H->tm_u, &b.tm_qkv, d, qa, H->num_sms, st), "qkv gemm");
+      } else {
+        EpiArgs qt = qa;  // swapped: rows = 3d output features, columns = tokens
+        qt.M = 3 * d;
+        qt.N = p.M;
+        DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_tc(EPI_QKV_T, 256, &b.ta_qkv, &H->tb_u, d, qt, H->num_sms, st),
+                   "qkv gemm");
+      }
       DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_tc(aa, H->attn_maps, H->status, st), "attention");
-      DIT_LAUNCH(H, DIT_KERNEL_PROJ, st, launch_gemm_tc(EPI_RESID, g.bn_proj, &H->tm_o, &b.tm_proj, d, pa, H->num_sms, st), "proj gemm");
+      EpiArgs pt = pa;  // swapped: rows = d output features, columns = tokens
+      pt.M = d;
+      pt.N = p.M;
+      DIT_LAUNCH(H, DIT_KERNEL_PROJ, st,
+                 launch_gemm_tc(EPI_RESID_T, 256, &b.ta_proj, &H->tb_o, d, pt, H->num_sms, st, &H->tm_h_red),
+                 "proj gemm");
     } else {
       DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_simt(EPI_QKV, static_cast<const float*>(H->u), static_cast<const float*>(b.qkv_w), p.M,
                                  3 * d, d, qa, st),
@@ -627,8 +654,15 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
     ln.scale = mb + 4 * d;
     DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "ln2");
     if (H->bf16) {
-      DIT_LAUNCH(H, DIT_KERNEL_FC1, st, launch_gemm_tc(EPI_GELU, g.bn_fc1, &H->tm_u, &b.tm_fc1, d, f1, H->num_sms, st), "fc1 gemm");
-      DIT_LAUNCH(H, DIT_KERNEL_FC2, st, launch_gemm_tc(EPI_RESID, g.bn_fc2, &H->tm_g, &b.tm_fc2, mlp, f2, H->num_sms, st), "fc2 gemm");
+      DIT_LAUNCH(H, DIT_KERNEL_FC1, st,
+                 launch_gemm_tc(EPI_GELU, g.bn_fc1, &H->tm_u, &b.tm_fc1, d, f1, H->num_sms, st, &H->tm_g_out),
+                 "fc1 gemm");
+      EpiArgs ft = f2;  // swapped: rows = d output features, columns = tokens
+      ft.M = d;
+      ft.N = p.M;
+      DIT_LAUNCH(H, DIT_KERNEL_FC2, st,
+                 launch_gemm_tc(EPI_RESID_T, 256, &b.ta_fc2, &H->tb_g, mlp, ft, H->num_sms, st, &H->tm_h_red),
+                 "fc2 gemm");
     } else {
       DIT_LAUNCH(H, DIT_KERNEL_FC1, st, launch_gemm_simt(EPI_GELU, static_cast<const float*>(H->u), static_cast<const float*>(b.fc1_w), p.M,
                                  mlp, d, f1, st),
@@ -688,6 +722,7 @@ dit_status dit_set_option(dit_handle* H, int option, int value) {
     H->use_graph = value != 0;
     return DIT_OK;
   }
+
   return fail(H, DIT_ERR_INVALID_ARG, "unknown option");
 }
 
@@ -790,17 +825,17 @@ dit_status dit_profile_read(dit_handle* H, float* total_ms, int* launches) {
   return DIT_OK;
 }
 
-dit_status dit_op_linear_bf16(const uint16_t* x, const uint16_t* w, const float* b, float* y, int M, int N, int K,
-                              int block_n, dit_stream_t stream) {
+static dit_status op_linear(const uint16_t* x, const uint16_t* w, const float* b, float* y, int M, int N, int K,
+                            int block_n, bool pair, cudaStream_t st) {
   if (x == nullptr || w == nullptr || y == nullptr || M < 0 || N <= 0 || K <= 0 || (K % 8) != 0)
     return DIT_ERR_INVALID_ARG;
-  if (!gemm_tc_supported_bn(block_n)) return DIT_ERR_INVALID_ARG;
+  if (!(pair ? gemm_tc2_supported_bn(block_n) : gemm_tc_supported_bn(block_n))) return DIT_ERR_INVALID_ARG;
   if (M == 0) return DIT_OK;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return DIT_ERR_NO_DEVICE;
   CUtensorMap ta, tb;
-  if (!make_tmap_bf16_kmajor(&ta, x, M, K, 128) || !make_tmap_bf16_kmajor(&tb, w, N, K, block_n))
+  if (!make_tmap_bf16_kmajor(&ta, x, M, K, 128) || !make_tmap_bf16_kmajor(&tb, w, N, K, pair ? block_n / 2 : block_n))
     return DIT_ERR_INVALID_ARG;
   EpiArgs ea = {};
   ea.M = M;
@@ -808,9 +843,19 @@ dit_status dit_op_linear_bf16(const uint16_t* x, const uint16_t* w, const float*
   ea.bias = b;
   ea.out = y;
   ea.ldo = N;
-  if (launch_gemm_tc(EPI_F32, block_n, &ta, &tb, K, ea, sms, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return DIT_ERR_CUDA;
-  return DIT_OK;
+  const cudaError_t e = pair ? launch_gemm_tc2(EPI_F32, block_n, &ta, &tb, K, ea, sms, st)
+                             : launch_gemm_tc(EPI_F32, block_n, &ta, &tb, K, ea, sms, st);
+  return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status dit_op_linear_bf16_pair(const uint16_t* x, const uint16_t* w, const float* b, float* y, int M, int N, int K,
+                                   int block_n, dit_stream_t stream) {
+  return op_linear(x, w, b, y, M, N, K, block_n, true, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dit_status dit_op_linear_bf16(const uint16_t* x, const uint16_t* w, const float* b, float* y, int M, int N, int K,
+                              int block_n, dit_stream_t stream) {
+  return op_linear(x, w, b, y, M, N, K, block_n, false, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

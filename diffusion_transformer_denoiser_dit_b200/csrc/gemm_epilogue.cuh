@@ -1,0 +1,390 @@
+// Fused epilogues of the tensor-core GEMMs.
+//
+// Eight epilogue warps per CTA: warp w reads TMEM lanes 32*(w%4)..+31 (one output
+// row per thread) and one half of the tile's columns.  Columns are read from TMEM in
+// chunks with tcgen05.ld; the load of chunk c+1 is in flight while chunk c is
+// processed (tcgen05.wait::ld only after the processing), so TMEM latency overlaps
+// the arithmetic and the global-memory traffic of the previous chunk.
+// Epilogues: bias (+ tanh-GELU) to bf16, gated residual update of the float32
+// stream, modulation-vector scatter, head-major Q / K / V^T scatter (per column, or
+// per whole head with QK-RMSNorm and 3D RoPE), plain float32 output.
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dit {
+
+template <int W>
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t* r) {
+  if constexpr (W == 32) {
+    tmem_ld32(taddr, r);
+  } else if constexpr (W == 16) {
+    tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+  } else {
+    static_assert(W == 8, "chunk width");
+    DIT_TMEM_LD_X8(taddr, r);
+  }
+}
+
+// Columns [n, n + W) of output row m from the registers v (already accumulated).
+template <int W, int EPI>
+__device__ __forceinline__ void epilogue_chunk(const EpiArgs& ea, const uint32_t* r, int m, int n) {
+  if (m >= ea.M || n >= ea.N) return;
+  const bool full = n + W <= ea.N;
+  if constexpr (EPI == EPI_ADALN) {
+    // rows of this GEMM are modulation features j = m, columns are sample rows
+    const float bj = __ldg(ea.bias + m);
+    float* o = static_cast<float*>(ea.out) + m;
+#pragma unroll
+    for (int i = 0; i < W; ++i)
+      if (n + i < ea.N) o[static_cast<size_t>(n + i) * ea.ldo] = __uint_as_float(r[i]) + bj;
+  } else if constexpr (EPI == EPI_F32) {
+    float* o = static_cast<float*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n;
+    if (full && (ea.ldo & 3) == 0) {
+#pragma unroll
+      for (int i = 0; i < W / 4; ++i) {
+        const float4 b4 =
+            ea.bias ? __ldg(reinterpret_cast<const float4*>(ea.bias + n) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4*>(o)[i] =
+            make_float4(__uint_as_float(r[4 * i]) + b4.x, __uint_as_float(r[4 * i + 1]) + b4.y,
+                        __uint_as_float(r[4 * i + 2]) + b4.z, __uint_as_float(r[4 * i + 3]) + b4.w);
+      }
+    } else {
+      for (int i = 0; i < W && n + i < ea.N; ++i) o[i] = __uint_as_float(r[i]) + (ea.bias ? __ldg(ea.bias + n + i) : 0.f);
+    }
+  } else if constexpr (EPI == EPI_GELU) {
+    uint16_t* o = static_cast<uint16_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n;
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < W / 8; ++i) {
+        const float4 b0 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + 2 * i);
+        const float4 b1 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + 2 * i + 1);
+        uint4 pk;
+        pk.x = pack_bf16x2(gelu_tanh_fast(__uint_as_float(r[8 * i + 0]) + b0.x),
+                           gelu_tanh_fast(__uint_as_float(r[8 * i + 1]) + b0.y));
+        pk.y = pack_bf16x2(gelu_tanh_fast(__uint_as_float(r[8 * i + 2]) + b0.z),
+                           gelu_tanh_fast(__uint_as_float(r[8 * i + 3]) + b0.w));
+        pk.z = pack_bf16x2(gelu_tanh_fast(__uint_as_float(r[8 * i + 4]) + b1.x),
+                           gelu_tanh_fast(__uint_as_float(r[8 * i + 5]) + b1.y));
+        pk.w = pack_bf16x2(gelu_tanh_fast(__uint_as_float(r[8 * i + 6]) + b1.z),
+                           gelu_tanh_fast(__uint_as_float(r[8 * i + 7]) + b1.w));
+        reinterpret_cast<uint4*>(o)[i] = pk;
+      }
+    } else {
+      for (int i = 0; i < W && n + i < ea.N; ++i)
+        o[i] = f32_to_bf16(gelu_tanh_fast(__uint_as_float(r[i]) + __ldg(ea.bias + n + i)));
+    }
+  } else if constexpr (EPI == EPI_RESID) {
+    const int row = m / ea.T;
+    const float* gt = ea.gate + static_cast<size_t>(row) * ea.ld_gate + n;
+    float* hp = ea.h + static_cast<size_t>(m) * ea.ldh + n;
+    if (full) {
+      float4 h4[W / 4];
+#pragma unroll
+      for (int i = 0; i < W / 4; ++i) h4[i] = reinterpret_cast<const float4*>(hp)[i];  // all loads in flight first
+#pragma unroll
+      for (int i = 0; i < W / 4; ++i) {
+        const float4 g4 = __ldg(reinterpret_cast<const float4*>(gt) + i);
+        const float4 b4 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + i);
+        h4[i].x = fmaf(g4.x, __uint_as_float(r[4 * i + 0]) + b4.x, h4[i].x);
+        h4[i].y = fmaf(g4.y, __uint_as_float(r[4 * i + 1]) + b4.y, h4[i].y);
+        h4[i].z = fmaf(g4.z, __uint_as_float(r[4 * i + 2]) + b4.z, h4[i].z);
+        h4[i].w = fmaf(g4.w, __uint_as_float(r[4 * i + 3]) + b4.w, h4[i].w);
+        reinterpret_cast<float4*>(hp)[i] = h4[i];
+      }
+    } else {
+      for (int i = 0; i < W && n + i < ea.N; ++i) hp[i] = fmaf(gt[i], __uint_as_float(r[i]) + ea.bias[n + i], hp[i]);
+    }
+  } else if constexpr (EPI == EPI_QKV) {
+    // per column: groups of 8 never straddle a head (head dim % 8 == 0, d % 8 == 0)
+    const int row = m / ea.T, tok = m - row * ea.T;
+#pragma unroll
+    for (int g8 = 0; g8 < W / 8; ++g8) {
+      const int nn = n + 8 * g8;
+      if (nn >= ea.N) break;
+      const int which = nn / ea.d;
+      const int within = nn - which * ea.d;
+      const int head = within / ea.dh, j = within - head * ea.dh;
+      const float4 b0 = __ldg(reinterpret_cast<const float4*>(ea.bias + nn));
+      const float4 b1 = __ldg(reinterpret_cast<const float4*>(ea.bias + nn) + 1);
+      const float v0 = __uint_as_float(r[8 * g8 + 0]) + b0.x, v1 = __uint_as_float(r[8 * g8 + 1]) + b0.y;
+      const float v2 = __uint_as_float(r[8 * g8 + 2]) + b0.z, v3 = __uint_as_float(r[8 * g8 + 3]) + b0.w;
+      const float v4 = __uint_as_float(r[8 * g8 + 4]) + b1.x, v5 = __uint_as_float(r[8 * g8 + 5]) + b1.y;
+      const float v6 = __uint_as_float(r[8 * g8 + 6]) + b1.z, v7 = __uint_as_float(r[8 * g8 + 7]) + b1.w;
+      if (which < 2) {
+        uint16_t* dst = static_cast<uint16_t*>(which == 0 ? ea.q : ea.k) +
+                        (static_cast<size_t>(row * ea.H + head) * ea.Tpad + tok) * ea.DP + j;
+        *reinterpret_cast<uint4*>(dst) =
+            make_uint4(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3), pack_bf16x2(v4, v5), pack_bf16x2(v6, v7));
+      } else {
+        uint16_t* dst =
+            static_cast<uint16_t*>(ea.v) + (static_cast<size_t>(row * ea.H + head) * ea.DP + j) * ea.Tpad + tok;
+        const size_t s = ea.Tpad;
+        dst[0] = f32_to_bf16(v0);
+        dst[s] = f32_to_bf16(v1);
+        dst[2 * s] = f32_to_bf16(v2);
+        dst[3 * s] = f32_to_bf16(v3);
+        dst[4 * s] = f32_to_bf16(v4);
+        dst[5 * s] = f32_to_bf16(v5);
+        dst[6 * s] = f32_to_bf16(v6);
+        dst[7 * s] = f32_to_bf16(v7);
+      }
+    }
+  }
+}
+
+// One whole head (DH columns) of q, k or v for output row m: bias, optional
+// QK-RMSNorm and 3D RoPE, head-major store.
+template <int DH>
+__device__ __forceinline__ void epilogue_head(const EpiArgs& ea, const uint32_t* r, int m, int n) {
+  if (n >= ea.N) return;
+  const int which = n / ea.d;
+  const int head = (n - which * ea.d) / DH;
+  const int row = m / ea.T, tok = m - row * ea.T;
+  float v[DH];
+#pragma unroll
+  for (int j = 0; j < DH; ++j) v[j] = __uint_as_float(r[j]) + __ldg(ea.bias + n + j);
+  if (which < 2) {
+    const float* gn = which == 0 ? ea.qn : ea.kn;
+    if (gn != nullptr) {
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < DH; ++j) ss = fmaf(v[j], v[j], ss);
+      const float rs = rsqrtf(ss * (1.0f / DH) + 1e-6f);
+#pragma unroll
+      for (int j = 0; j < DH; ++j) v[j] = v[j] * rs * __ldg(gn + j);
+    }
+    if (ea.rope != nullptr) {
+      const float* rp = ea.rope + static_cast<size_t>(tok) * DH;
+#pragma unroll
+      for (int i = 0; i < DH / 2; ++i) {
+        const float c = __ldg(rp + 2 * i), s = __ldg(rp + 2 * i + 1);
+        const float x0 = v[2 * i], x1 = v[2 * i + 1];
+        v[2 * i] = x0 * c - x1 * s;
+        v[2 * i + 1] = x0 * s + x1 * c;
+      }
+    }
+    if (m < ea.M) {
+      uint16_t* dst = static_cast<uint16_t*>(which == 0 ? ea.q : ea.k) +
+                      (static_cast<size_t>(row * ea.H + head) * ea.Tpad + tok) * ea.DP;
+#pragma unroll
+      for (int c = 0; c < DH / 8; ++c)
+        *reinterpret_cast<uint4*>(dst + c * 8) =
+            make_uint4(pack_bf16x2(v[c * 8 + 0], v[c * 8 + 1]), pack_bf16x2(v[c * 8 + 2], v[c * 8 + 3]),
+                       pack_bf16x2(v[c * 8 + 4], v[c * 8 + 5]), pack_bf16x2(v[c * 8 + 6], v[c * 8 + 7]));
+    }
+  } else if (m < ea.M) {
+    uint16_t* dst = static_cast<uint16_t*>(ea.v) + static_cast<size_t>(row * ea.H + head) * ea.DP * ea.Tpad + tok;
+#pragma unroll
+    for (int j = 0; j < DH; ++j) dst[static_cast<size_t>(j) * ea.Tpad] = f32_to_bf16(v[j]);
+  }
+}
+
+// The columns [n0 + c0, n0 + c0 + NC) of a tile for output row m; tacc addresses
+// column 0 of the tile in this warp's TMEM lanes.
+template <int NC, int EPI, bool HEADWISE>
+__device__ __forceinline__ void epilogue_cols(const EpiArgs& ea, uint32_t tacc, int m, int n0, int c0) {
+  if constexpr (HEADWISE) {
+    // NC is exactly one head: load it whole (8-column loads), then process
+    static_assert(NC % 8 == 0, "head width");
+    uint32_t r[NC];
+#pragma unroll
+    for (int c = 0; c < NC / 8; ++c) DIT_TMEM_LD_X8(tacc + c0 + c * 8, (r + c * 8));
+    tmem_ld_wait<NC>(r);
+    epilogue_head<NC>(ea, r, m, n0 + c0);
+  } else {
+    constexpr int W = NC % 32 == 0 ? 32 : (NC % 16 == 0 ? 16 : 8);
+    constexpr int NCH = NC / W;
+    uint32_t r[2][W];
+    tmem_ld_chunk<W>(tacc + c0, r[0]);
+    tmem_ld_wait<W>(r[0]);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      if (c + 1 < NCH) tmem_ld_chunk<W>(tacc + c0 + (c + 1) * W, r[(c + 1) & 1]);
+      epilogue_chunk<W, EPI>(ea, r[c & 1], m, n0 + c0 + c * W);
+      if (c + 1 < NCH) tmem_ld_wait<W>(r[(c + 1) & 1]);
+    }
+  }
+}
+
+// Epilogues that write through shared memory: each warp turns a 32-row x 32-column
+// chunk into a swizzled box in its own 4 KB staging buffer and one lane hands it to
+// the TMA unit (GELU: bf16 store; RESID: float32 reduce-add into the residual
+// stream, so the SM never reads the stream back).  Stores leave as whole rows
+// instead of 32 scattered row pieces per instruction.
+template <int EPI>
+__host__ __device__ constexpr bool epi_staged() {
+  return EPI == EPI_GELU || EPI == EPI_RESID_T;
+}
+constexpr int kStageBytesPerWarp = 4096;
+constexpr int kEpilogueWarps = 8;
+
+// GELU epilogue through shared memory: each 32-row x 32-column chunk is written to
+// the warp's staging buffer as rows of 64 bytes (bf16), with the 16-byte groups of row
+// r rotated by ((r >> 1) & 3) so the 32 lanes' row writes do not collide on banks,
+// then read back so that 4 consecutive lanes cover one 64-byte output row: each store
+// instruction writes 8 whole row segments instead of 32 scattered pieces.
+template <int NC, int EPI>
+__device__ __forceinline__ void epilogue_cols_staged(const EpiArgs& ea, const CUtensorMap* tmC, uint32_t tacc,
+                                                     int m_base, int lane, int n0, int c0, uint8_t* stg) {
+  static_assert(EPI == EPI_GELU, "staged row-major epilogue is the GELU output");
+  static_assert(NC % 32 == 0, "staged epilogues work on 32-column chunks");
+  (void)tmC;
+  constexpr int NCH = NC / 32;
+  uint32_t r[2][32];
+  tmem_ld_chunk<32>(tacc + c0, r[0]);
+  tmem_ld_wait<32>(r[0]);
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    if (c + 1 < NCH) tmem_ld_chunk<32>(tacc + c0 + (c + 1) * 32, r[(c + 1) & 1]);
+    const int n = n0 + c0 + c * 32;
+    const uint32_t* v = r[c & 1];
+    if (n < ea.N) {
+#pragma unroll
+      for (int c16 = 0; c16 < 4; ++c16) {
+        const float4 b0 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + 2 * c16);
+        const float4 b1 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + 2 * c16 + 1);
+        uint4 pk;
+        pk.x = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 0]) + b0.x),
+                           gelu_tanh_fast(__uint_as_float(v[8 * c16 + 1]) + b0.y));
+        pk.y = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 2]) + b0.z),
+                           gelu_tanh_fast(__uint_as_float(v[8 * c16 + 3]) + b0.w));
+        pk.z = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 4]) + b1.x),
+                           gelu_tanh_fast(__uint_as_float(v[8 * c16 + 5]) + b1.y));
+        pk.w = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 6]) + b1.z),
+                           gelu_tanh_fast(__uint_as_float(v[8 * c16 + 7]) + b1.w));
+        *reinterpret_cast<uint4*>(stg + lane * 64 + ((c16 ^ ((lane >> 1) & 3)) << 4)) = pk;
+      }
+      __syncwarp();
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {  // 8 rows x 64 bytes per instruction
+        const int rr = it * 8 + (lane >> 2), c16 = lane & 3;
+        const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((c16 ^ ((rr >> 1) & 3)) << 4));
+        const int m = m_base + rr;
+        if (m < ea.M)
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n + c16 * 8) = val;
+      }
+      __syncwarp();
+    }
+    if (c + 1 < NCH) tmem_ld_wait<32>(r[(c + 1) & 1]);
+  }
+}
+
+// Swapped-operand residual update: lane = output feature f (TMEM lane), columns =
+// tokens.  16-token x 32-feature boxes are staged as [token][feature] float32 rows
+// (128B swizzle: 16-byte group g of row t at g ^ (t & 7)) in two alternating 2 KB
+// buffers, written one token row per instruction by the 32 lanes, and added into the
+// residual stream by the TMA unit (cp.reduce.async.bulk .add), so the SM never reads
+// the stream back.
+template <int NC>
+__device__ __forceinline__ void epilogue_resid_t(const EpiArgs& ea, const CUtensorMap* tmC, uint32_t tacc, int f_base,
+                                                 int lane, int n0, int c0, uint8_t* stg) {
+  static_assert(NC % 32 == 0, "32-token chunks");
+  constexpr int NCH = NC / 32;
+  const int f = f_base + lane;
+  const bool fok = f < ea.M;
+  const float bf = fok ? __ldg(ea.bias + f) : 0.f;
+  uint32_t r[2][32];
+  tmem_ld_chunk<32>(tacc + c0, r[0]);
+  tmem_ld_wait<32>(r[0]);
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    if (c + 1 < NCH) tmem_ld_chunk<32>(tacc + c0 + (c + 1) * 32, r[(c + 1) & 1]);
+    const int tok0 = n0 + c0 + c * 32;
+    const uint32_t* v = r[c & 1];
+    if (tok0 < ea.N) {
+      const int last = min(tok0 + 31, ea.N - 1);
+      const int r0 = tok0 / ea.T, r1 = last / ea.T;
+      const float g0 = fok ? __ldg(ea.gate + static_cast<size_t>(r0) * ea.ld_gate + f) : 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {  // 16 tokens per box, alternating 2 KB buffers
+        uint8_t* buf = stg + half * 2048;
+        if (lane == 0) bulk_wait_read_but1();
+        __syncwarp();
+#pragma unroll
+        for (int tt = 0; tt < 16; ++tt) {
+          const int t = half * 16 + tt;
+          float g = g0;
+          if (r1 != r0) {
+            const int rt = min(tok0 + t, ea.N - 1) / ea.T;
+            g = fok ? __ldg(ea.gate + static_cast<size_t>(rt) * ea.ld_gate + f) : 0.f;
+          }
+          // [token][feature] float32 rows of 128 bytes, 128B swizzle
+          *reinterpret_cast<float*>(buf + tt * 128 + ((((lane >> 2) ^ (tt & 7)) << 4) | ((lane & 3) << 2))) =
+              g * (__uint_as_float(v[t]) + bf);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && f_base < ea.M && tok0 + half * 16 < ea.N) {
+          tma_reduce_add_2d(tmC, smem_u32(buf), f_base, tok0 + half * 16);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (c + 1 < NCH) tmem_ld_wait<32>(r[(c + 1) & 1]);
+  }
+}
+
+// Swapped-operand Q / K / V^T scatter: lane = output feature f of [q | k | v],
+// columns = tokens.  V^T rows are contiguous in tokens, so a lane writes 8 tokens per
+// 16-byte store; q and k are written one token per instruction (32 consecutive
+// head-dim entries across the lanes).
+template <int NC>
+__device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc, int f_base, int lane, int n0, int c0) {
+  static_assert(NC % 32 == 0, "32-token chunks");
+  constexpr int NCH = NC / 32;
+  const int f = f_base + lane;
+  const bool fok = f < ea.M;
+  const int which = fok ? f / ea.d : 0;
+  const int within = f - which * ea.d;
+  const int head = within / ea.dh, j = within - head * ea.dh;
+  const float bf = fok ? __ldg(ea.bias + f) : 0.f;
+  uint16_t* qk = static_cast<uint16_t*>(which == 0 ? ea.q : ea.k);
+  uint32_t r[2][32];
+  tmem_ld_chunk<32>(tacc + c0, r[0]);
+  tmem_ld_wait<32>(r[0]);
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    if (c + 1 < NCH) tmem_ld_chunk<32>(tacc + c0 + (c + 1) * 32, r[(c + 1) & 1]);
+    const int tok0 = n0 + c0 + c * 32;
+    const uint32_t* v = r[c & 1];
+    if (fok && tok0 < ea.N) {
+      const int last = min(tok0 + 31, ea.N - 1);
+      const int r0 = tok0 / ea.T, t0 = tok0 - r0 * ea.T;
+      const bool one_row = (last / ea.T) == r0 && last - tok0 == 31;
+      if (which == 2) {
+        if (one_row && (t0 & 7) == 0) {
+          uint16_t* dst = static_cast<uint16_t*>(ea.v) + (static_cast<size_t>(r0 * ea.H + head) * ea.DP + j) * ea.Tpad + t0;
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8)
+            reinterpret_cast<uint4*>(dst)[g8] =
+                make_uint4(pack_bf16x2(__uint_as_float(v[8 * g8 + 0]) + bf, __uint_as_float(v[8 * g8 + 1]) + bf),
+                           pack_bf16x2(__uint_as_float(v[8 * g8 + 2]) + bf, __uint_as_float(v[8 * g8 + 3]) + bf),
+                           pack_bf16x2(__uint_as_float(v[8 * g8 + 4]) + bf, __uint_as_float(v[8 * g8 + 5]) + bf),
+                           pack_bf16x2(__uint_as_float(v[8 * g8 + 6]) + bf, __uint_as_float(v[8 * g8 + 7]) + bf));
+        } else {
+          for (int t = 0; t < 32 && tok0 + t < ea.N; ++t) {
+            const int rt = (tok0 + t) / ea.T, tt = tok0 + t - rt * ea.T;
+            static_cast<uint16_t*>(ea.v)[(static_cast<size_t>(rt * ea.H + head) * ea.DP + j) * ea.Tpad + tt] =
+                f32_to_bf16(__uint_as_float(v[t]) + bf);
+          }
+        }
+      } else {
+        if (one_row) {
+          uint16_t* dst = qk + (static_cast<size_t>(r0 * ea.H + head) * ea.Tpad + t0) * ea.DP + j;
+#pragma unroll
+          for (int t = 0; t < 32; ++t) dst[static_cast<size_t>(t) * ea.DP] = f32_to_bf16(__uint_as_float(v[t]) + bf);
+        } else {
+          for (int t = 0; t < 32 && tok0 + t < ea.N; ++t) {
+            const int rt = (tok0 + t) / ea.T, tt = tok0 + t - rt * ea.T;
+            qk[(static_cast<size_t>(rt * ea.H + head) * ea.Tpad + tt) * ea.DP + j] = f32_to_bf16(__uint_as_float(v[t]) + bf);
+          }
+        }
+      }
+    }
+    if (c + 1 < NCH) tmem_ld_wait<32>(r[(c + 1) & 1]);
+  }
+}
+
+}  // namespace dit

@@ -13,157 +13,40 @@
 //               let the epilogue of tile i overlap the main loop of tile i+1.
 // Every mbarrier wait is bounded (common.cuh); no TMA multicast is used.
 #include "common.cuh"
+#include "gemm_epilogue.cuh"
 #include "internal.h"
 
 namespace dit {
 
-template <int BN>
+template <int BN, int EPI>
 struct TcCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES_FIT = (220 * 1024) / STAGE_BYTES;
+  static constexpr int STAGING = epi_staged<EPI>() ? kEpilogueWarps * kStageBytesPerWarp : 0;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int STAGES_FIT = (232448 - 1024 - BAR_BYTES - STAGING) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int ACC_COLS = 256;  // TMEM column distance of the two accumulators
   static constexpr int TMEM_COLS = 512;
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STAGING + BAR_BYTES + 1024;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N in [16, 256], N % 16 == 0");
   static_assert(B_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned for the 128B swizzle");
   static_assert(SMEM <= 232448, "dynamic shared memory above the sm_100 limit");
+  static_assert(STAGES >= 3, "pipeline too shallow");
 };
-
-// ------------------------------------------------------------------------- epilogues
-template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_tile(const EpiArgs& ea, uint32_t tacc, int m, int n0) {
-  const bool mok = m < ea.M;
-  if constexpr (EPI == EPI_QKV) {
-    constexpr int DH = BN / 2;  // one tile = two whole heads of q, k or v
-    static_assert(DH % 8 == 0, "head dim must be a multiple of 8");
-#pragma unroll 1
-    for (int g = 0; g < 2; ++g) {
-      uint32_t r[DH];
-#pragma unroll
-      for (int c = 0; c < DH / 8; ++c) DIT_TMEM_LD_X8(tacc + g * DH + c * 8, (r + c * 8));
-      tmem_ld_wait<DH>(r);
-      const int n = n0 + g * DH;
-      if (n >= ea.N) continue;
-      const int which = n / ea.d;
-      const int head = (n - which * ea.d) / DH;
-      const int row = m / ea.T, tok = m - row * ea.T;
-      float v[DH];
-#pragma unroll
-      for (int j = 0; j < DH; ++j) v[j] = __uint_as_float(r[j]) + __ldg(ea.bias + n + j);
-      if (which < 2) {
-        const float* gn = which == 0 ? ea.qn : ea.kn;
-        if (gn != nullptr) {
-          float ss = 0.f;
-#pragma unroll
-          for (int j = 0; j < DH; ++j) ss = fmaf(v[j], v[j], ss);
-          const float rs = rsqrtf(ss * (1.0f / DH) + 1e-6f);
-#pragma unroll
-          for (int j = 0; j < DH; ++j) v[j] = v[j] * rs * __ldg(gn + j);
-        }
-        if (ea.rope != nullptr) {
-          const float* rp = ea.rope + static_cast<size_t>(tok) * DH;
-#pragma unroll
-          for (int i = 0; i < DH / 2; ++i) {
-            const float c = __ldg(rp + 2 * i), s = __ldg(rp + 2 * i + 1);
-            const float x0 = v[2 * i], x1 = v[2 * i + 1];
-            v[2 * i] = x0 * c - x1 * s;
-            v[2 * i + 1] = x0 * s + x1 * c;
-          }
-        }
-        if (mok) {
-          uint16_t* dst = static_cast<uint16_t*>(which == 0 ? ea.q : ea.k) +
-                          (static_cast<size_t>(row * ea.H + head) * ea.Tpad + tok) * ea.DP;
-#pragma unroll
-          for (int c = 0; c < DH / 8; ++c) {
-            uint4 pk;
-            pk.x = pack_bf16x2(v[c * 8 + 0], v[c * 8 + 1]);
-            pk.y = pack_bf16x2(v[c * 8 + 2], v[c * 8 + 3]);
-            pk.z = pack_bf16x2(v[c * 8 + 4], v[c * 8 + 5]);
-            pk.w = pack_bf16x2(v[c * 8 + 6], v[c * 8 + 7]);
-            *reinterpret_cast<uint4*>(dst + c * 8) = pk;
-          }
-        }
-      } else if (mok) {
-        uint16_t* dst = static_cast<uint16_t*>(ea.v) + static_cast<size_t>(row * ea.H + head) * ea.DP * ea.Tpad + tok;
-#pragma unroll
-        for (int j = 0; j < DH; ++j) dst[static_cast<size_t>(j) * ea.Tpad] = f32_to_bf16(v[j]);
-      }
-    }
-  } else {
-#pragma unroll 1
-    for (int c = 0; c < BN / 16; ++c) {
-      uint32_t r[16];
-      tmem_ld16(tacc + c * 16, r);
-      tmem_ld_wait<16>(r);
-      const int n = n0 + c * 16;
-      if (!mok || n >= ea.N) continue;
-      float v[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-      const bool full = (n + 16 <= ea.N);
-      if constexpr (EPI == EPI_ADALN) {
-        // rows of this GEMM are modulation features j = m, columns are sample rows
-        const float bj = __ldg(ea.bias + m);
-        float* o = static_cast<float*>(ea.out) + m;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (n + i < ea.N) o[static_cast<size_t>(n + i) * ea.ldo] = v[i] + bj;
-      } else if constexpr (EPI == EPI_F32) {
-        float* o = static_cast<float*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (n + i < ea.N) o[i] = v[i] + (ea.bias ? __ldg(ea.bias + n + i) : 0.f);
-      } else if constexpr (EPI == EPI_GELU) {
-        uint16_t* o = static_cast<uint16_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n;
-        if (full) {
-          uint32_t p[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            p[i] = pack_bf16x2(gelu_tanh_fast(v[2 * i] + __ldg(ea.bias + n + 2 * i)),
-                               gelu_tanh_fast(v[2 * i + 1] + __ldg(ea.bias + n + 2 * i + 1)));
-          reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
-          reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
-        } else {
-          for (int i = 0; i < 16 && n + i < ea.N; ++i) o[i] = f32_to_bf16(gelu_tanh_fast(v[i] + __ldg(ea.bias + n + i)));
-        }
-      } else if constexpr (EPI == EPI_RESID) {
-        const int row = m / ea.T;
-        const float* gt = ea.gate + static_cast<size_t>(row) * ea.ld_gate + n;
-        float* hp = ea.h + static_cast<size_t>(m) * ea.ldh + n;
-        if (full) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 g4 = __ldg(reinterpret_cast<const float4*>(gt) + i);
-            const float4 b4 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + i);
-            float4 h4 = reinterpret_cast<float4*>(hp)[i];
-            h4.x = fmaf(g4.x, v[4 * i + 0] + b4.x, h4.x);
-            h4.y = fmaf(g4.y, v[4 * i + 1] + b4.y, h4.y);
-            h4.z = fmaf(g4.z, v[4 * i + 2] + b4.z, h4.z);
-            h4.w = fmaf(g4.w, v[4 * i + 3] + b4.w, h4.w);
-            reinterpret_cast<float4*>(hp)[i] = h4;
-          }
-        } else {
-          for (int i = 0; i < 16 && n + i < ea.N; ++i) hp[i] = fmaf(gt[i], v[i] + ea.bias[n + i], hp[i]);
-        }
-      }
-    }
-  }
-}
 
 // ------------------------------------------------------------------------- kernel
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const int K,
-                   const EpiArgs ea) {
-  using C = TcCfg<BN>;
+__global__ void __launch_bounds__(320, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, const int K, const EpiArgs ea) {
+  using C = TcCfg<BN, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + C::STAGING);
   uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 4);
   const uint32_t bar0 = smem_u32(bars);
   // barrier addresses: full[s], empty[s], tmem_full[a], tmem_empty[a]
@@ -185,7 +68,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(TFULL_BAR(a), 1);
-      mbar_init(TEMPTY_BAR(a), 128);
+      mbar_init(TEMPTY_BAR(a), 256);  // 8 epilogue warps
     }
     fence_barrier_init();
   }
@@ -258,7 +141,7 @@ __global__ void __launch_bounds__(192, 1)
         if (ok) mma_commit(TFULL_BAR(a));
       }
     }
-  } else {  // ------------------------ epilogue warps 2..5
+  } else {  // ------------------------ epilogue warps 2..9
     const int q = warp & 3;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
@@ -270,10 +153,21 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int m0 = (tile % m_tiles) * 128, n0 = (tile / m_tiles) * BN;
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * C::ACC_COLS;
-      epilogue_tile<BN, EPI>(ea, tacc, m0 + q * 32 + lane, n0);
+      if constexpr (EPI == EPI_RESID_T)
+        epilogue_resid_t<BN / 2>(ea, &tmC, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
+                                 staging + (warp - 2) * kStageBytesPerWarp);
+      else if constexpr (EPI == EPI_QKV_T)
+        epilogue_qkv_t<BN / 2>(ea, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2));
+      else if constexpr (epi_staged<EPI>())
+        epilogue_cols_staged<BN / 2, EPI>(ea, &tmC, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
+                                          staging + (warp - 2) * kStageBytesPerWarp);
+      else
+        epilogue_cols<BN / 2, (EPI == EPI_QKV_HEAD ? EPI_QKV : EPI), EPI == EPI_QKV_HEAD>(
+            ea, tacc, m0 + q * 32 + lane, n0, ((warp - 2) >> 2) * (BN / 2));
       tc_fence_before();
       mbar_arrive(TEMPTY_BAR(a));
     }
+    if (epi_staged<EPI>() && lane == 0) bulk_wait_all();  // TMA stores of this warp are complete
   }
   tc_fence_before();
   __syncthreads();
@@ -304,23 +198,33 @@ static PFN_encodeTiled_t encode_fn() {
   return fn;
 }
 
-bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
-                    uint32_t box_rows, int swizzle_bytes) {
+static bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, uint32_t esize, const void* base, uint64_t rows,
+                      uint64_t cols, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
   PFN_encodeTiled_t fn = encode_fn();
-  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (cols * 2) % 16 != 0 || box_rows == 0 ||
-      box_rows > 256 || box_cols == 0 || (box_cols * 2) % 16 != 0 || box_cols * 2 > (uint32_t)swizzle_bytes)
+  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (cols * esize) % 16 != 0 || box_rows == 0 ||
+      box_rows > 256 || box_cols == 0 || (box_cols * esize) % 16 != 0 ||
+      (swizzle_bytes > 0 && box_cols * esize > (uint32_t)swizzle_bytes))
     return false;
   CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                           : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                           : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
                                                 : CU_TENSOR_MAP_SWIZZLE_NONE;
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
+  cuuint64_t strides[1] = {cols * esize};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t es[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                    uint32_t box_rows, int swizzle_bytes) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, box_cols, box_rows, swizzle_bytes);
+}
+
+bool make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                   uint32_t box_rows, int swizzle_bytes) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, rows, cols, box_cols, box_rows, swizzle_bytes);
 }
 
 bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows) {
@@ -328,9 +232,9 @@ bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, ui
 }
 
 template <int BN, int EPI>
-static cudaError_t launch_bn(const CUtensorMap* tA, const CUtensorMap* tB, int K, const EpiArgs& ea, int num_sms,
-                             cudaStream_t st) {
-  using C = TcCfg<BN>;
+static cudaError_t launch_bn(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap* tC, int K,
+                             const EpiArgs& ea, int num_sms, cudaStream_t st) {
+  using C = TcCfg<BN, EPI>;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -340,7 +244,7 @@ static cudaError_t launch_bn(const CUtensorMap* tA, const CUtensorMap* tB, int K
   const int tiles = ((ea.M + 127) / 128) * ((ea.N + BN - 1) / BN);
   if (tiles == 0) return cudaSuccess;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_tc_kernel<BN, EPI><<<grid, 192, C::SMEM, st>>>(*tA, *tB, K, ea);
+  gemm_tc_kernel<BN, EPI><<<grid, 320, C::SMEM, st>>>(*tA, *tB, tC ? *tC : *tB, K, ea);
   return cudaGetLastError();
 }
 
@@ -349,9 +253,10 @@ int gemm_tc_supported_bn(int bn) {
 }
 
 cudaError_t launch_gemm_tc(int epi, int bn, const CUtensorMap* tA, const CUtensorMap* tB, int K, const EpiArgs& ea,
-                           int num_sms, cudaStream_t st) {
+                           int num_sms, cudaStream_t st, const CUtensorMap* tC) {
+  if ((epi == EPI_GELU || epi == EPI_RESID_T) && tC == nullptr) return cudaErrorInvalidValue;
 #define DIT_BN_CASE(BNV, EPIV) \
-  if (bn == BNV) return launch_bn<BNV, EPIV>(tA, tB, K, ea, num_sms, st);
+  if (bn == BNV) return launch_bn<BNV, EPIV>(tA, tB, tC, K, ea, num_sms, st);
   switch (epi) {
     case EPI_F32:
       DIT_BN_CASE(16, EPI_F32) DIT_BN_CASE(32, EPI_F32) DIT_BN_CASE(64, EPI_F32) DIT_BN_CASE(128, EPI_F32)
@@ -360,12 +265,18 @@ cudaError_t launch_gemm_tc(int epi, int bn, const CUtensorMap* tA, const CUtenso
       DIT_BN_CASE(16, EPI_ADALN) DIT_BN_CASE(32, EPI_ADALN) DIT_BN_CASE(64, EPI_ADALN)
       DIT_BN_CASE(128, EPI_ADALN) DIT_BN_CASE(256, EPI_ADALN) break;
     case EPI_GELU:
-      DIT_BN_CASE(128, EPI_GELU) DIT_BN_CASE(144, EPI_GELU) DIT_BN_CASE(192, EPI_GELU) DIT_BN_CASE(256, EPI_GELU) break;
+      DIT_BN_CASE(128, EPI_GELU) DIT_BN_CASE(192, EPI_GELU) DIT_BN_CASE(256, EPI_GELU) break;
     case EPI_RESID:
-      DIT_BN_CASE(128, EPI_RESID) DIT_BN_CASE(144, EPI_RESID) DIT_BN_CASE(192, EPI_RESID)
+      DIT_BN_CASE(128, EPI_RESID) DIT_BN_CASE(192, EPI_RESID)
       DIT_BN_CASE(256, EPI_RESID) break;
     case EPI_QKV:
-      DIT_BN_CASE(128, EPI_QKV) DIT_BN_CASE(144, EPI_QKV) break;
+      DIT_BN_CASE(128, EPI_QKV) DIT_BN_CASE(144, EPI_QKV) DIT_BN_CASE(192, EPI_QKV) DIT_BN_CASE(256, EPI_QKV) break;
+    case EPI_QKV_HEAD:
+      DIT_BN_CASE(128, EPI_QKV_HEAD) DIT_BN_CASE(144, EPI_QKV_HEAD) break;
+    case EPI_RESID_T:
+      DIT_BN_CASE(256, EPI_RESID_T) break;
+    case EPI_QKV_T:
+      DIT_BN_CASE(256, EPI_QKV_T) break;
     default:
       break;
   }

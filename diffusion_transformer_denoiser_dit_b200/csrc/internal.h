@@ -13,8 +13,13 @@ enum Epi : int {
   EPI_F32 = 0,    // out[m, n] = acc + bias[n]                              (float32)
   EPI_ADALN = 1,  // out[n, m] = acc + bias[m]   (A = modulation weights, B = SiLU(c) rows)
   EPI_GELU = 2,   // out[m, n] = gelu_tanh(acc + bias[n])                   (bf16 / f32)
-  EPI_RESID = 3,  // h[m, n]  += gate[row(m), n] * (acc + bias[n])          (float32 RMW)
-  EPI_QKV = 4,    // scatter to q, k, v head-major (+ QK-RMSNorm, 3D RoPE)
+  EPI_RESID = 3,  // h[m, n]  += gate[row(m), n] * (acc + bias[n])          (float32 RMW, direct)
+  EPI_QKV = 4,       // scatter to q, k, v head-major, column by column
+  EPI_QKV_HEAD = 5,  // same, one whole head at a time (+ QK-RMSNorm, 3D RoPE); tile = 2 heads
+  // Swapped operands (A = weights, B = activations: GEMM rows are output features,
+  // GEMM columns are tokens; ea.M = features, ea.N = tokens):
+  EPI_RESID_T = 6,   // h[tok, f] += gate[row(tok), f] * (acc + bias[f])   (TMA reduce-add)
+  EPI_QKV_T = 7,     // q, k, v^T scatter, column by column
 };
 
 struct EpiArgs {
@@ -41,9 +46,18 @@ struct EpiArgs {
 
 // tensor-core GEMM D[M, N] = A[M, K] B[N, K]^T with A, B bf16 K-major.
 // Returns cudaSuccess or the launch error.
+// EPI_GELU and EPI_RESID_T write through shared memory with TMA: tmC maps the output
+// (GELU: bf16 [M, N], box 32 rows x 32 columns, 64B swizzle; RESID_T: the float32
+// residual stream [tokens, features], box 16 tokens x 32 features, 128B swizzle,
+// updated with a TMA reduce-add).  Other epilogues ignore tmC.
 cudaError_t launch_gemm_tc(int epi, int block_n, const CUtensorMap* tmA, const CUtensorMap* tmB, int K,
-                           const EpiArgs& ea, int num_sms, cudaStream_t st);
+                           const EpiArgs& ea, int num_sms, cudaStream_t st, const CUtensorMap* tmC = nullptr);
 int gemm_tc_supported_bn(int block_n);
+// Same GEMM on SM pairs (cluster of 2, tcgen05 cta_group::2): 256 x block_n tiles;
+// tmA box = 128 rows x 64, tmB box = block_n/2 rows x 64.
+cudaError_t launch_gemm_tc2(int epi, int block_n, const CUtensorMap* tmA, const CUtensorMap* tmB, int K,
+                            const EpiArgs& ea, int num_sms, cudaStream_t st, const CUtensorMap* tmC = nullptr);
+int gemm_tc2_supported_bn(int block_n);
 // Build a 2-D bf16 K-major tensor map: rows x K, box = box_rows x 64, 128-byte swizzle.
 bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
 // General 2-D bf16 tensor map: rows x cols (cols contiguous), box box_rows x box_cols,
@@ -51,6 +65,9 @@ bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, ui
 // exceed the swizzle span.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                     uint32_t box_rows, int swizzle_bytes);
+// Same for a float32 matrix.
+bool make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                   uint32_t box_rows, int swizzle_bytes);
 
 // float32 SIMT GEMM with the same epilogues (f32 outputs everywhere).
 cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, int M, int N, int K, const EpiArgs& ea,

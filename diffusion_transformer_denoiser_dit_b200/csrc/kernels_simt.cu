@@ -24,42 +24,63 @@ __global__ void cond_sinusoid_kernel(const float* __restrict__ t, int B, int R, 
   }
 }
 
-// out[r, j] = act(sum_i W[j, i] in[r, i] + b[j]); one warp per output feature j, all rows.
+// out[r, j] = act(sum_i W[j, i] in[r, i] + b[j]) (+ e(y_r) for the condition's second
+// layer).  One warp per (output feature j, group of kRowsPerWarp rows): lanes split the
+// K-long dot products, so the weight row is read once per row group.
+constexpr int kRowsPerWarp = 8;
+
+__device__ __forceinline__ void rows_dot(const float* __restrict__ w, const float* __restrict__ in, int K, int r0,
+                                         int nr, int lane, float (&acc)[kRowsPerWarp]) {
+#pragma unroll
+  for (int q = 0; q < kRowsPerWarp; ++q) acc[q] = 0.f;
+  for (int i = lane; i < K; i += 32) {
+    const float wi = __ldg(w + i);
+#pragma unroll
+    for (int q = 0; q < kRowsPerWarp; ++q)
+      if (q < nr) acc[q] = fmaf(wi, in[static_cast<size_t>(r0 + q) * K + i], acc[q]);
+  }
+#pragma unroll
+  for (int q = 0; q < kRowsPerWarp; ++q) acc[q] = warp_sum(acc[q]);
+}
+
 template <bool SILU>
 __global__ void rows_linear_kernel(const float* __restrict__ in, const float* __restrict__ W,
                                    const float* __restrict__ b, float* __restrict__ out, int R, int K, int N) {
-  const int warps = blockDim.x >> 5;
-  const int j = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (j >= N) return;
-  const float* w = W + static_cast<size_t>(j) * K;
-  for (int r = 0; r < R; ++r) {
-    const float* x = in + static_cast<size_t>(r) * K;
-    float acc = 0.f;
-    for (int i = lane; i < K; i += 32) acc = fmaf(__ldg(w + i), x[i], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      float v = acc + b[j];
-      out[static_cast<size_t>(r) * N + j] = SILU ? silu_f(v) : v;
-    }
+  const int groups = (R + kRowsPerWarp - 1) / kRowsPerWarp;
+  if (gw >= N * groups) return;
+  const int j = gw / groups, r0 = (gw - j * groups) * kRowsPerWarp;
+  const int nr = min(kRowsPerWarp, R - r0);
+  float acc[kRowsPerWarp];
+  rows_dot(W + static_cast<size_t>(j) * K, in, K, r0, nr, lane, acc);
+  if (lane == 0) {
+#pragma unroll
+    for (int q = 0; q < kRowsPerWarp; ++q)
+      if (q < nr) {
+        const float v = acc[q] + b[j];
+        out[static_cast<size_t>(r0 + q) * N + j] = SILU ? silu_f(v) : v;
+      }
   }
 }
 
 // c[r, j] = W2 hid[r] + b2 + e(y_r);  sc = SiLU(c) (bf16 or f32).
 // Rows r >= B of a guided batch take the null label num_classes.
 __global__ void cond_out_kernel(CondArgs a) {
-  const int warps = blockDim.x >> 5;
-  const int j = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (j >= a.d) return;
-  const float* w = a.w2 + static_cast<size_t>(j) * a.d;
-  for (int r = 0; r < a.R; ++r) {
-    const float* x = a.hid + static_cast<size_t>(r) * a.d;
-    float acc = 0.f;
-    for (int i = lane; i < a.d; i += 32) acc = fmaf(__ldg(w + i), x[i], acc);
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      float v = acc + a.b2[j];
+  const int groups = (a.R + kRowsPerWarp - 1) / kRowsPerWarp;
+  if (gw >= a.d * groups) return;
+  const int j = gw / groups, r0 = (gw - j * groups) * kRowsPerWarp;
+  const int nr = min(kRowsPerWarp, a.R - r0);
+  float acc[kRowsPerWarp];
+  rows_dot(a.w2 + static_cast<size_t>(j) * a.d, a.hid, a.d, r0, nr, lane, acc);
+  if (lane == 0) {
+#pragma unroll
+    for (int q = 0; q < kRowsPerWarp; ++q) {
+      if (q >= nr) continue;
+      const int r = r0 + q;
+      float v = acc[q] + a.b2[j];
       if (a.cond_kind == DIT_COND_CLASS) {
         int lab;
         if (r < a.B) {
@@ -76,11 +97,11 @@ __global__ void cond_out_kernel(CondArgs a) {
         v += static_cast<const float*>(a.y)[static_cast<size_t>(r % a.B) * a.d + j];
       }
       if (a.c) a.c[static_cast<size_t>(r) * a.d + j] = v;
-      const float s = silu_f(v);
+      const float sv = silu_f(v);
       if (a.sc_bf16)
-        static_cast<uint16_t*>(a.sc)[static_cast<size_t>(r) * a.d + j] = f32_to_bf16(s);
+        static_cast<uint16_t*>(a.sc)[static_cast<size_t>(r) * a.d + j] = f32_to_bf16(sv);
       else
-        static_cast<float*>(a.sc)[static_cast<size_t>(r) * a.d + j] = s;
+        static_cast<float*>(a.sc)[static_cast<size_t>(r) * a.d + j] = sv;
     }
   }
 }
@@ -88,8 +109,10 @@ __global__ void cond_out_kernel(CondArgs a) {
 cudaError_t launch_condition(const CondArgs& a, cudaStream_t st) {
   const int n = a.R * a.freq;
   cond_sinusoid_kernel<<<(n + 255) / 256, 256, 0, st>>>(a.t, a.B, a.R, a.freq, a.t_scale, a.E);
-  rows_linear_kernel<true><<<(a.d + 7) / 8, 256, 0, st>>>(a.E, a.w1, a.b1, a.hid, a.R, a.freq, a.d);
-  cond_out_kernel<<<(a.d + 7) / 8, 256, 0, st>>>(a);
+  const int groups = (a.R + kRowsPerWarp - 1) / kRowsPerWarp;
+  const int warps = a.d * groups;
+  rows_linear_kernel<true><<<(warps + 7) / 8, 256, 0, st>>>(a.E, a.w1, a.b1, a.hid, a.R, a.freq, a.d);
+  cond_out_kernel<<<(warps + 7) / 8, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -150,34 +173,37 @@ cudaError_t launch_patch_embed(const PatchArgs& a, cudaStream_t st) {
 }
 
 // ============================================================================ LN + modulate
-// u = (h - mean) / sqrt(var + 1e-6) * (1 + scale[r]) + shift[r]; one warp per token row,
-// the row held in registers as float4 (two exact passes for mean and variance).
-constexpr int kLnMaxVec = 12;  // d <= 1536
+// u = (h - mean) / sqrt(var + 1e-6) * (1 + scale[r]) + shift[r]  (population variance).
+// One warp per token row, four rows per 128-thread block: the row's float4 loads are
+// all issued before any use, mean and variance are two exact passes over registers,
+// and u leaves as 8-byte (bf16) or 16-byte (f32) stores.  The pass is bound by the
+// memory system: 6 bytes per element for the bf16 output.
+constexpr int kLnMaxVec = 12;  // d <= 1536 (float4 per lane)
+constexpr int kLnRowsPerBlock = 4;
+
 template <bool BF16OUT>
-__global__ void ln_modulate_kernel(LnArgs a) {
-  const int warps = blockDim.x >> 5;
-  const int m = blockIdx.x * warps + (threadIdx.x >> 5);
+__global__ void __launch_bounds__(32 * kLnRowsPerBlock) ln_modulate_kernel(LnArgs a) {
+  const int m = blockIdx.x * kLnRowsPerBlock + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= a.M) return;
   const int nv = a.d >> 2;
   const float4* hp = reinterpret_cast<const float4*>(a.h + static_cast<size_t>(m) * a.d);
   float4 x[kLnMaxVec];
-  float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < kLnMaxVec; ++i) {
-    const int c = lane + 32 * i;
-    if (c < nv) {
-      x[i] = hp[c];
-      s += (x[i].x + x[i].y) + (x[i].z + x[i].w);
-    }
+  for (int k = 0; k < kLnMaxVec; ++k) {
+    const int c = lane + 32 * k;
+    x[k] = c < nv ? hp[c] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  const float mean = warp_sum(s) / a.d;
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < kLnMaxVec; ++k) sum += (x[k].x + x[k].y) + (x[k].z + x[k].w);
+  const float mean = warp_sum(sum) / a.d;
   float q = 0.f;
 #pragma unroll
-  for (int i = 0; i < kLnMaxVec; ++i) {
-    const int c = lane + 32 * i;
+  for (int k = 0; k < kLnMaxVec; ++k) {
+    const int c = lane + 32 * k;
     if (c < nv) {
-      const float dx = x[i].x - mean, dy = x[i].y - mean, dz = x[i].z - mean, dw = x[i].w - mean;
+      const float dx = x[k].x - mean, dy = x[k].y - mean, dz = x[k].z - mean, dw = x[k].w - mean;
       q += (dx * dx + dy * dy) + (dz * dz + dw * dw);
     }
   }
@@ -186,15 +212,15 @@ __global__ void ln_modulate_kernel(LnArgs a) {
   const float4* sh = reinterpret_cast<const float4*>(a.shift + static_cast<size_t>(r) * a.ld_mod);
   const float4* sc = reinterpret_cast<const float4*>(a.scale + static_cast<size_t>(r) * a.ld_mod);
 #pragma unroll
-  for (int i = 0; i < kLnMaxVec; ++i) {
-    const int c = lane + 32 * i;
+  for (int k = 0; k < kLnMaxVec; ++k) {
+    const int c = lane + 32 * k;
     if (c < nv) {
       const float4 s4 = __ldg(sc + c), b4 = __ldg(sh + c);
       float4 o;
-      o.x = (x[i].x - mean) * rstd * (1.f + s4.x) + b4.x;
-      o.y = (x[i].y - mean) * rstd * (1.f + s4.y) + b4.y;
-      o.z = (x[i].z - mean) * rstd * (1.f + s4.z) + b4.z;
-      o.w = (x[i].w - mean) * rstd * (1.f + s4.w) + b4.w;
+      o.x = (x[k].x - mean) * rstd * (1.f + s4.x) + b4.x;
+      o.y = (x[k].y - mean) * rstd * (1.f + s4.y) + b4.y;
+      o.z = (x[k].z - mean) * rstd * (1.f + s4.z) + b4.z;
+      o.w = (x[k].w - mean) * rstd * (1.f + s4.w) + b4.w;
       if (BF16OUT) {
         uint2 p;
         p.x = pack_bf16x2(o.x, o.y);
@@ -209,11 +235,12 @@ __global__ void ln_modulate_kernel(LnArgs a) {
 
 cudaError_t launch_ln_modulate(const LnArgs& a, cudaStream_t st) {
   if ((a.d & 3) != 0 || a.d > 4 * 32 * kLnMaxVec) return cudaErrorInvalidValue;
-  const int grid = (a.M + 7) / 8;
+  const int grid = (a.M + kLnRowsPerBlock - 1) / kLnRowsPerBlock;
+  if (grid == 0) return cudaSuccess;
   if (a.u_bf16)
-    ln_modulate_kernel<true><<<grid, 256, 0, st>>>(a);
+    ln_modulate_kernel<true><<<grid, 32 * kLnRowsPerBlock, 0, st>>>(a);
   else
-    ln_modulate_kernel<false><<<grid, 256, 0, st>>>(a);
+    ln_modulate_kernel<false><<<grid, 32 * kLnRowsPerBlock, 0, st>>>(a);
   return cudaGetLastError();
 }
 

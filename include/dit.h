@@ -235,6 +235,15 @@ dit_status dit_condition_static(const float* t, const void* y, int B, int guided
                                 int cond_kind, int num_classes, int freq_dim, int hidden, float t_scale,
                                 float* c_out, int* status, dit_stream_t stream);
 
+/*
+ * dit_op_linear_bf16_pair — the same product on SM pairs: a cluster of two CTAs
+ * issues tcgen05.mma.cta_group::2 on 256 x block_n output tiles, each SM loading half
+ * of the A rows and half of the W rows of every stage.  block_n: 64, 128, 144, 192 or
+ * 256.  Same argument rules as dit_op_linear_bf16.
+ */
+dit_status dit_op_linear_bf16_pair(const uint16_t* x, const uint16_t* w, const float* b, float* y,
+                                   int M, int N, int K, int block_n, dit_stream_t stream);
+
 /* Number of kernel launches one dit_forward enqueues for batch B (graph nodes if a
    graph is replayed). */
 int dit_forward_launch_count(const dit_handle* h, int B, float cfg_scale);

@@ -89,6 +89,22 @@ def test_tcgen05_linear_matches_definition(M, N, K, bn):
     assert err < 1e-5, err
 
 
+@pytest.mark.parametrize("M,N,K,bn", [
+    (256, 128, 64, 128), (300, 144, 1152, 144), (77, 64, 72, 64), (1000, 192, 200, 192),
+    (513, 256, 4608, 256), (8192, 3456, 1152, 144), (8192, 1152, 4608, 128), (8192, 4608, 1152, 256),
+])
+def test_tcgen05_pair_linear_matches_definition(M, N, K, bn):
+    g = torch.Generator(device="cuda").manual_seed(M * 11 + N)
+    x = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    w = torch.randn(N, K, device="cuda", generator=g).to(torch.bfloat16)
+    b = torch.randn(N, device="cuda", generator=g)
+    y = binding.linear_bf16(x, w, b, block_n=bn, pair=True)
+    torch.cuda.synchronize()
+    ref = x.double().cpu().numpy() @ w.double().cpu().numpy().T + b.double().cpu().numpy()
+    err = np.abs(y.cpu().numpy() - ref).max() / np.abs(ref).max()
+    assert err < 1e-5, err
+
+
 # ----------------------------------------------------------------------------- end to end
 @pytest.mark.parametrize("name", list(SMALL))
 @pytest.mark.parametrize("gates", ["random", "strong"])
