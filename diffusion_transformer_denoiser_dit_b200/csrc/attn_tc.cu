@@ -1,18 +1,18 @@
 // Tensor-core flash attention for sm_100a (full, non-causal, one head per CTA row).
 //
 // O = softmax(Q K^T / sqrt(dh)) V for a 128-query tile of one (sample row, head):
-//   warp 0   one thread loads Q once, then K_j and V_j^T per key tile (TMA, no
-//            multicast); single-buffered K and V, each refilled as soon as the MMA
-//            that read it completes (polled without blocking, so neither waits on
-//            the other).
-//   warp 1   allocates 256 TMEM columns (S: 128, O: 128) and one thread issues
-//            S_j = Q K_j^T (M=128, N=128, K=dh padded to 80) and O += P_{j-1} V_{j-1}
-//            (M=128, N=DP, K=128) with tcgen05.mma.
-//   warps 2-5 one query row per thread: S_j from TMEM into registers (then S is
-//            released for the next Q K^T), online softmax in base 2 with lazy O
-//            rescaling (only when the running max grows by more than 2^8), P_j as
-//            bf16 into swizzled shared memory, final O / l to global memory.
-// Two CTAs fit on one SM (about 93 KB shared memory and 256 TMEM columns each), so
+//   warp 0   one thread loads Q once, then K_j and V_j^T into two-stage rings (TMA,
+//            no multicast); a stage is refilled as soon as the MMA that read it
+//            completed (polled without blocking, so the K and V streams never wait on
+//            each other).  For T <= 256 every tile is requested at the start.
+//   warp 1   allocates 256 TMEM columns (S: 0..127, O: 128..) and one thread issues
+//            S_j = Q K_j^T (M=128, N=128, K=dh padded to 80, both operands in shared
+//            memory) and O += P_j V_j (M=128, N=DP, K=128) with P_j read from TMEM.
+//   warps 2-5 one query row per thread: S_j from TMEM into registers, online softmax
+//            in base 2 with lazy O rescaling (only when the running max grows by more
+//            than 2^8), P_j as packed bf16 written back over the first 64 columns of
+//            S (tcgen05.st), final O / l to global memory.
+// Two CTAs fit on one SM (about 102 KB shared memory and 256 TMEM columns each), so
 // one CTA's softmax overlaps the other's MMAs.
 //
 // Layouts: q, k [R*H, Tpad, DP] bf16 (rows of one head contiguous, head dim padded
@@ -28,26 +28,25 @@ namespace dit {
 template <int DH>
 struct AttnCfg {
   static constexpr int DP = (DH + 15) / 16 * 16;
-  static constexpr bool TAIL = DP > 64;                  // head-dim columns 64..DP-1
-  static constexpr int MAIN = 128 * 128;                 // 128 rows x 64 bf16
-  static constexpr int TAILB = TAIL ? 128 * 32 : 0;      // 128 rows x 16 bf16
-  static constexpr int V_ATOM = DP * 128;                // DP rows x 64 keys
+  static constexpr bool TAIL = DP > 64;                 // head-dim columns 64..DP-1
+  static constexpr int MAIN = 128 * 128;                // 128 rows x 64 bf16
+  static constexpr int TAILB = TAIL ? 128 * 32 : 0;     // 128 rows x 16 bf16
+  static constexpr int QK_TILE = MAIN + TAILB;          // one Q or K tile
+  static constexpr int V_ATOM = DP * 128;               // DP rows x 64 keys
+  static constexpr int V_TILE = 2 * V_ATOM;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_QT = OFF_Q + MAIN;
-  static constexpr int OFF_K = OFF_QT + TAILB;
-  static constexpr int OFF_KT = OFF_K + MAIN;
-  static constexpr int OFF_V = OFF_KT + TAILB;
-  static constexpr int OFF_P = OFF_V + 2 * V_ATOM;
-  static constexpr int OFF_BAR = OFF_P + 2 * MAIN;
+  static constexpr int OFF_K = OFF_Q + QK_TILE;         // two K stages
+  static constexpr int OFF_V = OFF_K + 2 * QK_TILE;     // two V^T stages
+  static constexpr int OFF_BAR = OFF_V + 2 * V_TILE;
   static constexpr int SMEM = OFF_BAR + 128 + 1024;
-  static constexpr int Q_BYTES = MAIN + TAILB;
-  static constexpr int V_BYTES = 2 * V_ATOM;
   static constexpr int TMEM_COLS = 256;
   static constexpr int O_COL = 128;
-  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_P % 1024 == 0 && V_ATOM % 1024 == 0, "alignment");
+  static_assert(QK_TILE % 1024 == 0 && V_ATOM % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
 };
 
-enum { B_Q = 0, B_K, B_V, B_S, B_SFREE, B_P, B_O, B_COUNT };
+// barriers: Q loaded; K / V^T stage full and empty (two stages each); S ready; P ready; P V done
+enum { B_Q = 0, B_KF0, B_KF1, B_KE0, B_KE1, B_VF0, B_VF1, B_VE0, B_VE1, B_S, B_P, B_O, B_COUNT };
 
 template <int DH>
 __global__ void __launch_bounds__(192, 2)
@@ -68,13 +67,7 @@ __global__ void __launch_bounds__(192, 2)
   const int nk = (a.T + 127) / 128;
 
   if (threadIdx.x == 0) {
-    mbar_init(BAR(B_Q), 1);
-    mbar_init(BAR(B_K), 1);
-    mbar_init(BAR(B_V), 1);
-    mbar_init(BAR(B_S), 1);
-    mbar_init(BAR(B_SFREE), 128);
-    mbar_init(BAR(B_P), 128);
-    mbar_init(BAR(B_O), 1);
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(BAR(i), i == B_P ? 128 : 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -85,33 +78,37 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *holder;
+  // set-up done: the next kernel may start its own; then wait for the inputs
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
-    if (lane == 0) {  // ---------------- Q once; K_j and V_j^T as soon as their buffers free up
+    if (lane == 0) {  // ---------------- loads: Q once; K_j and V_j^T into two-stage rings
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       const int qrow0 = rh * a.Tpad + qt * 128;
       const int vrow0 = rh * C::DP;
-      mbar_arrive_expect_tx(BAR(B_Q), C::Q_BYTES);
+      mbar_arrive_expect_tx(BAR(B_Q), C::QK_TILE);
       tma_load_2d(sbase + C::OFF_Q, &tmQ, BAR(B_Q), 0, qrow0);
-      if (C::TAIL) tma_load_2d(sbase + C::OFF_QT, &tmQt, BAR(B_Q), 64, qrow0);
+      if (C::TAIL) tma_load_2d(sbase + C::OFF_Q + C::MAIN, &tmQt, BAR(B_Q), 64, qrow0);
       int jk = 0, jv = 0;
       const uint64_t t0 = global_timer_ns();
       while (jk < nk || jv < nk) {
-        // K_jk may replace K_{jk-1} once Q K_{jk-1}^T completed; V_jv may replace
-        // V_{jv-1} once P_{jv-1} V_{jv-1} completed.
-        if (jk < nk && (jk == 0 || mbar_test(BAR(B_S), (jk - 1) & 1))) {
+        // stage j&1 is free once the MMA that read its previous tile (j-2) completed
+        if (jk < nk && (jk < 2 || mbar_test(BAR(B_KE0 + (jk & 1)), ((jk >> 1) & 1) ^ 1u))) {
+          const uint32_t dst = sbase + C::OFF_K + (jk & 1) * C::QK_TILE;
           const int krow0 = rh * a.Tpad + jk * 128;
-          mbar_arrive_expect_tx(BAR(B_K), C::Q_BYTES);
-          tma_load_2d(sbase + C::OFF_K, &tmK, BAR(B_K), 0, krow0);
-          if (C::TAIL) tma_load_2d(sbase + C::OFF_KT, &tmKt, BAR(B_K), 64, krow0);
+          mbar_arrive_expect_tx(BAR(B_KF0 + (jk & 1)), C::QK_TILE);
+          tma_load_2d(dst, &tmK, BAR(B_KF0 + (jk & 1)), 0, krow0);
+          if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmKt, BAR(B_KF0 + (jk & 1)), 64, krow0);
           ++jk;
         }
-        if (jv < nk && (jv == 0 || mbar_test(BAR(B_O), (jv - 1) & 1))) {
-          mbar_arrive_expect_tx(BAR(B_V), C::V_BYTES);
-          tma_load_2d(sbase + C::OFF_V, &tmV, BAR(B_V), jv * 128, vrow0);
-          tma_load_2d(sbase + C::OFF_V + C::V_ATOM, &tmV, BAR(B_V), jv * 128 + 64, vrow0);
+        if (jv < nk && (jv < 2 || mbar_test(BAR(B_VE0 + (jv & 1)), ((jv >> 1) & 1) ^ 1u))) {
+          const uint32_t dst = sbase + C::OFF_V + (jv & 1) * C::V_TILE;
+          mbar_arrive_expect_tx(BAR(B_VF0 + (jv & 1)), C::V_TILE);
+          tma_load_2d(dst, &tmV, BAR(B_VF0 + (jv & 1)), jv * 128, vrow0);
+          tma_load_2d(dst + C::V_ATOM, &tmV, BAR(B_VF0 + (jv & 1)), jv * 128 + 64, vrow0);
           ++jv;
         }
         if (global_timer_ns() - t0 > kWaitLimitNs) {
@@ -121,45 +118,40 @@ __global__ void __launch_bounds__(192, 2)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {  // ------------------------------ MMA issuer
+    if (lane == 0) {  // ---------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, C::DP);
       const uint32_t tS = tmem_base;
       const uint32_t tO = tmem_base + C::O_COL;
       bool ok = mbar_wait(BAR(B_Q), 0, status);
-      auto issue_pv = [&](int jj) -> bool {
-        if (!mbar_wait(BAR(B_P), jj & 1, status)) return false;
-        if (!mbar_wait(BAR(B_V), jj & 1, status)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t pa = sbase + C::OFF_P + (k >> 2) * C::MAIN + (k & 3) * 32;
-          const uint32_t vb = sbase + C::OFF_V + (k >> 2) * C::V_ATOM + (k & 3) * 32;
-          mma_bf16_ss(tO, sdesc_k_sw128(pa), sdesc_k_sw128(vb), idesc_o, (jj > 0 || k > 0) ? 1u : 0u);
-        }
-        mma_commit(BAR(B_O));
-        return true;
-      };
       for (int j = 0; j < nk && ok; ++j) {
-        if (!mbar_wait(BAR(B_K), j & 1, status)) {
-          ok = false;
-          break;
-        }
-        if (j > 0 && !mbar_wait(BAR(B_SFREE), (j - 1) & 1, status)) {
-          ok = false;
-          break;
-        }
+        const int st = j & 1;
+        const uint32_t use = (j >> 1) & 1;
+        ok = mbar_wait(BAR(B_KF0 + st), use, status);
+        // S (and P_{j-1}, which lives in S) may be overwritten once P_{j-1} V_{j-1} completed
+        if (ok && j > 0) ok = mbar_wait(BAR(B_O), (j - 1) & 1, status);
+        if (!ok) break;
         tc_fence_after();
+        const uint32_t kb = sbase + C::OFF_K + st * C::QK_TILE;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          mma_bf16_ss(tS, sdesc_k_sw128(sbase + C::OFF_Q + k * 32), sdesc_k_sw128(sbase + C::OFF_K + k * 32), idesc_s,
+          mma_bf16_ss(tS, sdesc_k_sw128(sbase + C::OFF_Q + k * 32), sdesc_k_sw128(kb + k * 32), idesc_s,
                       k > 0 ? 1u : 0u);
-        if (C::TAIL)
-          mma_bf16_ss(tS, sdesc_k_sw32(sbase + C::OFF_QT), sdesc_k_sw32(sbase + C::OFF_KT), idesc_s, 1u);
+        if (C::TAIL) mma_bf16_ss(tS, sdesc_k_sw32(sbase + C::OFF_Q + C::MAIN), sdesc_k_sw32(kb + C::MAIN), idesc_s, 1u);
         mma_commit(BAR(B_S));
-        if (j > 0 && !issue_pv(j - 1)) ok = false;
+        mma_commit(BAR(B_KE0 + st));
+        // O += P_j V_j: P_j (bf16, 64 TMEM columns over S) as the A operand
+        ok = mbar_wait(BAR(B_P), j & 1, status) && mbar_wait(BAR(B_VF0 + st), use, status);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t vb = sbase + C::OFF_V + st * C::V_TILE;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_bf16_ts(tO, tS + 8 * k, sdesc_k_sw128(vb + (k >> 2) * C::V_ATOM + (k & 3) * 32), idesc_o,
+                      (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(BAR(B_O));
+        mma_commit(BAR(B_VE0 + st));
       }
-      if (ok) issue_pv(nk - 1);
     }
   } else {  // ------------------------------------------ softmax / output warps 2..5
     const int q = warp & 3;
@@ -167,7 +159,6 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t tS = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t tO = tS + C::O_COL;
     const float sc = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
-    uint8_t* prow = smem + C::OFF_P + r * 128;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
@@ -182,9 +173,6 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s + c * 32);
       tmem_ld_wait<128>(s);
-      tc_fence_before();
-      mbar_arrive(BAR(B_SFREE));
-
       const int kvalid = a.T - j * 128;
       float mx = -INFINITY;
 #pragma unroll
@@ -195,19 +183,11 @@ __global__ void __launch_bounds__(192, 2)
         mx = fmaxf(mx, v);
       }
       const float m_new = fmaxf(m_ref, mx * sc);
-      bool waited_o = false;
       if (j == 0) {
         m_ref = m_new;
       } else if (__any_sync(0xffffffffu, m_new - m_ref > 8.0f)) {
-        // the previous P V must be complete before O is rescaled in place
-        const bool okw = mbar_wait(BAR(B_O), (j - 1) & 1, status);
-        __syncwarp();
-        if (__any_sync(0xffffffffu, !okw)) {
-          ok = false;
-          break;
-        }
-        waited_o = true;
-        tc_fence_after();
+        // lazy rescale: O only moves to the new reference when the maximum grew by more
+        // than 2^8 (P_{j-1} V_{j-1} has completed: Q K_j^T was issued after it)
         const float alpha = ex2_approx(m_ref - m_new);
 #pragma unroll
         for (int c = 0; c < C::DP / 16; ++c) {
@@ -218,35 +198,25 @@ __global__ void __launch_bounds__(192, 2)
           for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st16(tO + c * 16, o);
         }
-        tmem_st_wait();
         l *= alpha;
         m_ref = m_new;
       }
-      if (j > 0 && !waited_o) {  // P buffer is free once the previous P V completed
-        const bool okw = mbar_wait(BAR(B_O), (j - 1) & 1, status);
-        __syncwarp();
-        if (__any_sync(0xffffffffu, !okw)) {
-          ok = false;
-          break;
-        }
-      }
-      // P = 2^(s*sc - m_ref) as bf16, written in the 128B-swizzled K-major layout
+      // P = 2^(s*sc - m_ref) as bf16 pairs, written over the first 64 columns of S
       float rs = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        uint32_t pk[4];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[ch * 8 + 2 * e]), sc, -m_ref));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[ch * 8 + 2 * e + 1]), sc, -m_ref));
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * e]), sc, -m_ref));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * e + 1]), sc, -m_ref));
           rs += p0 + p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
-        const int atom = ch >> 3, c16 = ch & 7;
-        *reinterpret_cast<uint4*>(prow + atom * C::MAIN + ((c16 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        tmem_st32(tS + half * 32, pk);
       }
+      tmem_st_wait();
       l += rs;
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(BAR(B_P));
     }
@@ -309,8 +279,7 @@ static cudaError_t launch_dh(const AttnArgs& a, const AttnMaps& mp, int* status,
     attr_done = true;
   }
   dim3 grid(a.Tpad / 128, a.R * a.H);
-  attn_tc_kernel<DH><<<grid, 192, C::SMEM, st>>>(mp.q, mp.qt, mp.k, mp.kt, mp.v, a, status);
-  return cudaGetLastError();
+  return launch_kernel(attn_tc_kernel<DH>, grid, dim3(192), C::SMEM, st, mp.q, mp.qt, mp.k, mp.kt, mp.v, a, status);
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, const AttnMaps& maps, int* status, cudaStream_t st) {

@@ -722,6 +722,10 @@ dit_status dit_set_option(dit_handle* H, int option, int value) {
     H->use_graph = value != 0;
     return DIT_OK;
   }
+  if (option == DIT_OPT_OVERLAP_LAUNCH) {
+    dit::g_pdl = value != 0;
+    return DIT_OK;
+  }
 
   return fail(H, DIT_ERR_INVALID_ARG, "unknown option");
 }

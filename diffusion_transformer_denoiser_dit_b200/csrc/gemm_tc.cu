@@ -84,6 +84,9 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *holder;
+  // set-up done: the next kernel may start its own; then wait for the inputs
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {  // ---------------- TMA producer
@@ -244,8 +247,7 @@ static cudaError_t launch_bn(const CUtensorMap* tA, const CUtensorMap* tB, const
   const int tiles = ((ea.M + 127) / 128) * ((ea.N + BN - 1) / BN);
   if (tiles == 0) return cudaSuccess;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_tc_kernel<BN, EPI><<<grid, 320, C::SMEM, st>>>(*tA, *tB, tC ? *tC : *tB, K, ea);
-  return cudaGetLastError();
+  return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(320), C::SMEM, st, *tA, *tB, tC ? *tC : *tB, K, ea);
 }
 
 int gemm_tc_supported_bn(int bn) {

@@ -90,6 +90,9 @@ __global__ void __launch_bounds__(320, 1)
   cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *holder;
+  // set-up done: the next kernel may start its own; then wait for the inputs
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {  // ---------------- TMA producer (both CTAs)
@@ -235,13 +238,15 @@ static cudaError_t launch_pair_bn(const CUtensorMap* tA, const CUtensorMap* tB, 
   cfg.blockDim = dim3(320, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = g_pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, EPI>, *tA, *tB, tC ? *tC : *tB, K, ea);
 }
 

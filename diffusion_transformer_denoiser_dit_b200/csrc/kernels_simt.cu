@@ -8,11 +8,15 @@
 
 namespace dit {
 
+bool g_pdl = true;
+
 // ============================================================================ condition
 // E[r, i]: timestep sinusoid [cos(t' f_i) | sin(t' f_i)], f_i = 10000^(-i/half),
 // t' = t[b] * t_scale, in double so the argument (up to ~1000 rad) keeps full accuracy.
 __global__ void cond_sinusoid_kernel(const float* __restrict__ t, int B, int R, int freq, float t_scale,
                                      float* __restrict__ E) {
+  pdl_trigger();
+  pdl_wait();
   const int half = freq / 2;
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < R * freq; idx += gridDim.x * blockDim.x) {
     const int r = idx / freq, i = idx - r * freq;
@@ -46,6 +50,8 @@ __device__ __forceinline__ void rows_dot(const float* __restrict__ w, const floa
 template <bool SILU>
 __global__ void rows_linear_kernel(const float* __restrict__ in, const float* __restrict__ W,
                                    const float* __restrict__ b, float* __restrict__ out, int R, int K, int N) {
+  pdl_trigger();
+  pdl_wait();
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int groups = (R + kRowsPerWarp - 1) / kRowsPerWarp;
@@ -67,6 +73,8 @@ __global__ void rows_linear_kernel(const float* __restrict__ in, const float* __
 // c[r, j] = W2 hid[r] + b2 + e(y_r);  sc = SiLU(c) (bf16 or f32).
 // Rows r >= B of a guided batch take the null label num_classes.
 __global__ void cond_out_kernel(CondArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int groups = (a.R + kRowsPerWarp - 1) / kRowsPerWarp;
@@ -108,12 +116,15 @@ __global__ void cond_out_kernel(CondArgs a) {
 
 cudaError_t launch_condition(const CondArgs& a, cudaStream_t st) {
   const int n = a.R * a.freq;
-  cond_sinusoid_kernel<<<(n + 255) / 256, 256, 0, st>>>(a.t, a.B, a.R, a.freq, a.t_scale, a.E);
+  cudaError_t e = launch_kernel(cond_sinusoid_kernel, dim3((n + 255) / 256), dim3(256), 0, st, a.t, a.B, a.R, a.freq,
+                                 a.t_scale, a.E);
+  if (e != cudaSuccess) return e;
   const int groups = (a.R + kRowsPerWarp - 1) / kRowsPerWarp;
   const int warps = a.d * groups;
-  rows_linear_kernel<true><<<(warps + 7) / 8, 256, 0, st>>>(a.E, a.w1, a.b1, a.hid, a.R, a.freq, a.d);
-  cond_out_kernel<<<(warps + 7) / 8, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  e = launch_kernel(rows_linear_kernel<true>, dim3((warps + 7) / 8), dim3(256), 0, st, (const float*)a.E, a.w1, a.b1,
+                    a.hid, a.R, a.freq, a.d);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(cond_out_kernel, dim3((warps + 7) / 8), dim3(256), 0, st, a);
 }
 
 // ============================================================================ patch embed
@@ -121,6 +132,8 @@ cudaError_t launch_condition(const CondArgs& a, cudaStream_t st) {
 // Block: 16 tokens of one row; patch vectors gathered to shared memory first.
 constexpr int kPatchTok = 16;
 __global__ void patch_embed_kernel(PatchArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float sp[];  // [kPatchTok][Kp]
   const int gh = a.H / a.ph, gw = a.W / a.pw, gf = a.F / a.pt;
   const int T = gf * gh * gw;
@@ -168,8 +181,7 @@ cudaError_t launch_patch_embed(const PatchArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
   }
   dim3 grid((T + kPatchTok - 1) / kPatchTok, a.R);
-  patch_embed_kernel<<<grid, 256, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(patch_embed_kernel, grid, dim3(256), smem, st, a);
 }
 
 // ============================================================================ LN + modulate
@@ -183,6 +195,8 @@ constexpr int kLnRowsPerBlock = 4;
 
 template <bool BF16OUT>
 __global__ void __launch_bounds__(32 * kLnRowsPerBlock) ln_modulate_kernel(LnArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int m = blockIdx.x * kLnRowsPerBlock + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= a.M) return;
@@ -238,10 +252,8 @@ cudaError_t launch_ln_modulate(const LnArgs& a, cudaStream_t st) {
   const int grid = (a.M + kLnRowsPerBlock - 1) / kLnRowsPerBlock;
   if (grid == 0) return cudaSuccess;
   if (a.u_bf16)
-    ln_modulate_kernel<true><<<grid, 32 * kLnRowsPerBlock, 0, st>>>(a);
-  else
-    ln_modulate_kernel<false><<<grid, 32 * kLnRowsPerBlock, 0, st>>>(a);
-  return cudaGetLastError();
+    return launch_kernel(ln_modulate_kernel<true>, dim3(grid), dim3(32 * kLnRowsPerBlock), 0, st, a);
+  return launch_kernel(ln_modulate_kernel<false>, dim3(grid), dim3(32 * kLnRowsPerBlock), 0, st, a);
 }
 
 // ============================================================================ f32 GEMM
@@ -281,6 +293,8 @@ __device__ __forceinline__ void simt_epilogue(int epi, const EpiArgs& ea, int m,
 
 __global__ void __launch_bounds__(256) gemm_simt_kernel(int epi, const float* __restrict__ A,
                                                         const float* __restrict__ B, int K, EpiArgs ea) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -319,12 +333,13 @@ cudaError_t launch_gemm_simt(int epi, const float* A, const float* B, int M, int
                              cudaStream_t st) {
   dim3 grid((N + 63) / 64, (M + 63) / 64);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
-  gemm_simt_kernel<<<grid, 256, 0, st>>>(epi, A, B, K, ea);
-  return cudaGetLastError();
+  return launch_kernel(gemm_simt_kernel, grid, dim3(256), 0, st, epi, A, B, K, ea);
 }
 
 // ============================================================================ f32 QK-norm + RoPE
 __global__ void qknorm_rope_kernel(QkNormArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // one warp per (which, rh, tok)
   const int lane = threadIdx.x & 31;
   const int total = 2 * a.RH * a.T;
@@ -355,8 +370,7 @@ __global__ void qknorm_rope_kernel(QkNormArgs a) {
 
 cudaError_t launch_qknorm_rope_f32(const QkNormArgs& a, cudaStream_t st) {
   const int rows = 2 * a.RH * a.T;
-  qknorm_rope_kernel<<<(rows + 7) / 8, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(qknorm_rope_kernel, dim3((rows + 7) / 8), dim3(256), 0, st, a);
 }
 
 // ============================================================================ SIMT attention
@@ -364,6 +378,8 @@ cudaError_t launch_qknorm_rope_f32(const QkNormArgs& a, cudaStream_t st) {
 // shared memory; online softmax in base 2 with the 1/sqrt(dh) scale folded into q.
 template <int DH, bool BF16>
 __global__ void __launch_bounds__(128) attn_simt_kernel(AttnArgs a) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float Ks[32][DH];
   __shared__ float Vs[32][DH];
   const int rh = blockIdx.y;
@@ -446,11 +462,11 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnArgs a) {
 cudaError_t launch_attention_simt(const AttnArgs& a, cudaStream_t st) {
   dim3 grid((a.T + 127) / 128, a.R * a.H);
   if (a.dh == 64) {
-    if (a.bf16) attn_simt_kernel<64, true><<<grid, 128, 0, st>>>(a);
-    else attn_simt_kernel<64, false><<<grid, 128, 0, st>>>(a);
+    return a.bf16 ? launch_kernel(attn_simt_kernel<64, true>, grid, dim3(128), 0, st, a)
+                  : launch_kernel(attn_simt_kernel<64, false>, grid, dim3(128), 0, st, a);
   } else if (a.dh == 72) {
-    if (a.bf16) attn_simt_kernel<72, true><<<grid, 128, 0, st>>>(a);
-    else attn_simt_kernel<72, false><<<grid, 128, 0, st>>>(a);
+    return a.bf16 ? launch_kernel(attn_simt_kernel<72, true>, grid, dim3(128), 0, st, a)
+                  : launch_kernel(attn_simt_kernel<72, false>, grid, dim3(128), 0, st, a);
   } else {
     return cudaErrorInvalidValue;
   }
@@ -463,6 +479,8 @@ cudaError_t launch_attention_simt(const AttnArgs& a, cudaStream_t st) {
 // are decoded and combined as z_null + s (z_cond - z_null) before the scatter to
 // out[b, c, f*pt+it, i*ph+ih, j*pw+iw] with p = ((it*ph + ih)*pw + iw)*Cout + c.
 __global__ void decode_cfg_kernel(DecodeArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float su[];  // [2][d]
   const int tau = blockIdx.x, b = blockIdx.y;
   const int rows = a.guided ? 2 : 1;
@@ -505,8 +523,7 @@ __global__ void decode_cfg_kernel(DecodeArgs a) {
 cudaError_t launch_decode_cfg(const DecodeArgs& a, cudaStream_t st) {
   dim3 grid(a.T, a.B);
   const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float);
-  decode_cfg_kernel<<<grid, 256, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(decode_cfg_kernel, grid, dim3(256), smem, st, a);
 }
 
 // ============================================================================ set-up tables

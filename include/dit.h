@@ -154,8 +154,10 @@ void dit_destroy(dit_handle* h);
 
 /* Option switches (test use).  DIT_OPT_FORCE_GUIDANCE = 1 makes dit_forward run the
    2B guided rows even at cfg_scale == 1 (so e(null) + 1*(e(y)-e(null)) is returned).
-   DIT_OPT_USE_GRAPH = 0/1 disables / enables CUDA-graph replay of the forward. */
-enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2 };
+   DIT_OPT_USE_GRAPH = 0/1 disables / enables CUDA-graph replay of the forward.
+   DIT_OPT_OVERLAP_LAUNCH = 0/1 (process-wide, default 1): launch each kernel with
+   programmatic dependent launch so its set-up overlaps the tail of the previous one. */
+enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2, DIT_OPT_OVERLAP_LAUNCH = 3 };
 dit_status dit_set_option(dit_handle* h, int option, int value);
 
 /*
