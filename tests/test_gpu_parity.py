@@ -243,3 +243,23 @@ def test_host_side_errors_launch_nothing():
         m.forward(d["x"], d["t"], d["y"], 1.0)
     assert e.value.code == binding.DIT_ERR_INVALID_ARG
     m.close()
+
+
+# ----------------------------------------------------------------------------- full-size workloads
+# The benchmark's launch configuration (standard weights/inputs, full batch) on the GPU;
+# the oracle recomputes one sampled sample (rows of a batch are independent, so sample
+# b of the batched GPU output must equal the oracle run on sample b alone).
+@pytest.mark.parametrize("cfg", [S.DIT_XL2_CFG256, S.DIT_XL2_CFG512, S.VIDEO_RF], ids=["xl2_cfg256", "xl2_cfg512", "video_rf"])
+def test_full_size_sampled_parity(cfg):
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    got = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    assert m.sync_status() == binding.DIT_OK
+    m.close()
+    b = cfg.batch - 1   # the last sample: its guided partner is the last row of the batch
+    want = O.forward(cfg, S.weight_dict(cfg, W), inp["x"][b:b + 1], inp["t"][b:b + 1], inp["y"][b:b + 1])
+    assert_parity(cfg, got[b:b + 1], want, cfg.name)
+    # every sample: finite and of the expected shape
+    assert got.shape == cfg.out_shape() and np.all(np.isfinite(got))
