@@ -33,6 +33,9 @@ import dit_synth as S  # noqa: E402
 METRIC = "DiT-XL/2 bf16 fwd tokens/sec on 1 B200; % of dense BF16 tensor peak"
 CFG = S.DIT_XL2_CFG256
 L2_FLUSH_BYTES = 256 << 20
+# DRAM bytes (read + write) of one launch of each kernel, from the cold-cache ncu captures
+# summarised in profiles/xl2_cfg256_kernels_ncu.md; set to None when a kernel changes.
+TRAFFIC_BYTES = {"fc1": 60.0e6, "fc2": 130.7e6, "qkv": 46.0e6, "proj": 184.2e6, "attn": 65.6e6, "ln": 93.9e6}
 # fallback peaks (used only when MEASURED_PEAKS.json is absent)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -309,13 +312,13 @@ def main():
     if per.get(top, 0) > 0:
         ach = per[top] / avg_s / 1e12
         roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": sustained, "unit": "TFLOP/s",
-                "frac": ach / sustained, "traffic": None,
+                "frac": ach / sustained, "traffic": TRAFFIC_BYTES.get(top),
                 "peak_source": f"{pk_kind} bf16 dense, sustained (cuBLAS 8192^3 loop)",
                 "avg_launch_us": avg_s * 1e6, "flops_per_launch": per[top]}
     else:
         ach = ln_bytes(cfg) / avg_s / 1e9
         roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / pk["hbm_gbs"], "traffic": None, "peak_source": f"{pk_kind} copy bandwidth",
+                "frac": ach / pk["hbm_gbs"], "traffic": TRAFFIC_BYTES.get(top), "peak_source": f"{pk_kind} copy bandwidth",
                 "avg_launch_us": avg_s * 1e6}
     kernels = {k: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
                for k, v in kinds.items()}
