@@ -1,23 +1,27 @@
-// Tensor-core flash attention for sm_100a (full, non-causal, one head per CTA row).
+// Tensor-core flash attention for sm_100a (full, non-causal), persistent.
 //
-// O = softmax(Q K^T / sqrt(dh)) V for a 128-query tile of one (sample row, head):
-//   warp 0   one thread loads Q once, then K_j and V_j^T into two-stage rings (TMA,
-//            no multicast); a stage is refilled as soon as the MMA that read it
-//            completed (polled without blocking, so the K and V streams never wait on
-//            each other).  For T <= 256 every tile is requested at the start.
-//   warp 1   allocates 256 TMEM columns (S: 0..127, O: 128..) and one thread issues
-//            S_j = Q K_j^T (M=128, N=128, K=dh padded to 80, both operands in shared
-//            memory) and O += P_j V_j (M=128, N=DP, K=128) with P_j read from TMEM.
-//   warps 2-5 one query row per thread: S_j from TMEM into registers, online softmax
-//            in base 2 with lazy O rescaling (only when the running max grows by more
-//            than 2^8), P_j as packed bf16 written back over the first 64 columns of
-//            S (tcgen05.st), final O / l to global memory.
-// Two CTAs fit on one SM (about 102 KB shared memory and 256 TMEM columns each), so
-// one CTA's softmax overlaps the other's MMAs.
+// O = softmax(Q K^T / sqrt(dh)) V.  One CTA per SM walks work items; an item is a pair
+// of 128-query tiles of one (sample row, head), handled by two softmax warpgroups.
+//   warp 0    one thread streams Q (per item) and K_n / V_n^T (per key tile, two-stage
+//             rings) with TMA, no multicast; each buffer is refilled as soon as the MMA
+//             that read it completed (polled without blocking).
+//   warp 1    allocates all 512 TMEM columns (S_0, S_1, O_0, O_1) and one thread issues
+//             S_g = Q_g K_n^T (M=128, N=128, K = dh padded to 80: a 128B- and a
+//             32B-swizzled operand) and O_g += P_g V_n (M=128, N=DP, K=128).  The Q K^T of
+//             key tile n+1 is issued before the P V of tile n, so the tensor cores run
+//             while the softmax works.
+//   warps 4-7, 8-11  softmax of query group 0 / 1 (register budget raised with setmaxnreg,
+//             taken from warpgroup 0), one query row per thread: S from TMEM
+//             into registers (then S is released), online softmax in base 2 with lazy
+//             O rescaling (only when the running max grows by more than 2^8), P as bf16 in
+//             128B-swizzled shared memory, and at the end of an item O / l through a
+//             shared-memory staging tile and one TMA store (O is released as soon as it is
+//             in registers).
+// Every mbarrier wait is bounded.
 //
-// Layouts: q, k [R*H, Tpad, DP] bf16 (rows of one head contiguous, head dim padded
-// with zeros to DP = 80 for dh = 72); v transposed [R*H, DP, Tpad]; padded key rows
-// are zero and masked to -inf in the last key tile.  o [R*T, d] bf16, token-major.
+// Layouts: q, k [R*H, Tpad, DP] bf16 (rows of one head contiguous, head dim padded with
+// zeros to DP = 80 for dh = 72); v transposed [R*H, DP, Tpad]; padded key rows are zero
+// and masked to -inf in the last key tile.  o [R*T, d] bf16, token-major.
 #include <math.h>
 
 #include "common.cuh"
@@ -34,25 +38,49 @@ struct AttnCfg {
   static constexpr int QK_TILE = MAIN + TAILB;          // one Q or K tile
   static constexpr int V_ATOM = DP * 128;               // DP rows x 64 keys
   static constexpr int V_TILE = 2 * V_ATOM;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + QK_TILE;         // two K stages
+  static constexpr int P_TILE = 2 * MAIN;               // 128 queries x 128 keys bf16
+  static constexpr int O_ROW = DH * 2;                  // bytes of one output row
+  static constexpr bool O_SW128 = O_ROW == 128;         // 128B-swizzled staging (else rows packed)
+  static constexpr int O_TILE = (128 * O_ROW + 1023) / 1024 * 1024;
+  static constexpr int OFF_Q = 0;                       // Q of both query tiles of the item
+  static constexpr int OFF_K = OFF_Q + 2 * QK_TILE;     // two K stages
   static constexpr int OFF_V = OFF_K + 2 * QK_TILE;     // two V^T stages
-  static constexpr int OFF_BAR = OFF_V + 2 * V_TILE;
-  static constexpr int SMEM = OFF_BAR + 128 + 1024;
-  static constexpr int TMEM_COLS = 256;
-  static constexpr int O_COL = 128;
-  static_assert(QK_TILE % 1024 == 0 && V_ATOM % 1024 == 0, "1024-byte aligned tiles");
-  static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
+  static constexpr int OFF_P = OFF_V + 2 * V_TILE;      // P of both query tiles
+  static constexpr int OFF_O = OFF_P + 2 * P_TILE;      // output staging of both query tiles
+  static constexpr int OFF_BAR = OFF_O + 2 * O_TILE;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int TMEM_COLS = 512;                 // S0, S1, O0, O1 (128 columns each)
+  static constexpr int THREADS = 384;                   // warpgroup 0: loads, MMA; 1, 2: softmax
+  static constexpr int REG_CTRL = 80, REG_SOFTMAX = 200;
+  static constexpr int REG_POOL = 128 * REG_CTRL + 256 * REG_SOFTMAX;  // must fit the launch allocation
+  static_assert(QK_TILE % 1024 == 0 && V_ATOM % 1024 == 0 && OFF_O % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(O_ROW % 16 == 0, "16-byte output rows");
+  static_assert(SMEM <= 232448, "shared memory");
 };
 
-// barriers: Q loaded; K / V^T stage full and empty (two stages each); S ready; P ready; P V done
-enum { B_Q = 0, B_KF0, B_KF1, B_KE0, B_KE1, B_VF0, B_VF1, B_VE0, B_VE1, B_S, B_P, B_O, B_COUNT };
+enum {
+  B_QF = 0, B_QE,                    // Q of the item loaded / free (all its Q K^T done)
+  B_KF0, B_KF1, B_KE0, B_KE1,        // K stages full / empty
+  B_VF0, B_VF1, B_VE0, B_VE1,        // V^T stages full / empty
+  B_S0, B_S1,                        // S_g ready
+  B_SF0, B_SF1,                      // S_g read into registers (count 128)
+  B_P0, B_P1,                        // P_g written (count 128)
+  B_O0, B_O1,                        // P_g V done
+  B_OF0, B_OF1,                      // O_g read by the epilogue (count 128)
+  B_OS0, B_OS1,                      // output staging of group g free (previous store read it)
+  B_OW0, B_OW1,                      // output staging of group g written (count 128)
+  B_COUNT
+};
 
+// Persistent flash attention.  A work item is a pair of 128-query tiles of one (sample
+// row, head); CTA b walks the items b, b + gridDim.x, ...  The key tiles of all its items
+// form one sequence that streams through the two-stage K / V^T rings.
 template <int DH>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQt,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKt,
-                   const __grid_constant__ CUtensorMap tmV, const AttnArgs a, int* status) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const AttnArgs a,
+                   int* status) {
   using C = AttnCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -62,12 +90,19 @@ __global__ void __launch_bounds__(192, 2)
 #define BAR(i) (bar0 + 8u * (i))
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rh = blockIdx.y;
-  const int qt = blockIdx.x;
-  const int nk = (a.T + 127) / 128;
+  const int nk = (a.T + 127) / 128;            // key tiles per item
+  const int nq = a.Tpad / 128;                 // query tiles per head
+  const int pairs = (nq + 1) / 2;              // items per head
+  const int items = a.R * a.H * pairs;
+  const int my_items = static_cast<int>(blockIdx.x) < items ? (items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int ntiles = my_items * nk;            // key tiles this CTA streams
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < B_COUNT; ++i) mbar_init(BAR(i), i == B_P ? 128 : 1);
+    for (int i = 0; i < B_COUNT; ++i) {
+      const bool all = i == B_SF0 || i == B_SF1 || i == B_P0 || i == B_P1 || i == B_OF0 || i == B_OF1 ||
+                       i == B_OW0 || i == B_OW1;
+      mbar_init(BAR(i), all ? 128 : 1);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -82,171 +117,294 @@ __global__ void __launch_bounds__(192, 2)
   pdl_trigger();
   pdl_wait();
 
-  if (warp == 0) {
-    if (lane == 0) {  // ---------------- loads: Q once; K_j and V_j^T into two-stage rings
+  // item li of this CTA -> (row*H + head, first query tile, query tiles in the item: 1 or 2)
+  auto item_of = [&](int li, int& rh, int& qt0, int& ng) {
+    const int it = static_cast<int>(blockIdx.x) + li * static_cast<int>(gridDim.x);
+    rh = it / pairs;
+    qt0 = (it - rh * pairs) * 2;
+    ng = qt0 + 1 < nq ? 2 : 1;
+  };
+
+  if (warp < 4) {
+    regs_dec<C::REG_CTRL>();
+    if (warp == 0 && lane == 0) {  // ---------- loads: Q per item; K_n and V_n^T through two-stage rings
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int qrow0 = rh * a.Tpad + qt * 128;
-      const int vrow0 = rh * C::DP;
-      mbar_arrive_expect_tx(BAR(B_Q), C::QK_TILE);
-      tma_load_2d(sbase + C::OFF_Q, &tmQ, BAR(B_Q), 0, qrow0);
-      if (C::TAIL) tma_load_2d(sbase + C::OFF_Q + C::MAIN, &tmQt, BAR(B_Q), 64, qrow0);
-      int jk = 0, jv = 0;
-      const uint64_t t0 = global_timer_ns();
-      while (jk < nk || jv < nk) {
-        // stage j&1 is free once the MMA that read its previous tile (j-2) completed
-        if (jk < nk && (jk < 2 || mbar_test(BAR(B_KE0 + (jk & 1)), ((jk >> 1) & 1) ^ 1u))) {
-          const uint32_t dst = sbase + C::OFF_K + (jk & 1) * C::QK_TILE;
-          const int krow0 = rh * a.Tpad + jk * 128;
-          mbar_arrive_expect_tx(BAR(B_KF0 + (jk & 1)), C::QK_TILE);
-          tma_load_2d(dst, &tmK, BAR(B_KF0 + (jk & 1)), 0, krow0);
-          if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmKt, BAR(B_KF0 + (jk & 1)), 64, krow0);
-          ++jk;
+      int lq = 0, nkl = 0, nvl = 0;
+      uint64_t t0 = global_timer_ns();  // time of the last issued load
+      while (lq < my_items || nkl < ntiles || nvl < ntiles) {
+        const int progress = lq + nkl + nvl;
+        // Q of item lq once every Q K^T of item lq-1 completed
+        if (lq < my_items && (lq == 0 || mbar_test(BAR(B_QE), (lq - 1) & 1))) {
+          int rh, qt0, ng;
+          item_of(lq, rh, qt0, ng);
+          mbar_arrive_expect_tx(BAR(B_QF), ng * C::QK_TILE);
+          for (int g = 0; g < ng; ++g) {
+            const int row0 = rh * a.Tpad + (qt0 + g) * 128;
+            const uint32_t dst = sbase + C::OFF_Q + g * C::QK_TILE;
+            tma_load_2d(dst, &tmQ, BAR(B_QF), 0, row0);
+            if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmQt, BAR(B_QF), 64, row0);
+          }
+          ++lq;
         }
-        if (jv < nk && (jv < 2 || mbar_test(BAR(B_VE0 + (jv & 1)), ((jv >> 1) & 1) ^ 1u))) {
-          const uint32_t dst = sbase + C::OFF_V + (jv & 1) * C::V_TILE;
-          mbar_arrive_expect_tx(BAR(B_VF0 + (jv & 1)), C::V_TILE);
-          tma_load_2d(dst, &tmV, BAR(B_VF0 + (jv & 1)), jv * 128, vrow0);
-          tma_load_2d(dst + C::V_ATOM, &tmV, BAR(B_VF0 + (jv & 1)), jv * 128 + 64, vrow0);
-          ++jv;
+        // stage n & 1 is free once the MMA that read tile n-2 from it completed
+        if (nkl < ntiles && (nkl < 2 || mbar_test(BAR(B_KE0 + (nkl & 1)), ((nkl >> 1) & 1) ^ 1u))) {
+          int rh, qt0, ng;
+          item_of(nkl / nk, rh, qt0, ng);
+          const int krow0 = rh * a.Tpad + (nkl % nk) * 128;
+          const uint32_t dst = sbase + C::OFF_K + (nkl & 1) * C::QK_TILE;
+          mbar_arrive_expect_tx(BAR(B_KF0 + (nkl & 1)), C::QK_TILE);
+          tma_load_2d(dst, &tmK, BAR(B_KF0 + (nkl & 1)), 0, krow0);
+          if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmKt, BAR(B_KF0 + (nkl & 1)), 64, krow0);
+          ++nkl;
         }
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (nvl < ntiles && (nvl < 2 || mbar_test(BAR(B_VE0 + (nvl & 1)), ((nvl >> 1) & 1) ^ 1u))) {
+          int rh, qt0, ng;
+          item_of(nvl / nk, rh, qt0, ng);
+          const int kcol0 = (nvl % nk) * 128;
+          const uint32_t dst = sbase + C::OFF_V + (nvl & 1) * C::V_TILE;
+          mbar_arrive_expect_tx(BAR(B_VF0 + (nvl & 1)), C::V_TILE);
+          tma_load_2d(dst, &tmV, BAR(B_VF0 + (nvl & 1)), kcol0, rh * C::DP);
+          tma_load_2d(dst + C::V_ATOM, &tmV, BAR(B_VF0 + (nvl & 1)), kcol0 + 64, rh * C::DP);
+          ++nvl;
+        }
+        const uint64_t now = global_timer_ns();
+        if (lq + nkl + nvl != progress) {
+          t0 = now;
+        } else if (now - t0 > kWaitLimitNs) {
           record_status(status, DIT_ERR_DEVICE_TIMEOUT);
           break;
         }
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {  // ---------------- MMA issuer
+    } else if (warp == 1 && lane == 0) {  // ---------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, C::DP);
-      const uint32_t tS = tmem_base;
-      const uint32_t tO = tmem_base + C::O_COL;
-      bool ok = mbar_wait(BAR(B_Q), 0, status);
-      for (int j = 0; j < nk && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t use = (j >> 1) & 1;
-        ok = mbar_wait(BAR(B_KF0 + st), use, status);
-        // S (and P_{j-1}, which lives in S) may be overwritten once P_{j-1} V_{j-1} completed
-        if (ok && j > 0) ok = mbar_wait(BAR(B_O), (j - 1) & 1, status);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kb = sbase + C::OFF_K + st * C::QK_TILE;
+      int qk_cnt[2] = {0, 0};  // Q K^T issued per query group
+      int pv_cnt[2] = {0, 0};  // P V issued per query group
+      int it_cnt[2] = {0, 0};  // items whose first P V was issued, per group
+      // S_g = Q_g K_n^T for every query group of tile n
+      auto issue_qk = [&](int n) -> bool {
+        const int li = n / nk, j = n - li * nk;
+        int rh, qt0, ng;
+        item_of(li, rh, qt0, ng);
+        if (j == 0 && !mbar_wait(BAR(B_QF), li & 1, status)) return false;
+        if (!mbar_wait(BAR(B_KF0 + (n & 1)), (n >> 1) & 1, status)) return false;
+        const uint32_t kb = sbase + C::OFF_K + (n & 1) * C::QK_TILE;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16_ss(tS, sdesc_k_sw128(sbase + C::OFF_Q + k * 32), sdesc_k_sw128(kb + k * 32), idesc_s,
-                      k > 0 ? 1u : 0u);
-        if (C::TAIL) mma_bf16_ss(tS, sdesc_k_sw32(sbase + C::OFF_Q + C::MAIN), sdesc_k_sw32(kb + C::MAIN), idesc_s, 1u);
-        mma_commit(BAR(B_S));
-        mma_commit(BAR(B_KE0 + st));
-        // O += P_j V_j: P_j (bf16, 64 TMEM columns over S) as the A operand
-        ok = mbar_wait(BAR(B_P), j & 1, status) && mbar_wait(BAR(B_VF0 + st), use, status);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t vb = sbase + C::OFF_V + st * C::V_TILE;
+        for (int g = 0; g < 2; ++g) {
+          if (g >= ng) break;
+          // S_g may be overwritten once the softmax of group g has read its previous tile
+          if (qk_cnt[g] > 0 && !mbar_wait(BAR(B_SF0 + g), (qk_cnt[g] - 1) & 1, status)) return false;
+          tc_fence_after();
+          const uint32_t qb = sbase + C::OFF_Q + g * C::QK_TILE;
+          const uint32_t tS = tmem_base + g * 128;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_bf16_ts(tO, tS + 8 * k, sdesc_k_sw128(vb + (k >> 2) * C::V_ATOM + (k & 3) * 32), idesc_o,
-                      (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(BAR(B_O));
-        mma_commit(BAR(B_VE0 + st));
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(tS, sdesc_k_sw128(qb + k * 32), sdesc_k_sw128(kb + k * 32), idesc_s, k > 0 ? 1u : 0u);
+          if (C::TAIL) mma_bf16_ss(tS, sdesc_k_sw32(qb + C::MAIN), sdesc_k_sw32(kb + C::MAIN), idesc_s, 1u);
+          mma_commit(BAR(B_S0 + g));
+          ++qk_cnt[g];
+        }
+        mma_commit(BAR(B_KE0 + (n & 1)));
+        if (j == nk - 1) mma_commit(BAR(B_QE));
+        return true;
+      };
+      // O_g (+)= P_g V_n for every query group of tile n
+      auto issue_pv = [&](int n) -> bool {
+        const int li = n / nk, j = n - li * nk;
+        int rh, qt0, ng;
+        item_of(li, rh, qt0, ng);
+        if (!mbar_wait(BAR(B_VF0 + (n & 1)), (n >> 1) & 1, status)) return false;
+        const uint32_t vb = sbase + C::OFF_V + (n & 1) * C::V_TILE;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          if (g >= ng) break;
+          if (!mbar_wait(BAR(B_P0 + g), pv_cnt[g] & 1, status)) return false;
+          // a new item overwrites O_g: its epilogue for the previous item must have read it
+          if (j == 0 && it_cnt[g] > 0 && !mbar_wait(BAR(B_OF0 + g), (it_cnt[g] - 1) & 1, status)) return false;
+          tc_fence_after();
+          const uint32_t pb = sbase + C::OFF_P + g * C::P_TILE;
+          const uint32_t tO = tmem_base + 256 + g * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mma_bf16_ss(tO, sdesc_k_sw128(pb + (k >> 2) * C::MAIN + (k & 3) * 32),
+                        sdesc_k_sw128(vb + (k >> 2) * C::V_ATOM + (k & 3) * 32), idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+          mma_commit(BAR(B_O0 + g));
+          ++pv_cnt[g];
+          if (j == 0) ++it_cnt[g];
+        }
+        mma_commit(BAR(B_VE0 + (n & 1)));
+        return true;
+      };
+      // Q K^T of the next key tile goes in before P V of the current one, so the tensor
+      // cores work while the softmax runs; across an item boundary P V goes first (the
+      // next item's Q is loaded only after the current item's last Q K^T).
+      int n_qk = 0;
+      bool ok = true;
+      for (int n = 0; n < ntiles && ok; ++n) {
+        while (ok && (n_qk <= n || (n_qk == n + 1 && n_qk < ntiles && n_qk % nk != 0))) ok = issue_qk(n_qk++);
+        if (ok) ok = issue_pv(n);
       }
     }
-  } else {  // ------------------------------------------ softmax / output warps 2..5
+  } else {  // ------------------------------- softmax / output: group g = warps 4-7 / 8-11
+    regs_inc<C::REG_SOFTMAX>();
+    const int g = (warp - 4) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;  // query row within the tile
-    const uint32_t tS = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t tO = tS + C::O_COL;
+    const uint32_t tS = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + g * 128;
+    const uint32_t tO = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + 256 + g * 128;
     const float sc = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
-    float m_ref = -INFINITY, l = 0.f;
+    const uint32_t prow = sbase + C::OFF_P + g * C::P_TILE + r * 128;
+    const uint32_t r7 = static_cast<uint32_t>(r & 7);
+    const uint32_t ostage = sbase + C::OFF_O + g * C::O_TILE;
+    const bool issuer = q == 0 && lane == 0;  // issues this group's output stores
+    int cnt = 0;  // tiles of this group processed
+    int ne = 0;   // items of this group finished
     bool ok = true;
-    for (int j = 0; j < nk; ++j) {
-      ok = mbar_wait(BAR(B_S), j & 1, status);
+    for (int li = 0; li < my_items && ok; ++li) {
+      int rh, qt0, ng;
+      item_of(li, rh, qt0, ng);
+      if (g >= ng) continue;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < nk; ++j, ++cnt) {
+        ok = mbar_wait(BAR(B_S0 + g), cnt & 1, status);
+        __syncwarp();
+        if (__any_sync(0xffffffffu, !ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s + c * 32);
+        tmem_ld_wait<128>(s);
+        tc_fence_before();
+        mbar_arrive(BAR(B_SF0 + g));  // S_g is in registers: the next Q K^T may overwrite it
+
+        // row maximum with eight independent partial maxima
+        const int kvalid = a.T - j * 128;
+        if (kvalid < 128) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i >= kvalid) s[i] = __float_as_uint(-INFINITY);
+        }
+        float mp[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mp[e] = __uint_as_float(s[e]);
+#pragma unroll
+        for (int i = 8; i < 128; i += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(s[i + e]));
+        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        const float m_new = fmaxf(m_ref, mx * sc);
+        bool o_ready = false;  // the previous P V of this group has completed
+        if (j == 0) {
+          m_ref = m_new;
+        } else if (__any_sync(0xffffffffu, m_new - m_ref > 8.0f)) {
+          // lazy rescale: O moves to the new reference only when the maximum grew by more
+          // than 2^8; the previous P V must have completed first
+          const bool okw = mbar_wait(BAR(B_O0 + g), (cnt - 1) & 1, status);
+          __syncwarp();
+          if (__any_sync(0xffffffffu, !okw)) {
+            ok = false;
+            break;
+          }
+          o_ready = true;
+          tc_fence_after();
+          const float alpha = ex2_approx(m_ref - m_new);
+#pragma unroll
+          for (int c = 0; c < C::DP / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tO + c * 16, o);
+            tmem_ld_wait<16>(o);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(tO + c * 16, o);
+          }
+          tmem_st_wait();
+          l *= alpha;
+          m_ref = m_new;
+        }
+        if (cnt > 0 && !o_ready) {  // the P buffer is free once the previous P V completed
+          const bool okw = mbar_wait(BAR(B_O0 + g), (cnt - 1) & 1, status);
+          __syncwarp();
+          if (__any_sync(0xffffffffu, !okw)) {
+            ok = false;
+            break;
+          }
+        }
+        // P = 2^(s*sc - m_ref) as bf16 in the 128B-swizzled K-major layout; four partial sums
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(s[ch * 8 + 2 * e]), sc, -m_ref));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(s[ch * 8 + 2 * e + 1]), sc, -m_ref));
+            rs[e] += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          st_shared_v4(prow + (ch >> 3) * C::MAIN + (((ch & 7) ^ r7) << 4), pk[0], pk[1], pk[2], pk[3]);
+        }
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(B_P0 + g));
+      }
+      if (!ok) break;
+      // item epilogue: O_g / l through shared memory to global memory (one TMA store)
+      const bool okw = mbar_wait(BAR(B_O0 + g), (cnt - 1) & 1, status);
       __syncwarp();
-      if (__any_sync(0xffffffffu, !ok)) {
+      if (__any_sync(0xffffffffu, !okw)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t s[128];
+      uint32_t o[C::DP];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, s + c * 32);
-      tmem_ld_wait<128>(s);
-      const int kvalid = a.T - j * 128;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float v = __uint_as_float(s[i]);
-        if (i >= kvalid) v = -INFINITY;
-        s[i] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
-      }
-      const float m_new = fmaxf(m_ref, mx * sc);
-      if (j == 0) {
-        m_ref = m_new;
-      } else if (__any_sync(0xffffffffu, m_new - m_ref > 8.0f)) {
-        // lazy rescale: O only moves to the new reference when the maximum grew by more
-        // than 2^8 (P_{j-1} V_{j-1} has completed: Q K_j^T was issued after it)
-        const float alpha = ex2_approx(m_ref - m_new);
-#pragma unroll
-        for (int c = 0; c < C::DP / 16; ++c) {
-          uint32_t o[16];
-          tmem_ld16(tO + c * 16, o);
-          tmem_ld_wait<16>(o);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st16(tO + c * 16, o);
-        }
-        l *= alpha;
-        m_ref = m_new;
-      }
-      // P = 2^(s*sc - m_ref) as bf16 pairs, written over the first 64 columns of S
-      float rs = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * e]), sc, -m_ref));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[half * 64 + 2 * e + 1]), sc, -m_ref));
-          rs += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + half * 32, pk);
-      }
-      tmem_st_wait();
-      l += rs;
+      for (int c = 0; c < C::DP / 16; ++c) tmem_ld16(tO + c * 16, *reinterpret_cast<uint32_t(*)[16]>(o + c * 16));
+      tmem_ld_wait<C::DP>(o);
       tc_fence_before();
-      mbar_arrive(BAR(B_P));
-    }
-    if (ok) {
-      const bool okw = mbar_wait(BAR(B_O), (nk - 1) & 1, status);
+      mbar_arrive(BAR(B_OF0 + g));  // O_g is in registers: the next item may overwrite it
+      if (issuer) {
+        bulk_wait_read_all();  // the previous store has finished reading the staging tile
+        mbar_arrive(BAR(B_OS0 + g));
+      }
+      const bool okf = mbar_wait(BAR(B_OS0 + g), ne & 1, status);
       __syncwarp();
-      if (!__any_sync(0xffffffffu, !okw)) {
-        tc_fence_after();
-        uint32_t o[C::DP];
+      if (__any_sync(0xffffffffu, !okf)) {
+        ok = false;
+        break;
+      }
+      const float inv = 1.0f / l;
+      const uint32_t orow = ostage + r * C::O_ROW;
 #pragma unroll
-        for (int c = 0; c < C::DP / 16; ++c) tmem_ld16(tO + c * 16, *reinterpret_cast<uint32_t(*)[16]>(o + c * 16));
-        tmem_ld_wait<C::DP>(o);
-        const int qi = qt * 128 + r;
-        if (qi < a.T) {
-          const float inv = 1.0f / l;
+      for (int c = 0; c < DH / 8; ++c) {
+        const uint32_t off = C::O_SW128 ? ((static_cast<uint32_t>(c) ^ r7) << 4) : static_cast<uint32_t>(c) * 16u;
+        st_shared_v4(orow + off,
+                     pack_bf16x2(__uint_as_float(o[c * 8 + 0]) * inv, __uint_as_float(o[c * 8 + 1]) * inv),
+                     pack_bf16x2(__uint_as_float(o[c * 8 + 2]) * inv, __uint_as_float(o[c * 8 + 3]) * inv),
+                     pack_bf16x2(__uint_as_float(o[c * 8 + 4]) * inv, __uint_as_float(o[c * 8 + 5]) * inv),
+                     pack_bf16x2(__uint_as_float(o[c * 8 + 6]) * inv, __uint_as_float(o[c * 8 + 7]) * inv));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(B_OW0 + g));
+      if (issuer) {
+        if (!mbar_wait(BAR(B_OW0 + g), ne & 1, status)) {
+          ok = false;
+        } else {
           const int row = rh / a.H, head = rh - row * a.H;
-          uint16_t* dst = static_cast<uint16_t*>(a.o) + (static_cast<size_t>(row) * a.T + qi) * a.d + head * DH;
-#pragma unroll
-          for (int c = 0; c < DH / 8; ++c) {
-            uint4 pk;
-            pk.x = pack_bf16x2(__uint_as_float(o[c * 8 + 0]) * inv, __uint_as_float(o[c * 8 + 1]) * inv);
-            pk.y = pack_bf16x2(__uint_as_float(o[c * 8 + 2]) * inv, __uint_as_float(o[c * 8 + 3]) * inv);
-            pk.z = pack_bf16x2(__uint_as_float(o[c * 8 + 4]) * inv, __uint_as_float(o[c * 8 + 5]) * inv);
-            pk.w = pack_bf16x2(__uint_as_float(o[c * 8 + 6]) * inv, __uint_as_float(o[c * 8 + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c * 8) = pk;
-          }
+          tma_store_3d(&tmO, ostage, head * DH, (qt0 + g) * 128, row);  // rows past T are clipped
+          bulk_commit_group();
         }
       }
+      ++ne;
     }
+    if (issuer) bulk_wait_all();
   }
+  __syncwarp();  // lane-divergent roles reconverge before the block barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -256,10 +414,12 @@ __global__ void __launch_bounds__(192, 2)
 #undef BAR
 }
 
-bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* v, int RH, int Tpad, int DP) {
-  const uint64_t qrows = static_cast<uint64_t>(RH) * Tpad;
+bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* v, void* o, int R, int H, int T,
+                         int Tpad, int dh, int DP, int d) {
+  const uint64_t qrows = static_cast<uint64_t>(R) * H * Tpad;
   bool ok = make_tmap_bf16(&m->q, q, qrows, DP, 64, 128, 128) && make_tmap_bf16(&m->k, k, qrows, DP, 64, 128, 128) &&
-            make_tmap_bf16(&m->v, v, static_cast<uint64_t>(RH) * DP, Tpad, 64, DP, 128);
+            make_tmap_bf16(&m->v, v, static_cast<uint64_t>(R) * H * DP, Tpad, 64, DP, 128) &&
+            make_tmap_bf16_3d(&m->o, o, d, T, R, dh, 128, dh * 2 == 128 ? 128 : 0);
   if (DP > 64)
     ok = ok && make_tmap_bf16(&m->qt, q, qrows, DP, 16, 128, 32) && make_tmap_bf16(&m->kt, k, qrows, DP, 16, 128, 32);
   else {
@@ -272,14 +432,25 @@ bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* 
 template <int DH>
 static cudaError_t launch_dh(const AttnArgs& a, const AttnMaps& mp, int* status, cudaStream_t st) {
   using C = AttnCfg<DH>;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static int num_sms = 0;
+  if (num_sms == 0) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    // the register split (setmaxnreg) must fit in the launch allocation, or it would wait forever
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attn_tc_kernel<DH>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * C::THREADS < C::REG_POOL) return cudaErrorInvalidConfiguration;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return cudaErrorInvalidDevice;
   }
-  dim3 grid(a.Tpad / 128, a.R * a.H);
-  return launch_kernel(attn_tc_kernel<DH>, grid, dim3(192), C::SMEM, st, mp.q, mp.qt, mp.k, mp.kt, mp.v, a, status);
+  const int nq = a.Tpad / 128;
+  const int items = a.R * a.H * ((nq + 1) / 2);
+  const int grid = items < num_sms ? items : num_sms;
+  if (grid == 0) return cudaSuccess;
+  return launch_kernel(attn_tc_kernel<DH>, dim3(grid), dim3(C::THREADS), C::SMEM, st, mp.q, mp.qt, mp.k, mp.kt, mp.v,
+                       mp.o, a, status);
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, const AttnMaps& maps, int* status, cudaStream_t st) {

@@ -394,7 +394,7 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
     ok = ok && make_tmap_bf16_kmajor(&H->tb_u, H->u, g.Mmax, d, 256);
     ok = ok && make_tmap_bf16_kmajor(&H->tb_o, H->o, g.Mmax, d, 256);
     ok = ok && make_tmap_bf16_kmajor(&H->tb_g, H->gbuf, g.Mmax, mlp, 256);
-    ok = ok && make_attention_maps(&H->attn_maps, H->q, H->k, H->v, g.Rmax * cfg->heads, g.Tpad, g.DP);
+    ok = ok && make_attention_maps(&H->attn_maps, H->q, H->k, H->v, H->o, g.Rmax, cfg->heads, g.T, g.Tpad, g.dh, g.DP, d);
     for (int i = 0; i < N && ok; ++i) {
       BlockW& b = H->blk[i];
       ok = make_tmap_bf16_kmajor(&b.tm_qkv, b.qkv_w, 3 * d, d, g.headwise ? g.bn_qkv : 128) &&

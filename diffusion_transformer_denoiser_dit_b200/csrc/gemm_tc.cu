@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (epi_staged<EPI>() && lane == 0) bulk_wait_all();  // TMA stores of this warp are complete
   }
+  __syncwarp();  // lane-divergent roles reconverge before the block barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -228,6 +229,23 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 bool make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
                    uint32_t box_rows, int swizzle_bytes) {
   return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, rows, cols, box_cols, box_rows, swizzle_bytes);
+}
+
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                       uint32_t box1, int swizzle_bytes) {
+  PFN_encodeTiled_t fn = encode_fn();
+  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (d0 * 2) % 16 != 0 || box0 == 0 ||
+      box0 > 256 || box1 == 0 || box1 > 256 || (box0 * 2) % 16 != 0 ||
+      (swizzle_bytes > 0 && box0 * 2 > (uint32_t)swizzle_bytes))
+    return false;
+  CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows) {

@@ -60,6 +60,9 @@ cudaError_t launch_gemm_tc2(int epi, int block_n, const CUtensorMap* tmA, const 
 int gemm_tc2_supported_bn(int block_n);
 // Build a 2-D bf16 K-major tensor map: rows x K, box = box_rows x 64, 128-byte swizzle.
 bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
+// 3-d bf16 map: dims d0 (innermost) x d1 x d2, box box0 x box1 x 1, 128B swizzle or none.
+bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                       uint32_t box1, int swizzle_bytes);
 // General 2-D bf16 tensor map: rows x cols (cols contiguous), box box_rows x box_cols,
 // swizzle 128 / 64 / 32 bytes (0 = none).  The box row (box_cols * 2 bytes) must not
 // exceed the swizzle span.
@@ -119,11 +122,13 @@ struct AttnArgs {
 cudaError_t launch_attention_simt(const AttnArgs& a, cudaStream_t st);
 // Tensor maps of the tensor-core attention: q / k main (box 128 x 64, 128B swizzle),
 // q / k tail (head-dim columns 64..79, box 128 x 16, 32B swizzle; unused when dh = 64),
-// v (transposed, box DP x 64, 128B swizzle).
+// v (transposed, box DP x 64, 128B swizzle), o (output [R][T][d] as a 3-d map, box dh x 128 x 1,
+// so rows past T are clipped).
 struct AttnMaps {
-  CUtensorMap q, qt, k, kt, v;
+  CUtensorMap q, qt, k, kt, v, o;
 };
-bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* v, int RH, int Tpad, int DP);
+bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* v, void* o, int R, int H, int T,
+                         int Tpad, int dh, int DP, int d);
 cudaError_t launch_attention_tc(const AttnArgs& a, const AttnMaps& maps, int* status, cudaStream_t st);
 
 struct QkNormArgs {   // f32 path: RMSNorm + RoPE applied in place to q, k [R*H, T, dh]
