@@ -289,66 +289,73 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 128; ++i)
             if (i >= kvalid) s[i] = __float_as_uint(-INFINITY);
         }
-        float mp[8];
+        float mp[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mp[e] = __uint_as_float(s[e]);
+        for (int e = 0; e < 4; ++e) mp[e] = fmaxf(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1]));
 #pragma unroll
         for (int i = 8; i < 128; i += 8)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(s[i + e]));
-        const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+          for (int e = 0; e < 4; ++e) mp[e] = max3f(mp[e], __uint_as_float(s[i + 2 * e]), __uint_as_float(s[i + 2 * e + 1]));
+        const float mx = fmaxf(max3f(mp[0], mp[1], mp[2]), mp[3]);
         const float m_new = fmaxf(m_ref, mx * sc);
-        bool o_ready = false;  // the previous P V of this group has completed
+        // lazy rescale: the reference maximum moves (and O with it) only when the row maximum
+        // grew by more than 2^8
+        bool rescale = false;
+        float alpha = 1.f;
         if (j == 0) {
           m_ref = m_new;
         } else if (__any_sync(0xffffffffu, m_new - m_ref > 8.0f)) {
-          // lazy rescale: O moves to the new reference only when the maximum grew by more
-          // than 2^8; the previous P V must have completed first
+          rescale = true;
+          alpha = ex2_approx(m_ref - m_new);
+          m_ref = m_new;
+        }
+        // P = 2^(s*sc - m_ref) as packed bf16 in registers (paired f32 scaling and row sums)
+        uint32_t pk[64];
+        const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m_ref, -m_ref);
+        uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2), x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          rs2[i & 1] = f2_add(rs2[i & 1], f2_pack(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        // the previous P V must be complete before O is rescaled and the P buffer rewritten
+        if (cnt > 0) {
           const bool okw = mbar_wait(BAR(B_O0 + g), (cnt - 1) & 1, status);
           __syncwarp();
           if (__any_sync(0xffffffffu, !okw)) {
             ok = false;
             break;
           }
-          o_ready = true;
+        }
+        if (rescale) {
           tc_fence_after();
-          const float alpha = ex2_approx(m_ref - m_new);
 #pragma unroll
           for (int c = 0; c < C::DP / 16; ++c) {
             uint32_t o[16];
             tmem_ld16(tO + c * 16, o);
             tmem_ld_wait<16>(o);
+            const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            for (int i = 0; i < 16; i += 2)
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2),
+                        reinterpret_cast<float&>(o[i]), reinterpret_cast<float&>(o[i + 1]));
             tmem_st16(tO + c * 16, o);
           }
           tmem_st_wait();
           l *= alpha;
-          m_ref = m_new;
         }
-        if (cnt > 0 && !o_ready) {  // the P buffer is free once the previous P V completed
-          const bool okw = mbar_wait(BAR(B_O0 + g), (cnt - 1) & 1, status);
-          __syncwarp();
-          if (__any_sync(0xffffffffu, !okw)) {
-            ok = false;
-            break;
-          }
-        }
-        // P = 2^(s*sc - m_ref) as bf16 in the 128B-swizzled K-major layout; four partial sums
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        float r0, r1, r2, r3;
+        f2_unpack(rs2[0], r0, r1);
+        f2_unpack(rs2[1], r2, r3);
+        l += (r0 + r1) + (r2 + r3);
+        // P into the 128B-swizzled K-major layout the P V MMA reads
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(s[ch * 8 + 2 * e]), sc, -m_ref));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(s[ch * 8 + 2 * e + 1]), sc, -m_ref));
-            rs[e] += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          st_shared_v4(prow + (ch >> 3) * C::MAIN + (((ch & 7) ^ r7) << 4), pk[0], pk[1], pk[2], pk[3]);
-        }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        for (int ch = 0; ch < 16; ++ch)
+          st_shared_v4(prow + (ch >> 3) * C::MAIN + (((ch & 7) ^ r7) << 4), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2],
+                       pk[4 * ch + 3]);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_P0 + g));
