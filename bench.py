@@ -35,7 +35,7 @@ CFG = S.DIT_XL2_CFG256
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one launch of each kernel, from the cold-cache ncu captures
 # summarised in profiles/xl2_cfg256_kernels_ncu.md; set to None when a kernel changes.
-TRAFFIC_BYTES = {"fc1": 60.0e6, "fc2": 130.7e6, "qkv": 46.0e6, "proj": 184.2e6, "attn": None, "ln": 38.1e6}
+TRAFFIC_BYTES = {"fc1": 60.0e6, "fc2": 130.7e6, "qkv": 46.0e6, "proj": 184.2e6, "attn": 66.2e6, "ln": 38.1e6}
 # fallback peaks (used only when MEASURED_PEAKS.json is absent)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -201,10 +201,11 @@ def cpu_baseline(cfg, weights):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every kernel directly instead of replaying a CUDA graph")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -212,6 +213,7 @@ def main():
     import torch
     import torch.distributed as dist
     from diffusion_transformer_denoiser_dit_b200 import DiT
+    from diffusion_transformer_denoiser_dit_b200.binding import DIT_OPT_USE_GRAPH
 
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -222,6 +224,7 @@ def main():
     cfg = CFG
     weights = S.make_weights(cfg)
     model = DiT(cfg, weights)
+    model.set_option(DIT_OPT_USE_GRAPH, 0 if args.no_graph else 1)
     inp = S.make_inputs(cfg, seed=S.inputs_seed(cfg) + rank)
     x = torch.from_numpy(inp["x"]).cuda()
     t = torch.from_numpy(inp["t"]).cuda()
@@ -336,7 +339,8 @@ def main():
         "config": {"workload": workload_desc(cfg), "global_batch": cfg.batch * world, "rows_per_gpu": cfg.rows,
                    "tokens_per_step_per_gpu": tokens, "seq_len": cfg.tokens,
                    "l2": "flushed between timed steps (256 MB write outside the events)",
-                   "parallelism": f"replicas x{world} (weak scaling, no data-path collective)"},
+                   "parallelism": f"replicas x{world} (weak scaling, no data-path collective)",
+                   "launch": "direct launches" if args.no_graph else "CUDA graph replay of the whole forward"},
         "images_per_s": cfg.batch * world * args.steps / (total_ms / 1e3),
         "pct_of_bf16_peak": {"achieved_tflops": achieved_tf, "peak_tflops": sustained,
                              "frac": achieved_tf / sustained, "peak_source": f"{pk_kind} sustained",

@@ -152,6 +152,23 @@ struct dit_handle {
   CUtensorMap tb_u, tb_o, tb_g;     // activations as the B operand of the swapped GEMMs (box 256 rows)
   AttnMaps attn_maps;
   int force_guidance = 0;
+  // CUDA-graph replay of the whole forward (DIT_OPT_USE_GRAPH): one cached executable graph,
+  // valid for the exact pointers and parameters it was captured with
+  struct GraphKey {
+    const void *x, *t, *y;
+    float* out;
+    int B, R, depth;
+    bool guided, pdl;
+    float s;
+    bool operator==(const GraphKey& o) const {
+      return x == o.x && t == o.t && y == o.y && out == o.out && B == o.B && R == o.R && depth == o.depth &&
+             guided == o.guided && pdl == o.pdl && s == o.s;
+    }
+  };
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t gexec = nullptr;
+  GraphKey gkey{}, gseen{};
+  bool has_gseen = false;
   int use_graph = 0;
   // per-launch event timing (dit_profile_enable)
   bool prof = false;
@@ -212,6 +229,8 @@ const char* dit_last_error(const dit_handle* h) { return h ? h->err.c_str() : "n
 void dit_destroy(dit_handle* h) {
   if (h == nullptr) return;
   cudaDeviceSynchronize();
+  if (h->gexec != nullptr) cudaGraphExecDestroy(h->gexec);
+  if (h->cap_stream != nullptr) cudaStreamDestroy(h->cap_stream);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   for (void* p : h->allocs) cudaFree(p);
   delete h;
@@ -708,6 +727,46 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
   return DIT_OK;
 }
 
+// The forward through a cached CUDA graph when DIT_OPT_USE_GRAPH is on.  A new set of
+// pointers / parameters runs directly the first time it is seen (which also performs the
+// kernels' one-time attribute set-up), is captured on a private stream the second time,
+// and replays as one graph launch on the caller's stream from then on.  A capture that
+// fails turns the option off and runs directly.
+dit_status run_forward_cached(dit_handle* H, const float* x, const float* t, const void* y, const RunPlan& p,
+                              float* out, cudaStream_t st) {
+  const int depth = H->cfg.depth;
+  if (!H->use_graph || H->prof) return run_forward(H, x, t, y, p, depth, out, st);
+  dit_handle::GraphKey k{x, t, y, out, p.B, p.R, depth, p.guided, g_pdl, p.s};
+  if (H->gexec != nullptr && k == H->gkey) {
+    DIT_CK(H, cudaGraphLaunch(H->gexec, st), "graph launch");
+    return DIT_OK;
+  }
+  if (!(H->has_gseen && k == H->gseen)) {
+    H->gseen = k;
+    H->has_gseen = true;
+    return run_forward(H, x, t, y, p, depth, out, st);
+  }
+  if (H->cap_stream == nullptr) DIT_CK(H, cudaStreamCreateWithFlags(&H->cap_stream, cudaStreamNonBlocking), "capture stream");
+  DIT_CK(H, cudaStreamBeginCapture(H->cap_stream, cudaStreamCaptureModeThreadLocal), "begin capture");
+  const dit_status s = run_forward(H, x, t, y, p, depth, out, H->cap_stream);
+  cudaGraph_t graph = nullptr;
+  cudaError_t e = cudaStreamEndCapture(H->cap_stream, &graph);
+  cudaGraphExec_t ex = nullptr;
+  if (s == DIT_OK && e == cudaSuccess) e = cudaGraphInstantiate(&ex, graph, 0);
+  if (graph != nullptr) cudaGraphDestroy(graph);
+  if (s != DIT_OK || e != cudaSuccess || ex == nullptr) {
+    cudaGetLastError();
+    H->use_graph = 0;
+    if (s != DIT_OK) return s;
+    return run_forward(H, x, t, y, p, depth, out, st);
+  }
+  if (H->gexec != nullptr) cudaGraphExecDestroy(H->gexec);
+  H->gexec = ex;
+  H->gkey = k;
+  DIT_CK(H, cudaGraphLaunch(H->gexec, st), "graph launch");
+  return DIT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -736,7 +795,7 @@ dit_status dit_forward(dit_handle* H, const float* x, const float* t, const void
   dit_status s = check_run(H, x, t, y, B, cfg_scale, p);
   if (s != DIT_OK) return s;
   if (out == nullptr) return fail(H, DIT_ERR_INVALID_ARG, "null output pointer");
-  return run_forward(H, x, t, y, p, H->cfg.depth, out, reinterpret_cast<cudaStream_t>(stream));
+  return run_forward_cached(H, x, t, y, p, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
 dit_status dit_forward_host(dit_handle* H, const float* x, const float* t, const void* y, int B, float cfg_scale,
@@ -753,7 +812,7 @@ dit_status dit_forward_host(dit_handle* H, const float* x, const float* t, const
   DIT_CK(H, cudaMemcpyAsync(H->x_stage, x, xin * 4, cudaMemcpyHostToDevice, st), "x upload");
   DIT_CK(H, cudaMemcpyAsync(H->t_stage, t, (size_t)B * 4, cudaMemcpyHostToDevice, st), "t upload");
   DIT_CK(H, cudaMemcpyAsync(H->y_stage, y, ybytes, cudaMemcpyHostToDevice, st), "y upload");
-  s = run_forward(H, H->x_stage, H->t_stage, H->y_stage, p, c.depth, H->out_stage, st);
+  s = run_forward_cached(H, H->x_stage, H->t_stage, H->y_stage, p, H->out_stage, st);
   if (s != DIT_OK) return s;
   DIT_CK(H, cudaMemcpyAsync(out, H->out_stage, xout * 4, cudaMemcpyDeviceToHost, st), "out download");
   DIT_CK(H, cudaStreamSynchronize(st), "stream sync");

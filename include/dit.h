@@ -154,7 +154,13 @@ void dit_destroy(dit_handle* h);
 
 /* Option switches (test use).  DIT_OPT_FORCE_GUIDANCE = 1 makes dit_forward run the
    2B guided rows even at cfg_scale == 1 (so e(null) + 1*(e(y)-e(null)) is returned).
-   DIT_OPT_USE_GRAPH = 0/1 disables / enables CUDA-graph replay of the forward.
+   DIT_OPT_USE_GRAPH = 0/1 (default 0) disables / enables CUDA-graph replay of the forward:
+   for dit_forward and dit_forward_host, a call whose device pointers, batch and cfg_scale
+   repeat the previous call's runs directly the first time, is captured into a graph (on a
+   private stream) the second time and then replays as one graph launch on the caller's
+   stream.  New pointers or parameters start over; the contents of the buffers may change
+   freely.  While profiling is enabled the graph is bypassed.  If the capture fails the
+   option turns itself off and the call runs directly.
    DIT_OPT_OVERLAP_LAUNCH = 0/1 (process-wide, default 1): launch each kernel with
    programmatic dependent launch so its set-up overlaps the tail of the previous one. */
 enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2, DIT_OPT_OVERLAP_LAUNCH = 3 };
