@@ -198,6 +198,53 @@ def cpu_baseline(cfg, weights):
                       f"float64 numpy oracle, {el:.1f} s"}
 
 
+def time_config(cfg, steps, warmup, graph, flush):
+    """Device time of `steps` whole forwards of `cfg` (seeded weights and inputs, L2 flushed between
+    steps outside the events).  Returns per-step milliseconds."""
+    import torch
+    from diffusion_transformer_denoiser_dit_b200 import DiT
+    from diffusion_transformer_denoiser_dit_b200.binding import DIT_OPT_USE_GRAPH
+    model = DiT(cfg, S.make_weights(cfg))
+    model.set_option(DIT_OPT_USE_GRAPH, 1 if graph else 0)
+    inp = S.make_inputs(cfg)
+    x, t, y = (torch.from_numpy(inp[k]).cuda() for k in ("x", "t", "y"))
+    out = torch.empty(cfg.out_shape(), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        model.forward(x, t, y, cfg.cfg_scale, out=out, stream=stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        model.forward(x, t, y, cfg.cfg_scale, out=out, stream=stream)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    status = model.sync_status()
+    model.close()
+    if status != 0:
+        raise RuntimeError(f"device status {status} while timing {cfg}")
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def all_configs(steps, warmup, graph, flush, peak_tf):
+    res = {}
+    for name, cfg in (("c1 S/8 fp32", S.DIT_S8_F32), ("c2 B/4 bf16", S.DIT_B4_BF16),
+                      ("c3 XL/2 CFG 256px", S.DIT_XL2_CFG256), ("c4 XL/2 CFG 512px", S.DIT_XL2_CFG512),
+                      ("c5 video RF 4096 tokens", S.VIDEO_RF)):
+        ms = time_config(cfg, steps, warmup, graph, flush)
+        med = statistics.median(ms)
+        _, fl = kernel_flops(cfg)
+        tf = fl / (med / 1e3) / 1e12
+        res[name] = {"ms_per_step_median": med, "ms_per_step_min": min(ms),
+                     "tokens_per_s": cfg.rows * cfg.tokens / (med / 1e3),
+                     "samples_per_s": cfg.batch / (med / 1e3), "tflops": tf,
+                     "frac_of_sustained_bf16": tf / peak_tf if cfg.dtype == S.DTYPE_BF16 else None,
+                     "dtype": "bf16" if cfg.dtype == S.DTYPE_BF16 else "f32",
+                     "rows": cfg.rows, "tokens_per_row": cfg.tokens, "flops_per_step": fl}
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -206,6 +253,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel directly instead of replaying a CUDA graph")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="also time the other workloads (S/8 fp32, B/4, XL/2 512px CFG, video) and report them under "
+                         "'all_configs' in the same JSON line")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -265,6 +315,7 @@ def main():
     sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = sum(step_ms)
+    ms_median, ms_min = statistics.median(step_ms), min(step_ms)
     if world > 1:
         tt = torch.tensor([total_ms], device="cuda")
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -334,7 +385,8 @@ def main():
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "ms_per_step_median": ms_median,
+        "ms_per_step_min": ms_min, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) latents, N(0,0.02) weights)",
         "config": {"workload": workload_desc(cfg), "global_batch": cfg.batch * world, "rows_per_gpu": cfg.rows,
                    "tokens_per_step_per_gpu": tokens, "seq_len": cfg.tokens,
@@ -357,6 +409,9 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, weights)
     del weights
+    if args.all_configs and world == 1:
+        model.close()
+        line["all_configs"] = all_configs(min(args.steps, 30), max(args.warmup, 3), not args.no_graph, flush, sustained)
     if rank == 0:
         print(json.dumps(line), flush=True)
     model.close()
