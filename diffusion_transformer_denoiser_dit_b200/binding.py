@@ -18,16 +18,17 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdit_b200
 DIT_OK, DIT_ERR_INVALID_ARG, DIT_ERR_UNSUPPORTED, DIT_ERR_OOM, DIT_ERR_CUDA = 0, 1, 2, 3, 4
 DIT_ERR_DEVICE_TIMEOUT, DIT_ERR_BAD_LABEL, DIT_ERR_NO_DEVICE = 5, 6, 7
 DIT_OPT_FORCE_GUIDANCE, DIT_OPT_USE_GRAPH, DIT_OPT_OVERLAP_LAUNCH = 1, 2, 3
+DIT_SAMPLER_DDIM, DIT_SAMPLER_EULER = 0, 1
 
 # every exported symbol declared in include/dit.h
 EXPORTS = [
     "dit_create", "dit_weight_count", "dit_forward", "dit_forward_host", "dit_sync_status", "dit_last_error",
     "dit_status_string", "dit_destroy", "dit_set_option", "dit_debug_residual", "dit_debug_condition",
     "dit_debug_wait_probe", "dit_op_linear_bf16", "dit_forward_launch_count", "dit_profile_enable",
-    "dit_profile_read", "dit_condition_static", "dit_op_linear_bf16_pair",
+    "dit_profile_read", "dit_condition_static", "dit_op_linear_bf16_pair", "dit_sampler_step", "dit_sample",
 ]
 
-KERNEL_KINDS = ["cond", "adaln", "patch", "ln", "qkv", "attn", "proj", "fc1", "fc2", "decode"]
+KERNEL_KINDS = ["cond", "adaln", "patch", "ln", "qkv", "attn", "proj", "fc1", "fc2", "decode", "sampler"]
 
 
 class DitConfig(ctypes.Structure):
@@ -61,6 +62,8 @@ def load() -> ctypes.CDLL:
         "dit_weight_count": (c_int, [POINTER(DitConfig)]),
         "dit_forward": (c_int, [P, P, P, P, c_int, c_float, P, P]),
         "dit_forward_host": (c_int, [P, P, P, P, c_int, c_float, P, P]),
+        "dit_sampler_step": (c_int, [P, c_int, P, P, c_int, c_float, c_float, P, P]),
+        "dit_sample": (c_int, [P, c_int, P, P, c_int, c_float, c_int, POINTER(c_float), POINTER(c_float), P]),
         "dit_sync_status": (c_int, [P]),
         "dit_last_error": (ctypes.c_char_p, [P]),
         "dit_status_string": (ctypes.c_char_p, [c_int]),
@@ -180,6 +183,30 @@ class DiT:
         rc = self.lib.dit_debug_condition(self.h, _ptr(t), _ptr(y), B, float(cfg_scale), _ptr(c), _stream(stream))
         self._check(rc, "dit_debug_condition")
         return c
+
+    def sampler_step(self, kind: int, x, model_out, a: float, b: float, x_next=None, stream=None):
+        """One sampler update (DIT_SAMPLER_DDIM: a, b = abar now / next; DIT_SAMPLER_EULER:
+        a, b = t now / next) of the device latent x given dit_forward's output; in place when
+        x_next is x."""
+        import torch
+        if x_next is None:
+            x_next = torch.empty_like(x)
+        rc = self.lib.dit_sampler_step(self.h, int(kind), _ptr(x), _ptr(model_out), x.shape[0], float(a), float(b),
+                                       _ptr(x_next), _stream(stream))
+        self._check(rc, "dit_sampler_step")
+        return x_next
+
+    def sample(self, kind: int, x, y, cfg_scale: float, model_t, levels, stream=None):
+        """len(model_t) steps of forward + update, in place on the device latent x."""
+        mt = np.ascontiguousarray(model_t, dtype=np.float32)
+        lv = np.ascontiguousarray(levels, dtype=np.float32)
+        if lv.size != mt.size + 1:
+            raise ValueError("levels needs one more entry than model_t")
+        fp = POINTER(c_float)
+        rc = self.lib.dit_sample(self.h, int(kind), _ptr(x), _ptr(y), x.shape[0], float(cfg_scale), int(mt.size),
+                                 mt.ctypes.data_as(fp), lv.ctypes.data_as(fp), _stream(stream))
+        self._check(rc, "dit_sample")
+        return x
 
     def set_option(self, option: int, value: int):
         self._check(self.lib.dit_set_option(self.h, option, value), "dit_set_option")

@@ -169,6 +169,26 @@ struct dit_handle {
   cudaGraphExec_t gexec = nullptr;
   GraphKey gkey{}, gseen{};
   bool has_gseen = false;
+  // dit_sample: per-step timestep table on the device and the cached graph of the loop
+  float* t_sched = nullptr;
+  size_t t_sched_cap = 0;
+  std::vector<float> t_host;
+  struct SampleKey {
+    float* x = nullptr;
+    const void* y = nullptr;
+    const float* t_sched = nullptr;
+    int B = 0, R = 0, kind = 0, steps = 0;
+    bool guided = false, pdl = false;
+    float s = 0.f;
+    std::vector<float> levels;
+    bool operator==(const SampleKey& o) const {
+      return x == o.x && y == o.y && t_sched == o.t_sched && B == o.B && R == o.R && kind == o.kind &&
+             steps == o.steps && guided == o.guided && pdl == o.pdl && s == o.s && levels == o.levels;
+    }
+  };
+  cudaGraphExec_t sexec = nullptr;
+  SampleKey skey, sseen;
+  bool has_sseen = false;
   int use_graph = 0;
   // per-launch event timing (dit_profile_enable)
   bool prof = false;
@@ -230,6 +250,8 @@ void dit_destroy(dit_handle* h) {
   if (h == nullptr) return;
   cudaDeviceSynchronize();
   if (h->gexec != nullptr) cudaGraphExecDestroy(h->gexec);
+  if (h->sexec != nullptr) cudaGraphExecDestroy(h->sexec);
+  if (h->t_sched != nullptr) cudaFree(h->t_sched);
   if (h->cap_stream != nullptr) cudaStreamDestroy(h->cap_stream);
   for (cudaEvent_t e : h->ev_pool) cudaEventDestroy(e);
   for (void* p : h->allocs) cudaFree(p);
@@ -767,6 +789,55 @@ dit_status run_forward_cached(dit_handle* H, const float* x, const float* t, con
   return DIT_OK;
 }
 
+// One sampler update (the coefficients of x_next = c0 x + c1 pred formed in double).
+dit_status enqueue_sampler_step(dit_handle* H, int kind, const float* x, const float* pred, int B, float a, float b,
+                                float* x_next, cudaStream_t st) {
+  const dit_config& c = H->cfg;
+  const long long plane = static_cast<long long>(c.frames) * c.height * c.width;
+  double c0 = 1.0, c1 = 0.0;
+  if (kind == DIT_SAMPLER_DDIM) {
+    const double da = a, db = b;
+    c0 = std::sqrt(db / da);
+    c1 = std::sqrt(1.0 - db) - std::sqrt(db) * std::sqrt(1.0 - da) / std::sqrt(da);
+  } else {
+    c1 = static_cast<double>(b) - static_cast<double>(a);
+  }
+  SamplerArgs sa;
+  sa.x = x;
+  sa.pred = pred;
+  sa.x_next = x_next;
+  sa.n_sample = plane * c.in_channels;
+  sa.ld_pred = plane * H->g.Cout;
+  sa.B = B;
+  sa.c0 = static_cast<float>(c0);
+  sa.c1 = static_cast<float>(c1);
+  DIT_LAUNCH(H, DIT_KERNEL_SAMPLER, st, launch_sampler_step(sa, H->num_sms, st), "sampler step");
+  return DIT_OK;
+}
+
+dit_status check_sampler(dit_handle* H, int kind, int B, const float* levels, int n_levels) {
+  if (B < 1 || B > H->cfg.max_batch) return fail(H, DIT_ERR_INVALID_ARG, "batch outside [1, max_batch]");
+  if (kind != DIT_SAMPLER_DDIM && kind != DIT_SAMPLER_EULER) return fail(H, DIT_ERR_INVALID_ARG, "unknown sampler kind");
+  for (int i = 0; i < n_levels; ++i) {
+    const float v = levels[i];
+    if (!std::isfinite(v)) return fail(H, DIT_ERR_INVALID_ARG, "sampler level is not finite");
+    if (kind == DIT_SAMPLER_DDIM && !(v > 0.f && v <= 1.f)) return fail(H, DIT_ERR_INVALID_ARG, "DDIM level outside (0, 1]");
+  }
+  return DIT_OK;
+}
+
+// steps x (forward into the handle's output buffer, then the update in place on x)
+dit_status run_sample_loop(dit_handle* H, int kind, float* x, const void* y, const RunPlan& p, int steps,
+                           const std::vector<float>& levels, cudaStream_t st) {
+  for (int i = 0; i < steps; ++i) {
+    dit_status s = run_forward(H, x, H->t_sched + static_cast<size_t>(i) * p.B, y, p, H->cfg.depth, H->out_stage, st);
+    if (s != DIT_OK) return s;
+    s = enqueue_sampler_step(H, kind, x, H->out_stage, p.B, levels[i], levels[i + 1], x, st);
+    if (s != DIT_OK) return s;
+  }
+  return DIT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -796,6 +867,88 @@ dit_status dit_forward(dit_handle* H, const float* x, const float* t, const void
   if (s != DIT_OK) return s;
   if (out == nullptr) return fail(H, DIT_ERR_INVALID_ARG, "null output pointer");
   return run_forward_cached(H, x, t, y, p, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dit_status dit_sampler_step(dit_handle* H, int kind, const float* x, const float* model_out, int B, float a, float b,
+                            float* x_next, dit_stream_t stream) {
+  if (H == nullptr) return DIT_ERR_INVALID_ARG;
+  if (x == nullptr || model_out == nullptr || x_next == nullptr) return fail(H, DIT_ERR_INVALID_ARG, "null pointer");
+  const float lv[2] = {a, b};
+  dit_status s = check_sampler(H, kind, B, lv, 2);
+  if (s != DIT_OK) return s;
+  return enqueue_sampler_step(H, kind, x, model_out, B, a, b, x_next, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dit_status dit_sample(dit_handle* H, int kind, float* x, const void* y, int B, float cfg_scale, int steps,
+                      const float* model_t, const float* levels, dit_stream_t stream) {
+  if (H == nullptr) return DIT_ERR_INVALID_ARG;
+  if (steps < 1 || model_t == nullptr || levels == nullptr) return fail(H, DIT_ERR_INVALID_ARG, "bad step schedule");
+  RunPlan p;
+  dit_status s = check_run(H, x, model_t, y, B, cfg_scale, p);
+  if (s != DIT_OK) return s;
+  s = check_sampler(H, kind, B, levels, steps + 1);
+  if (s != DIT_OK) return s;
+  for (int i = 0; i < steps; ++i)
+    if (!std::isfinite(model_t[i])) return fail(H, DIT_ERR_INVALID_ARG, "model timestep is not finite");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the per-step timestep of every sample, uploaded every call (outside any graph)
+  const size_t need = static_cast<size_t>(steps) * B;
+  if (need > H->t_sched_cap) {
+    if (H->t_sched != nullptr) DIT_CK(H, cudaFree(H->t_sched), "timestep table");
+    H->t_sched = nullptr;
+    H->t_sched_cap = 0;
+    DIT_CK(H, cudaMalloc(&H->t_sched, need * sizeof(float)), "timestep table");
+    H->t_sched_cap = need;
+  }
+  H->t_host.assign(need, 0.f);
+  for (int i = 0; i < steps; ++i)
+    for (int b = 0; b < B; ++b) H->t_host[static_cast<size_t>(i) * B + b] = model_t[i];
+  DIT_CK(H, cudaMemcpyAsync(H->t_sched, H->t_host.data(), need * sizeof(float), cudaMemcpyHostToDevice, st),
+         "timestep upload");
+  std::vector<float> lv(levels, levels + steps + 1);
+  if (!H->use_graph || H->prof) return run_sample_loop(H, kind, x, y, p, steps, lv, st);
+  dit_handle::SampleKey k;
+  k.x = x;
+  k.y = y;
+  k.t_sched = H->t_sched;
+  k.B = B;
+  k.R = p.R;
+  k.kind = kind;
+  k.steps = steps;
+  k.guided = p.guided;
+  k.pdl = g_pdl;
+  k.s = p.s;
+  k.levels = lv;
+  if (H->sexec != nullptr && k == H->skey) {
+    DIT_CK(H, cudaGraphLaunch(H->sexec, st), "graph launch");
+    return DIT_OK;
+  }
+  if (!(H->has_sseen && k == H->sseen)) {
+    H->sseen = k;
+    H->has_sseen = true;
+    return run_sample_loop(H, kind, x, y, p, steps, lv, st);
+  }
+  if (H->cap_stream == nullptr) DIT_CK(H, cudaStreamCreateWithFlags(&H->cap_stream, cudaStreamNonBlocking), "capture stream");
+  // the capture stream must see the timestep upload: it is ordered on `st`, so the graph
+  // is launched on `st` after it; capturing itself records without executing.
+  DIT_CK(H, cudaStreamBeginCapture(H->cap_stream, cudaStreamCaptureModeThreadLocal), "begin capture");
+  const dit_status ls = run_sample_loop(H, kind, x, y, p, steps, lv, H->cap_stream);
+  cudaGraph_t graph = nullptr;
+  cudaError_t e = cudaStreamEndCapture(H->cap_stream, &graph);
+  cudaGraphExec_t ex = nullptr;
+  if (ls == DIT_OK && e == cudaSuccess) e = cudaGraphInstantiate(&ex, graph, 0);
+  if (graph != nullptr) cudaGraphDestroy(graph);
+  if (ls != DIT_OK || e != cudaSuccess || ex == nullptr) {
+    cudaGetLastError();
+    H->use_graph = 0;
+    if (ls != DIT_OK) return ls;
+    return run_sample_loop(H, kind, x, y, p, steps, lv, st);
+  }
+  if (H->sexec != nullptr) cudaGraphExecDestroy(H->sexec);
+  H->sexec = ex;
+  H->skey = k;
+  DIT_CK(H, cudaGraphLaunch(H->sexec, st), "graph launch");
+  return DIT_OK;
 }
 
 dit_status dit_forward_host(dit_handle* H, const float* x, const float* t, const void* y, int B, float cfg_scale,

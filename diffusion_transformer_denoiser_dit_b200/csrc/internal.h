@@ -149,6 +149,18 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode_cfg(const DecodeArgs& a, cudaStream_t st);
 
+// Sampler update x_next = c0 * x + c1 * pred, pred = the first n_sample values of each
+// sample's ld_pred-long block of the denoiser output (its first C channels).
+struct SamplerArgs {
+  const float* x;        // [B, n_sample]
+  const float* pred;     // [B, ld_pred]
+  float* x_next;         // [B, n_sample], may alias x
+  long long n_sample, ld_pred;
+  int B;
+  float c0, c1;
+};
+cudaError_t launch_sampler_step(const SamplerArgs& a, int num_sms, cudaStream_t st);
+
 cudaError_t launch_pos_tables(float* pos, float* rope, int gf, int gh, int gw, int d, int dh, cudaStream_t st);
 cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaStream_t st);
 cudaError_t launch_wait_probe(int* flag, int* status, long long limit_ns, cudaStream_t st);

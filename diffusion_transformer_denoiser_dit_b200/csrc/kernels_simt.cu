@@ -526,6 +526,47 @@ cudaError_t launch_decode_cfg(const DecodeArgs& a, cudaStream_t st) {
   return launch_kernel(decode_cfg_kernel, grid, dim3(256), smem, st, a);
 }
 
+// ============================================================================ sampler step
+// x_next = c0 x + c1 pred over [B, n_sample]; pred rows are ld_pred apart (the first C
+// channels of a C_out-channel denoiser output).  Grid-stride, 16-byte accesses when every
+// row start is 16-byte aligned.  x_next may alias x: each element is read, then written,
+// by the same thread.
+template <bool VEC>
+__global__ void __launch_bounds__(256) sampler_step_kernel(SamplerArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  if (VEC) {
+    const long long per = a.n_sample >> 2, ld = a.ld_pred >> 2, total = per * a.B;
+    const float4* x = reinterpret_cast<const float4*>(a.x);
+    const float4* p = reinterpret_cast<const float4*>(a.pred);
+    float4* o = reinterpret_cast<float4*>(a.x_next);
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+      const long long b = i / per, r = i - b * per;
+      const float4 xv = x[i], pv = p[b * ld + r];
+      o[i] = make_float4(fmaf(a.c0, xv.x, a.c1 * pv.x), fmaf(a.c0, xv.y, a.c1 * pv.y), fmaf(a.c0, xv.z, a.c1 * pv.z),
+                         fmaf(a.c0, xv.w, a.c1 * pv.w));
+    }
+  } else {
+    const long long total = a.n_sample * a.B;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+      const long long b = i / a.n_sample, r = i - b * a.n_sample;
+      a.x_next[i] = fmaf(a.c0, a.x[i], a.c1 * a.pred[b * a.ld_pred + r]);
+    }
+  }
+}
+
+cudaError_t launch_sampler_step(const SamplerArgs& a, int num_sms, cudaStream_t st) {
+  if (a.B <= 0 || a.n_sample <= 0) return cudaSuccess;
+  const bool vec = (a.n_sample % 4) == 0 && (a.ld_pred % 4) == 0 && (reinterpret_cast<uintptr_t>(a.x) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(a.pred) & 15u) == 0 && (reinterpret_cast<uintptr_t>(a.x_next) & 15u) == 0;
+  const long long work = vec ? a.n_sample / 4 * a.B : a.n_sample * a.B;
+  const long long want = (work + 255) / 256;
+  const int grid = static_cast<int>(want < 4LL * num_sms ? want : 4LL * num_sms);
+  if (vec) return launch_kernel(sampler_step_kernel<true>, dim3(grid), dim3(256), 0, st, a);
+  return launch_kernel(sampler_step_kernel<false>, dim3(grid), dim3(256), 0, st, a);
+}
+
 // ============================================================================ set-up tables
 // pos[tau, :] (2D sin-cos, images): first d/2 dims encode the grid row, the last d/2
 // the column; each half [sin(p w_k) | cos(p w_k)], w_k = 10000^(-k/(d/4)).

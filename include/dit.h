@@ -135,6 +135,51 @@ dit_status dit_forward_host(dit_handle* h, const float* x_host, const float* t_h
                             const void* y_host, int B, float cfg_scale, float* out_host,
                             dit_stream_t stream);
 
+/* ------------------------------------------------------------------------------ */
+/* Sampling: the update around the denoiser.                                      */
+/* ------------------------------------------------------------------------------ */
+
+enum { DIT_SAMPLER_DDIM = 0, DIT_SAMPLER_EULER = 1 };
+
+/*
+ * dit_sampler_step — one sampler update of the latent x given the denoiser output
+ * model_out of dit_forward (one fused elementwise kernel):
+ *   DIT_SAMPLER_DDIM  (noise head): eps = the first C of the C_out output channels (a
+ *       learned-covariance head writes [eps | Sigma]); with a = abar now, b = abar next,
+ *       x_next = sqrt(b) (x - sqrt(1-a) eps) / sqrt(a) + sqrt(1-b) eps, i.e. the clean
+ *       latent that eps implies under the DDPM forward process x_t = sqrt(abar_t) x_0 +
+ *       sqrt(1-abar_t) eps ("Sora / DiT", method section, training-objective bullet)
+ *       carried to level b with the same eps.  The two coefficients are formed on the host
+ *       in double precision.
+ *   DIT_SAMPLER_EULER (velocity head): x_next = x + (b - a) v, v = the first C channels,
+ *       with a = t now, b = t next, one Euler step along x_t = t x_1 + (1-t) x_0 ("GOKU",
+ *       §2.3 rectified flow).
+ * x, x_next: device float32 [B, C, F, H, W] (F omitted for images); x_next may equal x.
+ * model_out: device float32 [B, C_out, F, H, W].  Asynchronous on `stream`.
+ * Errors (nothing is launched): DIT_ERR_INVALID_ARG for null pointers, B outside
+ * [1, max_batch], an unknown kind, or DDIM levels outside (0, 1].
+ */
+dit_status dit_sampler_step(dit_handle* h, int kind, const float* x, const float* model_out, int B, float a,
+                            float b, float* x_next, dit_stream_t stream);
+
+/*
+ * dit_sample — `steps` sampling steps in place on x: for i = 0 .. steps-1,
+ *   out = dit_forward(x, t = model_t[i] for every sample, y, B, cfg_scale) into the
+ *         handle's own output buffer, then
+ *   x   = dit_sampler_step(kind, x, out, levels[i], levels[i+1]).
+ * x: device float32 [B, C, F, H, W] (in: the starting noise; out: the sample).
+ * y: device labels / text vectors as for dit_forward.  model_t: host float[steps], the
+ * timestep value the denoiser sees at step i; levels: host float[steps+1] (abar for DDIM,
+ * t for Euler).  Both host arrays are read before the call returns; the work is
+ * asynchronous on `stream`.  With DIT_OPT_USE_GRAPH the whole loop (steps forwards and
+ * updates) is captured and replayed like dit_forward: a call that repeats the previous
+ * call's pointers, batch, cfg_scale, kind and levels replays the graph (model_t is
+ * uploaded every call, so it may change).  Errors as dit_forward and dit_sampler_step,
+ * plus DIT_ERR_INVALID_ARG for steps < 1 or null host arrays; nothing is launched then.
+ */
+dit_status dit_sample(dit_handle* h, int kind, float* x, const void* y, int B, float cfg_scale, int steps,
+                      const float* model_t, const float* levels, dit_stream_t stream);
+
 /* Reads and clears the handle's device status word (synchronises the device first).
    Returns DIT_OK or the first device-side error recorded since the last call. */
 dit_status dit_sync_status(dit_handle* h);
@@ -210,7 +255,7 @@ dit_status dit_op_linear_bf16(const uint16_t* x, const uint16_t* w, const float*
  */
 enum { DIT_KERNEL_COND = 0, DIT_KERNEL_ADALN = 1, DIT_KERNEL_PATCH = 2, DIT_KERNEL_LN = 3, DIT_KERNEL_QKV = 4,
        DIT_KERNEL_ATTN = 5, DIT_KERNEL_PROJ = 6, DIT_KERNEL_FC1 = 7, DIT_KERNEL_FC2 = 8, DIT_KERNEL_DECODE = 9,
-       DIT_KERNEL_COUNT = 10 };
+       DIT_KERNEL_SAMPLER = 10, DIT_KERNEL_COUNT = 11 };
 dit_status dit_profile_enable(dit_handle* h, int enable);
 dit_status dit_profile_read(dit_handle* h, float* total_ms, int* launches);
 
