@@ -151,6 +151,28 @@ def dist_setup():
     return world, rank, local
 
 
+def replica_seed(cfg, rank: int) -> int:
+    """Input seed of replica `rank`: the workload's seed + rank, so every replica denoises its
+    own latents (weak scaling, no data shared between ranks)."""
+    return S.inputs_seed(cfg) + rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The maximum of a per-rank float over all ranks (the job's time is its slowest rank)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def aggregate_rate(units_per_rank_step: float, world: int, steps: int, seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank_step * world * steps / seconds
+
+
 def run_reference(args):
     """The oracle (float64 numpy on the host cores) on a bounded sample per step."""
     world, rank, _ = dist_setup()
@@ -275,7 +297,7 @@ def main():
     weights = S.make_weights(cfg)
     model = DiT(cfg, weights)
     model.set_option(DIT_OPT_USE_GRAPH, 0 if args.no_graph else 1)
-    inp = S.make_inputs(cfg, seed=S.inputs_seed(cfg) + rank)
+    inp = S.make_inputs(cfg, seed=replica_seed(cfg, rank))
     x = torch.from_numpy(inp["x"]).cuda()
     t = torch.from_numpy(inp["t"]).cuda()
     y = torch.from_numpy(inp["y"]).cuda()
@@ -314,12 +336,8 @@ def main():
         dist.barrier()
     sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
     ms_median, ms_min = statistics.median(step_ms), min(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), world, "cuda")
     status = model.sync_status()
 
     # per-kernel durations: a second pass with events around every launch
@@ -345,10 +363,7 @@ def main():
         t0 = time.perf_counter()
         model.forward_host_ptr(xh.data_ptr(), th.data_ptr(), yh.data_ptr(), cfg.batch, cfg.cfg_scale, oh.data_ptr())
         e2e_s += time.perf_counter() - t0
-    if world > 1:
-        tt = torch.tensor([e2e_s], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_s = float(tt.item())
+    e2e_s = max_over_ranks(e2e_s, world, "cuda")
 
     # sampler loop: forward + fused DDIM update per step, the whole loop replayed as one graph
     from diffusion_transformer_denoiser_dit_b200.binding import DIT_SAMPLER_DDIM
@@ -388,7 +403,7 @@ def main():
 
     per, step_flops = kernel_flops(cfg)
     tokens = cfg.rows * cfg.tokens
-    value = tokens * world * args.steps / (total_ms / 1e3)
+    value = aggregate_rate(tokens, world, args.steps, total_ms / 1e3)
     ms_per_step = total_ms / args.steps
     pk, pk_kind = peaks()
     sustained = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
@@ -435,7 +450,7 @@ def main():
                              "frac_of_nominal_2250": achieved_tf / 2250.0},
         "roofline": roof,
         "kernels": kernels,
-        "e2e": {"value": tokens * world * args.steps / e2e_s, "unit": "tokens/s",
+        "e2e": {"value": aggregate_rate(tokens, world, args.steps, e2e_s), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xh.numel() * 4 + th.numel() * 4 + yh.numel() * 4),
                 "d2h_bytes_per_step": int(oh.numel() * 4), "api": "dit_forward_host"},
         "gpu_launches": model.launch_count(cfg.batch, cfg.cfg_scale) * args.steps,
