@@ -294,3 +294,47 @@ def test_full_size_sampled_parity(cfg):
     assert_parity(cfg, got[b:b + 1], want, cfg.name)
     # every sample: finite and of the expected shape
     assert got.shape == cfg.out_shape() and np.all(np.isfinite(got))
+
+
+# ----------------------------------------------------------------------------- edge shapes
+EDGE = {
+    # no blocks at all: the forward is the final layer of the embedding
+    "depth0_bf16": lambda: small_image_bf16_dh72().with_(depth=0),
+    "depth0_f32": lambda: small_video_f32().with_(depth=0),
+    # one token per row: softmax over a single key is 1, attention returns V
+    "one_token_bf16": lambda: small_image_bf16_dh64().with_(height=4, width=4),
+    "one_token_guided_dh72": lambda: small_image_bf16_dh72().with_(height=2, width=2),
+    # the widest supported models for each head dim (hidden <= 1536)
+    "widest_dh64": lambda: small_image_bf16_dh64().with_(hidden=1536, heads=24, mlp_hidden=6144, depth=1, batch=2),
+    "widest_dh72": lambda: small_image_bf16_dh72().with_(hidden=1440, heads=20, mlp_hidden=5760, depth=1, height=16,
+                                                         width=16, batch=2),
+    # a single sample
+    "batch1_video": lambda: small_video_bf16().with_(batch=1),
+}
+
+
+@pytest.mark.parametrize("name", list(EDGE))
+def test_edge_shape_parity(name):
+    cfg = EDGE[name]()
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    want = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    m = DiT(cfg, W)
+    d = dev(inp)
+    got = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale)
+    assert m.sync_status() == binding.DIT_OK
+    assert_parity(cfg, got.cpu().numpy(), want, name)
+    m.close()
+
+
+def test_empty_batch_is_rejected_without_launch():
+    cfg = small_image_bf16_dh64()
+    m = DiT(cfg, S.make_weights(cfg))
+    d = dev(S.make_inputs(cfg, batch=1))
+    out = torch.full((8,), 7.0, device="cuda")
+    rc = m.lib.dit_forward(m.h, d["x"].data_ptr(), d["t"].data_ptr(), d["y"].data_ptr(), 0, 1.0, out.data_ptr(), None)
+    assert rc == binding.DIT_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())
+    assert m.sync_status() == binding.DIT_OK
+    m.close()
