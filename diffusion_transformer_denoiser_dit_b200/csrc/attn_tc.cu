@@ -51,7 +51,7 @@ struct AttnCfg {
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int TMEM_COLS = 512;                 // S0, S1, O0, O1 (128 columns each)
   static constexpr int THREADS = 384;                   // warpgroup 0: loads, MMA; 1, 2: softmax
-  static constexpr int REG_CTRL = 80, REG_SOFTMAX = 200;
+  static constexpr int REG_CTRL = 96, REG_SOFTMAX = 200;
   static constexpr int REG_POOL = 128 * REG_CTRL + 256 * REG_SOFTMAX;  // must fit the launch allocation
   static_assert(QK_TILE % 1024 == 0 && V_ATOM % 1024 == 0 && OFF_O % 1024 == 0, "1024-byte aligned tiles");
   static_assert(O_ROW % 16 == 0, "16-byte output rows");
@@ -180,61 +180,86 @@ __global__ void __launch_bounds__(384, 1)
     } else if (warp == 1 && lane == 0) {  // ---------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, C::DP);
+      // The issuing thread is a serial chain that shares its scheduler with two softmax
+      // warps, so the per-tile path does no division: items and key tiles are followed by
+      // cursors, and every descriptor is a constant high word plus base + offset.
+      const uint32_t q_lo = sdesc_lo(sbase + C::OFF_Q), k_lo = sdesc_lo(sbase + C::OFF_K);
+      const uint32_t v_lo = sdesc_lo(sbase + C::OFF_V), p_lo = sdesc_lo(sbase + C::OFF_P);
+      const int pmod = static_cast<int>(gridDim.x) % pairs;
+      struct Cursor {
+        int li, j, pidx, ng;  // item, key tile in the item, query-tile pair of the item, groups
+      };
+      auto first = [&]() {
+        Cursor c{0, 0, static_cast<int>(blockIdx.x) % pairs, 0};
+        c.ng = 2 * c.pidx + 1 < nq ? 2 : 1;
+        return c;
+      };
+      auto advance = [&](Cursor& c) {
+        if (++c.j == nk) {
+          c.j = 0;
+          ++c.li;
+          c.pidx += pmod;
+          if (c.pidx >= pairs) c.pidx -= pairs;
+          c.ng = 2 * c.pidx + 1 < nq ? 2 : 1;
+        }
+      };
       int qk_cnt[2] = {0, 0};  // Q K^T issued per query group
       int pv_cnt[2] = {0, 0};  // P V issued per query group
       int it_cnt[2] = {0, 0};  // items whose first P V was issued, per group
-      // S_g = Q_g K_n^T for every query group of tile n
+      Cursor cq = first(), cp = first();
+      // S_g = Q_g K_n^T for every query group of tile n (cursor cq is at tile n)
       auto issue_qk = [&](int n) -> bool {
-        const int li = n / nk, j = n - li * nk;
-        int rh, qt0, ng;
-        item_of(li, rh, qt0, ng);
-        if (j == 0 && !mbar_wait(BAR(B_QF), li & 1, status)) return false;
+        if (cq.j == 0 && !mbar_wait(BAR(B_QF), cq.li & 1, status)) return false;
         if (!mbar_wait(BAR(B_KF0 + (n & 1)), (n >> 1) & 1, status)) return false;
-        const uint32_t kb = sbase + C::OFF_K + (n & 1) * C::QK_TILE;
+        const uint32_t kb = k_lo + (n & 1) * (C::QK_TILE >> 4);
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          if (g >= ng) break;
+          if (g >= cq.ng) break;
           // S_g may be overwritten once the softmax of group g has read its previous tile
           if (qk_cnt[g] > 0 && !mbar_wait(BAR(B_SF0 + g), (qk_cnt[g] - 1) & 1, status)) return false;
           tc_fence_after();
-          const uint32_t qb = sbase + C::OFF_Q + g * C::QK_TILE;
+          const uint32_t qb = q_lo + g * (C::QK_TILE >> 4);
           const uint32_t tS = tmem_base + g * 128;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(tS, sdesc_k_sw128(qb + k * 32), sdesc_k_sw128(kb + k * 32), idesc_s, k > 0 ? 1u : 0u);
-          if (C::TAIL) mma_bf16_ss(tS, sdesc_k_sw32(qb + C::MAIN), sdesc_k_sw32(kb + C::MAIN), idesc_s, 1u);
+            mma_bf16_ss(tS, sdesc_make(qb + 2 * k, kSdescHiSw128), sdesc_make(kb + 2 * k, kSdescHiSw128), idesc_s,
+                        k > 0 ? 1u : 0u);
+          if (C::TAIL)
+            mma_bf16_ss(tS, sdesc_make(qb + (C::MAIN >> 4), kSdescHiSw32), sdesc_make(kb + (C::MAIN >> 4), kSdescHiSw32),
+                        idesc_s, 1u);
           mma_commit(BAR(B_S0 + g));
           ++qk_cnt[g];
         }
         mma_commit(BAR(B_KE0 + (n & 1)));
-        if (j == nk - 1) mma_commit(BAR(B_QE));
+        if (cq.j == nk - 1) mma_commit(BAR(B_QE));
+        advance(cq);
         return true;
       };
-      // O_g (+)= P_g V_n for every query group of tile n
+      // O_g (+)= P_g V_n for every query group of tile n (cursor cp is at tile n)
       auto issue_pv = [&](int n) -> bool {
-        const int li = n / nk, j = n - li * nk;
-        int rh, qt0, ng;
-        item_of(li, rh, qt0, ng);
         if (!mbar_wait(BAR(B_VF0 + (n & 1)), (n >> 1) & 1, status)) return false;
-        const uint32_t vb = sbase + C::OFF_V + (n & 1) * C::V_TILE;
+        const uint32_t vb = v_lo + (n & 1) * (C::V_TILE >> 4);
+        const bool first_tile = cp.j == 0;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          if (g >= ng) break;
+          if (g >= cp.ng) break;
           if (!mbar_wait(BAR(B_P0 + g), pv_cnt[g] & 1, status)) return false;
           // a new item overwrites O_g: its epilogue for the previous item must have read it
-          if (j == 0 && it_cnt[g] > 0 && !mbar_wait(BAR(B_OF0 + g), (it_cnt[g] - 1) & 1, status)) return false;
+          if (first_tile && it_cnt[g] > 0 && !mbar_wait(BAR(B_OF0 + g), (it_cnt[g] - 1) & 1, status)) return false;
           tc_fence_after();
-          const uint32_t pb = sbase + C::OFF_P + g * C::P_TILE;
+          const uint32_t pb = p_lo + g * (C::P_TILE >> 4);
           const uint32_t tO = tmem_base + 256 + g * 128;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_bf16_ss(tO, sdesc_k_sw128(pb + (k >> 2) * C::MAIN + (k & 3) * 32),
-                        sdesc_k_sw128(vb + (k >> 2) * C::V_ATOM + (k & 3) * 32), idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+            mma_bf16_ss(tO, sdesc_make(pb + (k >> 2) * (C::MAIN >> 4) + (k & 3) * 2, kSdescHiSw128),
+                        sdesc_make(vb + (k >> 2) * (C::V_ATOM >> 4) + (k & 3) * 2, kSdescHiSw128), idesc_o,
+                        (!first_tile || k > 0) ? 1u : 0u);
           mma_commit(BAR(B_O0 + g));
           ++pv_cnt[g];
-          if (j == 0) ++it_cnt[g];
+          if (first_tile) ++it_cnt[g];
         }
         mma_commit(BAR(B_VE0 + (n & 1)));
+        advance(cp);
         return true;
       };
       // Q K^T of the next key tile goes in before P V of the current one, so the tensor
@@ -243,7 +268,7 @@ __global__ void __launch_bounds__(384, 1)
       int n_qk = 0;
       bool ok = true;
       for (int n = 0; n < ntiles && ok; ++n) {
-        while (ok && (n_qk <= n || (n_qk == n + 1 && n_qk < ntiles && n_qk % nk != 0))) ok = issue_qk(n_qk++);
+        while (ok && (n_qk <= n || (n_qk == n + 1 && n_qk < ntiles && cq.j != 0))) ok = issue_qk(n_qk++);
         if (ok) ok = issue_pv(n);
       }
     }

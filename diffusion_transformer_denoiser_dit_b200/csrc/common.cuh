@@ -247,6 +247,16 @@ __device__ __forceinline__ uint64_t sdesc_k_sw32(uint32_t saddr) {
   return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (16ull << 32) | (1ull << 46) | (6ull << 61);
 }
 
+// The same descriptors as a constant high word and a low word (start address >> 4 and
+// the LBO bit), so that the descriptor of base + offset is one 32-bit add on the low word
+// (shared addresses are below 256 KB: the 14-bit start field never carries).
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr) { return ((saddr & 0x3FFFFu) >> 4) | (1u << 16); }
+constexpr uint32_t kSdescHiSw128 = 64u | (1u << 14) | (2u << 29);
+constexpr uint32_t kSdescHiSw32 = 16u | (1u << 14) | (6u << 29);
+__device__ __forceinline__ uint64_t sdesc_make(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // tcgen05.ld: 32 lanes x 32 bits, N consecutive columns per thread.
 #define DIT_TMEM_LD_X8(taddr, r)                                                                                 \
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"                          \
