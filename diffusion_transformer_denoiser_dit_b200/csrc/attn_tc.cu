@@ -128,53 +128,45 @@ __global__ void __launch_bounds__(384, 1)
   if (warp < 4) {
     regs_dec<C::REG_CTRL>();
     if (warp == 0 && lane == 0) {  // ---------- loads: Q per item; K_n and V_n^T through two-stage rings
+      // One fixed order (Q of an item, then K_n, V_n of each of its key tiles) with blocking
+      // bounded waits, so the thread sleeps instead of polling next to the softmax warps.
+      // Each wait depends only on MMAs whose operands were loaded earlier in this order.
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      int lq = 0, nkl = 0, nvl = 0;
-      uint64_t t0 = global_timer_ns();  // time of the last issued load
-      while (lq < my_items || nkl < ntiles || nvl < ntiles) {
-        const int progress = lq + nkl + nvl;
-        // Q of item lq once every Q K^T of item lq-1 completed
-        if (lq < my_items && (lq == 0 || mbar_test(BAR(B_QE), (lq - 1) & 1))) {
-          int rh, qt0, ng;
-          item_of(lq, rh, qt0, ng);
-          mbar_arrive_expect_tx(BAR(B_QF), ng * C::QK_TILE);
-          for (int g = 0; g < ng; ++g) {
-            const int row0 = rh * a.Tpad + (qt0 + g) * 128;
-            const uint32_t dst = sbase + C::OFF_Q + g * C::QK_TILE;
-            tma_load_2d(dst, &tmQ, BAR(B_QF), 0, row0);
-            if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmQt, BAR(B_QF), 64, row0);
+      int n = 0;  // key tile of this CTA
+      bool ok = true;
+      for (int li = 0; li < my_items && ok; ++li) {
+        int rh, qt0, ng;
+        item_of(li, rh, qt0, ng);
+        // Q of item li once every Q K^T of item li-1 completed
+        if (li > 0 && !mbar_wait(BAR(B_QE), (li - 1) & 1, status)) break;
+        mbar_arrive_expect_tx(BAR(B_QF), ng * C::QK_TILE);
+        for (int g = 0; g < ng; ++g) {
+          const int row0 = rh * a.Tpad + (qt0 + g) * 128;
+          const uint32_t dst = sbase + C::OFF_Q + g * C::QK_TILE;
+          tma_load_2d(dst, &tmQ, BAR(B_QF), 0, row0);
+          if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmQt, BAR(B_QF), 64, row0);
+        }
+        for (int j = 0; j < nk; ++j, ++n) {
+          const uint32_t st = n & 1, free_parity = ((n >> 1) & 1) ^ 1u;
+          // stage n & 1 is free once the MMA that read tile n-2 from it completed
+          if (n >= 2 && !mbar_wait(BAR(B_KE0 + st), free_parity, status)) {
+            ok = false;
+            break;
           }
-          ++lq;
-        }
-        // stage n & 1 is free once the MMA that read tile n-2 from it completed
-        if (nkl < ntiles && (nkl < 2 || mbar_test(BAR(B_KE0 + (nkl & 1)), ((nkl >> 1) & 1) ^ 1u))) {
-          int rh, qt0, ng;
-          item_of(nkl / nk, rh, qt0, ng);
-          const int krow0 = rh * a.Tpad + (nkl % nk) * 128;
-          const uint32_t dst = sbase + C::OFF_K + (nkl & 1) * C::QK_TILE;
-          mbar_arrive_expect_tx(BAR(B_KF0 + (nkl & 1)), C::QK_TILE);
-          tma_load_2d(dst, &tmK, BAR(B_KF0 + (nkl & 1)), 0, krow0);
-          if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmKt, BAR(B_KF0 + (nkl & 1)), 64, krow0);
-          ++nkl;
-        }
-        if (nvl < ntiles && (nvl < 2 || mbar_test(BAR(B_VE0 + (nvl & 1)), ((nvl >> 1) & 1) ^ 1u))) {
-          int rh, qt0, ng;
-          item_of(nvl / nk, rh, qt0, ng);
-          const int kcol0 = (nvl % nk) * 128;
-          const uint32_t dst = sbase + C::OFF_V + (nvl & 1) * C::V_TILE;
-          mbar_arrive_expect_tx(BAR(B_VF0 + (nvl & 1)), C::V_TILE);
-          tma_load_2d(dst, &tmV, BAR(B_VF0 + (nvl & 1)), kcol0, rh * C::DP);
-          tma_load_2d(dst + C::V_ATOM, &tmV, BAR(B_VF0 + (nvl & 1)), kcol0 + 64, rh * C::DP);
-          ++nvl;
-        }
-        const uint64_t now = global_timer_ns();
-        if (lq + nkl + nvl != progress) {
-          t0 = now;
-        } else if (now - t0 > kWaitLimitNs) {
-          record_status(status, DIT_ERR_DEVICE_TIMEOUT);
-          break;
+          const uint32_t kdst = sbase + C::OFF_K + st * C::QK_TILE;
+          mbar_arrive_expect_tx(BAR(B_KF0 + st), C::QK_TILE);
+          tma_load_2d(kdst, &tmK, BAR(B_KF0 + st), 0, rh * a.Tpad + j * 128);
+          if (C::TAIL) tma_load_2d(kdst + C::MAIN, &tmKt, BAR(B_KF0 + st), 64, rh * a.Tpad + j * 128);
+          if (n >= 2 && !mbar_wait(BAR(B_VE0 + st), free_parity, status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t vdst = sbase + C::OFF_V + st * C::V_TILE;
+          mbar_arrive_expect_tx(BAR(B_VF0 + st), C::V_TILE);
+          tma_load_2d(vdst, &tmV, BAR(B_VF0 + st), j * 128, rh * C::DP);
+          tma_load_2d(vdst + C::V_ATOM, &tmV, BAR(B_VF0 + st), j * 128 + 64, rh * C::DP);
         }
       }
     } else if (warp == 1 && lane == 0) {  // ---------------- MMA issuer
