@@ -235,9 +235,17 @@ def condition(cfg, W: Dict[str, np.ndarray], t, y):
     return c
 
 
-def cfg_combine(eps_cond, eps_uncond, s: float):
-    """Classifier-free guidance: eps(∅) + s (eps(c) - eps(∅)) ([Sora-DiT] guidance bullet)."""
-    return eps_uncond + s * (eps_cond - eps_uncond)
+def cfg_combine(eps_cond, eps_uncond, s: float, channels: Optional[int] = None):
+    """Classifier-free guidance: eps(∅) + s (eps(c) - eps(∅)) ([Sora-DiT] guidance bullet).
+    With `channels` = n, only output channels c < n are guided, the variant [DiT-wiki]
+    "ImageNet 클래스 조건 생성" attributes to the official code (n = 3); the other channels
+    keep the conditional prediction (reading: the page does not say what they hold)."""
+    g = eps_uncond + s * (eps_cond - eps_uncond)
+    if channels is None or channels <= 0 or channels >= eps_cond.shape[1]:
+        return g
+    out = np.array(eps_cond, dtype=F64, copy=True)
+    out[:, :channels] = g[:, :channels]
+    return out
 
 
 # --------------------------------------------------------------------------- #
@@ -318,14 +326,15 @@ def embed(cfg, W, x5):
 
 def forward(cfg, weights: Sequence[np.ndarray] | Dict[str, np.ndarray], x, t, y,
             cfg_scale: Optional[float] = None, force_guidance: bool = False,
-            stop_after_block: Optional[int] = None):
+            stop_after_block: Optional[int] = None, cfg_channels: Optional[int] = None):
     """Denoiser output for a batch.
 
     Returns the guided prediction [B, C_out, (F,) H, W] (float64), or, when
     ``stop_after_block`` is k, the residual stream [rows, T, d] after k blocks
     (k = 0: right after the embedding), rows ordered [cond; uncond] if guided.
     Guidance runs when the model is class-conditional and s != 1 (or when
-    forced): rows [x; x] with labels [y; null] are evaluated and combined.
+    forced): rows [x; x] with labels [y; null] are evaluated and combined, on every output
+    channel or, with ``cfg_channels`` = n > 0, on channels c < n only.
     """
     from_list = not isinstance(weights, dict)
     if from_list:
@@ -354,7 +363,7 @@ def forward(cfg, weights: Sequence[np.ndarray] | Dict[str, np.ndarray], x, t, y,
     z = final_layer(h, sc, W)
     img = unpatchify(z, cfg.out_channels, cfg.grid, cfg.patch_t, cfg.patch_h, cfg.patch_w)
     if guided:
-        img = cfg_combine(img[:b], img[b:], s)
+        img = cfg_combine(img[:b], img[b:], s, cfg_channels)
     if img.shape[2] == 1 and np.asarray(x).ndim == 4:
         img = img[:, :, 0]
     return img

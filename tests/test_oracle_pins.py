@@ -302,6 +302,28 @@ def test_guidance_special_cases():
     assert np.allclose(s3 - s15, (3.0 - 1.5) * (cond - uncond), rtol=1e-10, atol=1e-10)
 
 
+def test_guidance_on_the_first_channels_only():
+    """[DiT-wiki] "ImageNet 클래스 조건 생성": the official code guides only the first three
+    output channels.  Those channels equal full guidance; the rest equal the unguided
+    conditional prediction (computed here by a separate, unduplicated forward)."""
+    cfg = small_image(cfg_scale=1.5)
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    x, t, y = inp["x"], inp["t"], inp["y"]
+    full = O.forward(cfg, W, x, t, y)
+    part = O.forward(cfg, W, x, t, y, cfg_channels=3)
+    cond = O.forward(cfg, W, x, t, y, cfg_scale=1.0)
+    assert cfg.out_channels > 3
+    assert np.array_equal(part[:, :3], full[:, :3])
+    assert np.allclose(part[:, 3:], cond[:, 3:], rtol=1e-12, atol=1e-12)
+    assert not np.allclose(part[:, 3:], full[:, 3:], rtol=1e-6, atol=1e-6)     # the guidance mattered there
+    assert np.array_equal(O.forward(cfg, W, x, t, y, cfg_channels=cfg.out_channels), full)
+    assert np.array_equal(O.forward(cfg, W, x, t, y, cfg_channels=0), full)
+    # planted slip: the unguided channels taken from the unconditional rows
+    uncond = O.forward(cfg, W, x, t, np.full_like(y, cfg.num_classes), cfg_scale=1.0)
+    assert not np.allclose(uncond[:, 3:], cond[:, 3:], rtol=1e-6, atol=1e-6)
+
+
 @pytest.mark.parametrize("kind", ["image", "image_guided", "video"])
 def test_forward_matches_torch_layers(kind):
     from torch_reference import reference_forward
