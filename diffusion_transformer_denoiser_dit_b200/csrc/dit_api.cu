@@ -152,17 +152,18 @@ struct dit_handle {
   CUtensorMap tb_u, tb_o, tb_g;     // activations as the B operand of the swapped GEMMs (box 256 rows)
   AttnMaps attn_maps;
   int force_guidance = 0;
+  int cfg_channels = 0;  // DIT_OPT_CFG_CHANNELS: guided output channels (0: all)
   // CUDA-graph replay of the whole forward (DIT_OPT_USE_GRAPH): one cached executable graph,
   // valid for the exact pointers and parameters it was captured with
   struct GraphKey {
     const void *x, *t, *y;
     float* out;
-    int B, R, depth;
+    int B, R, depth, gch;
     bool guided, pdl;
     float s;
     bool operator==(const GraphKey& o) const {
       return x == o.x && t == o.t && y == o.y && out == o.out && B == o.B && R == o.R && depth == o.depth &&
-             guided == o.guided && pdl == o.pdl && s == o.s;
+             gch == o.gch && guided == o.guided && pdl == o.pdl && s == o.s;
     }
   };
   cudaStream_t cap_stream = nullptr;
@@ -177,12 +178,12 @@ struct dit_handle {
     float* x = nullptr;
     const void* y = nullptr;
     const float* t_sched = nullptr;
-    int B = 0, R = 0, kind = 0, steps = 0;
+    int B = 0, R = 0, kind = 0, steps = 0, gch = 0;
     bool guided = false, pdl = false;
     float s = 0.f;
     std::vector<float> levels;
     bool operator==(const SampleKey& o) const {
-      return x == o.x && y == o.y && t_sched == o.t_sched && B == o.B && R == o.R && kind == o.kind &&
+      return x == o.x && y == o.y && t_sched == o.t_sched && B == o.B && R == o.R && kind == o.kind && gch == o.gch &&
              steps == o.steps && guided == o.guided && pdl == o.pdl && s == o.s && levels == o.levels;
     }
   };
@@ -745,6 +746,7 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
   da.pw = c.patch_w;
   da.guided = p.guided;
   da.s = p.s;
+  da.gch = H->cfg_channels;
   DIT_LAUNCH(H, DIT_KERNEL_DECODE, st, launch_decode_cfg(da, st), "decode");
   return DIT_OK;
 }
@@ -758,7 +760,7 @@ dit_status run_forward_cached(dit_handle* H, const float* x, const float* t, con
                               float* out, cudaStream_t st) {
   const int depth = H->cfg.depth;
   if (!H->use_graph || H->prof) return run_forward(H, x, t, y, p, depth, out, st);
-  dit_handle::GraphKey k{x, t, y, out, p.B, p.R, depth, p.guided, g_pdl, p.s};
+  dit_handle::GraphKey k{x, t, y, out, p.B, p.R, depth, H->cfg_channels, p.guided, g_pdl, p.s};
   if (H->gexec != nullptr && k == H->gkey) {
     DIT_CK(H, cudaGraphLaunch(H->gexec, st), "graph launch");
     return DIT_OK;
@@ -856,6 +858,11 @@ dit_status dit_set_option(dit_handle* H, int option, int value) {
     dit::g_pdl = value != 0;
     return DIT_OK;
   }
+  if (option == DIT_OPT_CFG_CHANNELS) {
+    if (value < 0) return fail(H, DIT_ERR_INVALID_ARG, "guided channel count must be >= 0");
+    H->cfg_channels = value;
+    return DIT_OK;
+  }
 
   return fail(H, DIT_ERR_INVALID_ARG, "unknown option");
 }
@@ -915,6 +922,7 @@ dit_status dit_sample(dit_handle* H, int kind, float* x, const void* y, int B, f
   k.R = p.R;
   k.kind = kind;
   k.steps = steps;
+  k.gch = H->cfg_channels;
   k.guided = p.guided;
   k.pdl = g_pdl;
   k.s = p.s;

@@ -145,6 +145,7 @@ struct DecodeArgs {
   const float* b;        // [P]
   float* out;            // [B, Cout, F, H, W]
   int B, T, d, P, Cout, F, H, W, pt, ph, pw, guided;
+  int gch;               // guided channels: c < gch are guided, the rest keep z_cond (0: all)
   float s;
 };
 cudaError_t launch_decode_cfg(const DecodeArgs& a, cudaStream_t st);

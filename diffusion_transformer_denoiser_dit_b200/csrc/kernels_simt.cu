@@ -476,7 +476,8 @@ cudaError_t launch_attention_simt(const AttnArgs& a, cudaStream_t st) {
 // ============================================================================ decoder + unpatchify + CFG
 // One block per (sample b, token tau).  Each warp computes decoder outputs p
 // (stride 8); lanes split the d-long dot products.  Guided: both rows b and b+B
-// are decoded and combined as z_null + s (z_cond - z_null) before the scatter to
+// are decoded and combined as z_null + s (z_cond - z_null) (on channels c < gch only
+// when gch > 0; the others keep z_cond) before the scatter to
 // out[b, c, f*pt+it, i*ph+ih, j*pw+iw] with p = ((it*ph + ih)*pw + iw)*Cout + c.
 __global__ void decode_cfg_kernel(DecodeArgs a) {
   pdl_trigger();
@@ -505,13 +506,13 @@ __global__ void decode_cfg_kernel(DecodeArgs a) {
     zc = warp_sum(zc);
     zu = warp_sum(zu);
     if (lane == 0) {
+      const int c = p % a.Cout;
       zc += a.b[p];
       float val = zc;
-      if (a.guided) {
+      if (a.guided && (a.gch <= 0 || c < a.gch)) {
         zu += a.b[p];
         val = zu + a.s * (zc - zu);
       }
-      const int c = p % a.Cout;
       const int iw = (p / a.Cout) % a.pw, ih = (p / (a.Cout * a.pw)) % a.ph, it = p / (a.Cout * a.pw * a.ph);
       const size_t oi = ((((static_cast<size_t>(b) * a.Cout + c) * a.F + f * a.pt + it) * a.H + gi * a.ph + ih) * a.W) +
                         gj * a.pw + iw;

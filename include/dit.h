@@ -207,8 +207,13 @@ void dit_destroy(dit_handle* h);
    freely.  While profiling is enabled the graph is bypassed.  If the capture fails the
    option turns itself off and the call runs directly.
    DIT_OPT_OVERLAP_LAUNCH = 0/1 (process-wide, default 1): launch each kernel with
-   programmatic dependent launch so its set-up overlaps the tail of the previous one. */
-enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2, DIT_OPT_OVERLAP_LAUNCH = 3 };
+   programmatic dependent launch so its set-up overlaps the tail of the previous one.
+   DIT_OPT_CFG_CHANNELS = n >= 0 (default 0 = every channel): classifier-free guidance
+   combines only output channels c < n; the other channels return the conditional
+   prediction.  n = 3 is the variant that "확산 트랜스포머" ("ImageNet 클래스 조건 생성")
+   attributes to the official code; guidance on every channel is the standard form.
+   A negative n is DIT_ERR_INVALID_ARG. */
+enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2, DIT_OPT_OVERLAP_LAUNCH = 3, DIT_OPT_CFG_CHANNELS = 4 };
 dit_status dit_set_option(dit_handle* h, int option, int value);
 
 /*

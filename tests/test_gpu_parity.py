@@ -338,3 +338,33 @@ def test_empty_batch_is_rejected_without_launch():
     assert bool((out == 7.0).all())
     assert m.sync_status() == binding.DIT_OK
     m.close()
+
+
+def test_guidance_on_the_first_channels_only():
+    """DIT_OPT_CFG_CHANNELS = 3 against the oracle's cfg_channels = 3; the option is part of
+    the graph cache key, so replay picks up a change."""
+    cfg = small_image_bf16_dh72()
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    want = O.forward(cfg, W, inp["x"], inp["t"], inp["y"], cfg_channels=3)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    m.set_option(binding.DIT_OPT_CFG_CHANNELS, 3)
+    direct = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    assert_parity(cfg, direct, want, "cfg_channels=3")
+    m.set_option(binding.DIT_OPT_CFG_CHANNELS, 0)
+    full = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    assert np.array_equal(full[:, :3], direct[:, :3]) and not np.array_equal(full[:, 3:], direct[:, 3:])
+    m.set_option(binding.DIT_OPT_USE_GRAPH, 1)
+    out = torch.empty(cfg.out_shape(), device="cuda")
+    for _ in range(3):
+        m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale, out=out)
+    assert np.array_equal(out.cpu().numpy(), full)
+    m.set_option(binding.DIT_OPT_CFG_CHANNELS, 3)
+    for _ in range(3):
+        m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale, out=out)
+        assert np.array_equal(out.cpu().numpy(), direct)
+    with pytest.raises(binding.DitError):
+        m.set_option(binding.DIT_OPT_CFG_CHANNELS, -1)
+    assert m.sync_status() == binding.DIT_OK
+    m.close()
