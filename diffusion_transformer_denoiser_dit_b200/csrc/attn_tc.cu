@@ -456,7 +456,10 @@ bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* 
 template <int DH>
 static cudaError_t launch_dh(const AttnArgs& a, const AttnMaps& mp, int* status, cudaStream_t st) {
   using C = AttnCfg<DH>;
-  static int num_sms = 0;
+  static int sms_of[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  int& num_sms = sms_of[dev];
   if (num_sms == 0) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
@@ -465,9 +468,10 @@ static cudaError_t launch_dh(const AttnArgs& a, const AttnMaps& mp, int* status,
     e = cudaFuncGetAttributes(&fa, attn_tc_kernel<DH>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * C::THREADS < C::REG_POOL) return cudaErrorInvalidConfiguration;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       return cudaErrorInvalidDevice;
+    num_sms = n;
   }
   const int nq = a.Tpad / 128;
   const int items = a.R * a.H * ((nq + 1) / 2);

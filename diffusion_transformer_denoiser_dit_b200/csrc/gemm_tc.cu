@@ -256,11 +256,13 @@ template <int BN, int EPI>
 static cudaError_t launch_bn(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap* tC, int K,
                              const EpiArgs& ea, int num_sms, cudaStream_t st) {
   using C = TcCfg<BN, EPI>;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static bool attr_done[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    attr_done[dev] = true;
   }
   const int tiles = ((ea.M + 127) / 128) * ((ea.N + BN - 1) / BN);
   if (tiles == 0) return cudaSuccess;

@@ -210,7 +210,10 @@ template <int BN, int EPI>
 static cudaError_t launch_pair_bn(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap* tC, int K,
                                   const EpiArgs& ea, int num_sms, cudaStream_t st) {
   using C = Tc2Cfg<BN, EPI>;
-  static int max_clusters = 0;
+  static int clusters_of[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  int& max_clusters = clusters_of[dev];
   if (max_clusters == 0) {
     cudaError_t e =
         cudaFuncSetAttribute(gemm_tc2_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);

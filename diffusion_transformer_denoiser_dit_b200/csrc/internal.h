@@ -59,6 +59,15 @@ cudaError_t launch_gemm_tc2(int epi, int block_n, const CUtensorMap* tmA, const 
                             const EpiArgs& ea, int num_sms, cudaStream_t st, const CUtensorMap* tmC = nullptr);
 int gemm_tc2_supported_bn(int block_n);
 // Build a 2-D bf16 K-major tensor map: rows x K, box = box_rows x 64, 128-byte swizzle.
+// Per-device one-time launch set-up (a kernel's shared-memory attribute is set on the
+// current device): index of the current device, or -1 if there is none or it is beyond
+// kMaxDevices.
+constexpr int kMaxDevices = 64;
+inline int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
 bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
 // 3-d bf16 map: dims d0 (innermost) x d1 x d2, box box0 x box1 x 1, 128B swizzle or none.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
