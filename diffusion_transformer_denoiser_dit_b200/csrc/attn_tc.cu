@@ -5,11 +5,13 @@
 //   warp 0    one thread streams Q (per item) and K_n / V_n^T (per key tile, two-stage
 //             rings) with TMA, no multicast; each buffer is refilled as soon as the MMA
 //             that read it completed (polled without blocking).
-//   warp 1    allocates all 512 TMEM columns (S_0, S_1, O_0, O_1) and one thread issues
+//   warp 1    allocates all 512 TMEM columns (S_0, S_1, O_0, O_1); one thread of warp 1 (group 0)
+//             and one of warp 2 (group 1) each issue
 //             S_g = Q_g K_n^T (M=128, N=128, K = dh padded to 80: a 128B- and a
 //             32B-swizzled operand) and O_g += P_g V_n (M=128, N=DP, K=128).  The Q K^T of
 //             key tile n+1 is issued before the P V of tile n, so the tensor cores run
-//             while the softmax works.
+//             while the softmax works.  Group 1 starts once group 0 has written its first P,
+//             so the two groups' exp2 phases alternate on the MUFU pipe.
 //   warps 4-7, 8-11  softmax of query group 0 / 1 (register budget raised with setmaxnreg,
 //             taken from warpgroup 0), one query row per thread: S from TMEM
 //             into registers (then S is released), online softmax in base 2 with lazy
@@ -69,6 +71,7 @@ enum {
   B_OF0, B_OF1,                      // O_g read by the epilogue (count 128)
   B_OS0, B_OS1,                      // output staging of group g free (previous store read it)
   B_OW0, B_OW1,                      // output staging of group g written (count 128)
+  B_GO,                              // group 0 wrote its first P: group 1 may start (completes once)
   B_COUNT
 };
 
@@ -101,7 +104,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < B_COUNT; ++i) {
       const bool all = i == B_SF0 || i == B_SF1 || i == B_P0 || i == B_P1 || i == B_OF0 || i == B_OF1 ||
                        i == B_OW0 || i == B_OW1;
-      mbar_init(BAR(i), all ? 128 : 1);
+      const bool both_issuers = i == B_QE || i == B_KE0 || i == B_KE1 || i == B_VE0 || i == B_VE1;
+      mbar_init(BAR(i), all ? 128 : both_issuers ? 2 : 1);
     }
     fence_barrier_init();
   }
@@ -169,14 +173,21 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_2d(vdst + C::V_ATOM, &tmV, BAR(B_VF0 + st), j * 128 + 64, rh * C::DP);
         }
       }
-    } else if (warp == 1 && lane == 0) {  // ---------------- MMA issuer
+    } else if ((warp == 1 || warp == 2) && lane == 0) {  // ---- MMA issuers: warp 1 group 0, warp 2 group 1
+      // One issuing thread per query group, so neither group's MMAs queue behind the other's
+      // and each issuer's serial chain stays short.  The shared K / V stages and the Q buffer
+      // are released by both issuers (barrier count 2); an issuer whose group has no part in
+      // an item still releases them (a commit with nothing new to track), and every release
+      // comes after the matching full-barrier wait, so no issuer can run two phases ahead.
+      const int g = warp - 1;
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, C::DP);
-      // The issuing thread is a serial chain that shares its scheduler with two softmax
-      // warps, so the per-tile path does no division: items and key tiles are followed by
-      // cursors, and every descriptor is a constant high word plus base + offset.
-      const uint32_t q_lo = sdesc_lo(sbase + C::OFF_Q), k_lo = sdesc_lo(sbase + C::OFF_K);
-      const uint32_t v_lo = sdesc_lo(sbase + C::OFF_V), p_lo = sdesc_lo(sbase + C::OFF_P);
+      // No division in the per-tile path: items and key tiles are followed by cursors, and
+      // every descriptor is a constant high word plus base + offset.
+      const uint32_t qb = sdesc_lo(sbase + C::OFF_Q) + g * (C::QK_TILE >> 4);
+      const uint32_t k_lo = sdesc_lo(sbase + C::OFF_K), v_lo = sdesc_lo(sbase + C::OFF_V);
+      const uint32_t pb = sdesc_lo(sbase + C::OFF_P) + g * (C::P_TILE >> 4);
+      const uint32_t tS = tmem_base + g * 128, tO = tmem_base + 256 + g * 128;
       const int pmod = static_cast<int>(gridDim.x) % pairs;
       struct Cursor {
         int li, j, pidx, ng;  // item, key tile in the item, query-tile pair of the item, groups
@@ -195,23 +206,17 @@ __global__ void __launch_bounds__(384, 1)
           c.ng = 2 * c.pidx + 1 < nq ? 2 : 1;
         }
       };
-      int qk_cnt[2] = {0, 0};  // Q K^T issued per query group
-      int pv_cnt[2] = {0, 0};  // P V issued per query group
-      int it_cnt[2] = {0, 0};  // items whose first P V was issued, per group
+      int qk_cnt = 0, pv_cnt = 0, it_cnt = 0;  // this group's Q K^T, P V and started items
       Cursor cq = first(), cp = first();
-      // S_g = Q_g K_n^T for every query group of tile n (cursor cq is at tile n)
+      // S_g = Q_g K_n^T (cursor cq is at tile n)
       auto issue_qk = [&](int n) -> bool {
         if (cq.j == 0 && !mbar_wait(BAR(B_QF), cq.li & 1, status)) return false;
         if (!mbar_wait(BAR(B_KF0 + (n & 1)), (n >> 1) & 1, status)) return false;
-        const uint32_t kb = k_lo + (n & 1) * (C::QK_TILE >> 4);
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          if (g >= cq.ng) break;
+        if (g < cq.ng) {
           // S_g may be overwritten once the softmax of group g has read its previous tile
-          if (qk_cnt[g] > 0 && !mbar_wait(BAR(B_SF0 + g), (qk_cnt[g] - 1) & 1, status)) return false;
+          if (qk_cnt > 0 && !mbar_wait(BAR(B_SF0 + g), (qk_cnt - 1) & 1, status)) return false;
           tc_fence_after();
-          const uint32_t qb = q_lo + g * (C::QK_TILE >> 4);
-          const uint32_t tS = tmem_base + g * 128;
+          const uint32_t kb = k_lo + (n & 1) * (C::QK_TILE >> 4);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_bf16_ss(tS, sdesc_make(qb + 2 * k, kSdescHiSw128), sdesc_make(kb + 2 * k, kSdescHiSw128), idesc_s,
@@ -220,35 +225,31 @@ __global__ void __launch_bounds__(384, 1)
             mma_bf16_ss(tS, sdesc_make(qb + (C::MAIN >> 4), kSdescHiSw32), sdesc_make(kb + (C::MAIN >> 4), kSdescHiSw32),
                         idesc_s, 1u);
           mma_commit(BAR(B_S0 + g));
-          ++qk_cnt[g];
+          ++qk_cnt;
         }
         mma_commit(BAR(B_KE0 + (n & 1)));
         if (cq.j == nk - 1) mma_commit(BAR(B_QE));
         advance(cq);
         return true;
       };
-      // O_g (+)= P_g V_n for every query group of tile n (cursor cp is at tile n)
+      // O_g (+)= P_g V_n (cursor cp is at tile n)
       auto issue_pv = [&](int n) -> bool {
         if (!mbar_wait(BAR(B_VF0 + (n & 1)), (n >> 1) & 1, status)) return false;
-        const uint32_t vb = v_lo + (n & 1) * (C::V_TILE >> 4);
-        const bool first_tile = cp.j == 0;
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          if (g >= cp.ng) break;
-          if (!mbar_wait(BAR(B_P0 + g), pv_cnt[g] & 1, status)) return false;
+        if (g < cp.ng) {
+          const bool first_tile = cp.j == 0;
+          if (!mbar_wait(BAR(B_P0 + g), pv_cnt & 1, status)) return false;
           // a new item overwrites O_g: its epilogue for the previous item must have read it
-          if (first_tile && it_cnt[g] > 0 && !mbar_wait(BAR(B_OF0 + g), (it_cnt[g] - 1) & 1, status)) return false;
+          if (first_tile && it_cnt > 0 && !mbar_wait(BAR(B_OF0 + g), (it_cnt - 1) & 1, status)) return false;
           tc_fence_after();
-          const uint32_t pb = p_lo + g * (C::P_TILE >> 4);
-          const uint32_t tO = tmem_base + 256 + g * 128;
+          const uint32_t vb = v_lo + (n & 1) * (C::V_TILE >> 4);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mma_bf16_ss(tO, sdesc_make(pb + (k >> 2) * (C::MAIN >> 4) + (k & 3) * 2, kSdescHiSw128),
                         sdesc_make(vb + (k >> 2) * (C::V_ATOM >> 4) + (k & 3) * 2, kSdescHiSw128), idesc_o,
                         (!first_tile || k > 0) ? 1u : 0u);
           mma_commit(BAR(B_O0 + g));
-          ++pv_cnt[g];
-          if (first_tile) ++it_cnt[g];
+          ++pv_cnt;
+          if (first_tile) ++it_cnt;
         }
         mma_commit(BAR(B_VE0 + (n & 1)));
         advance(cp);
@@ -259,6 +260,10 @@ __global__ void __launch_bounds__(384, 1)
       // next item's Q is loaded only after the current item's last Q K^T).
       int n_qk = 0;
       bool ok = true;
+      // Group 1 starts about half a key-tile period behind group 0 (once group 0 has written
+      // its first P), so that the two groups' exp2 phases alternate on the MUFU pipe instead
+      // of coinciding; group 0 needs nothing from group 1 to get there.
+      if (g == 1 && !mbar_wait(BAR(B_GO), 0, status)) ok = false;
       for (int n = 0; n < ntiles && ok; ++n) {
         while (ok && (n_qk <= n || (n_qk == n + 1 && n_qk < ntiles && cq.j != 0))) ok = issue_qk(n_qk++);
         if (ok) ok = issue_pv(n);
@@ -376,6 +381,7 @@ __global__ void __launch_bounds__(384, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(B_P0 + g));
+        if (g == 0 && cnt == 0 && q == 0 && lane == 0) mbar_arrive(BAR(B_GO));
       }
       if (!ok) break;
       // item epilogue: O_g / l through shared memory to global memory (one TMA store)
@@ -456,10 +462,7 @@ bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* 
 template <int DH>
 static cudaError_t launch_dh(const AttnArgs& a, const AttnMaps& mp, int* status, cudaStream_t st) {
   using C = AttnCfg<DH>;
-  static int sms_of[kMaxDevices] = {};
-  const int dev = current_device();
-  if (dev < 0) return cudaErrorInvalidDevice;
-  int& num_sms = sms_of[dev];
+  static int num_sms = 0;
   if (num_sms == 0) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
@@ -468,10 +471,9 @@ static cudaError_t launch_dh(const AttnArgs& a, const AttnMaps& mp, int* status,
     e = cudaFuncGetAttributes(&fa, attn_tc_kernel<DH>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * C::THREADS < C::REG_POOL) return cudaErrorInvalidConfiguration;
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return cudaErrorInvalidDevice;
-    num_sms = n;
   }
   const int nq = a.Tpad / 128;
   const int items = a.R * a.H * ((nq + 1) / 2);
