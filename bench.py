@@ -35,7 +35,7 @@ CFG = S.DIT_XL2_CFG256
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one launch of each kernel, from the cold-cache ncu captures
 # summarised in profiles/xl2_cfg256_kernels_ncu.md; set to None when a kernel changes.
-TRAFFIC_BYTES = {"fc1": 58.6e6, "fc2": 128.5e6, "qkv": 43.0e6, "proj": 59.5e6, "attn": None, "ln": 38.1e6}
+TRAFFIC_BYTES = {"fc1": 58.6e6, "fc2": 128.5e6, "qkv": 43.0e6, "proj": 59.5e6, "attn": 65.4e6, "ln": 38.1e6}
 # fallback peaks (used only when MEASURED_PEAKS.json is absent)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
