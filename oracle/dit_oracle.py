@@ -19,7 +19,7 @@ Sources (web pages on the Diffusion Transformer; cited by title and section):
               §2.2 (full attention, 3D RoPE, Q-K normalisation), §2.3 (rectified
               flow: the network predicts a velocity).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * timestep sinusoid: 256 dims, half = 128, f_i = 10000^(-i/128), layout
     [cos | sin], argument t * t_scale (t_scale = 1 for integer steps, 1000 for
     t in [0, 1));

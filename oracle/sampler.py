@@ -12,7 +12,7 @@ Sources (cited by page title and section):
               flow): x_t = t x_1 + (1 - t) x_0, the network predicts the velocity that
               moves x_t toward x_1.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * the epsilon step is the deterministic one implied by the forward process: the
     clean latent implied by the predicted noise is carried to the next noise level
     with the same noise (no fresh noise is drawn);
