@@ -17,7 +17,11 @@
  *   classifier-free guidance  e = e(null) + s (e(c) - e(null))   "Sora / DiT", guidance bullet;
  *   video variant: spacetime patches, QK-RMSNorm and 3D RoPE, velocity head
  *                                                                "GOKU : Flow Based Video
- *     Generative Foundation Models" (blog.outta.ai), sections 2.2 and 2.3.
+ *     Generative Foundation Models" (blog.outta.ai), sections 2.2 and 2.3;
+ *   and the sampler update around it (dit_sampler_step, dit_sample): a deterministic
+ *     step of the DDPM forward process x_t = sqrt(abar_t) x_0 + sqrt(1-abar_t) eps
+ *     ("Sora / DiT", training-objective bullet) or an Euler step of the rectified-flow
+ *     path x_t = t x_1 + (1-t) x_0 ("GOKU", section 2.3).
  *
  * Conventions for every entry point:
  *   - Pointers named "dev" are CUDA device pointers on the current device; "host"
@@ -117,7 +121,8 @@ int dit_weight_count(const dit_config* cfg);
  *   y   dev int32 [B] class labels (DIT_COND_CLASS) or float32 [B, d] (DIT_COND_VECTOR)
  *   out dev float32 [B, C_out, (F,) H, W]
  * Guidance: with a class-conditional model and cfg_scale != 1 the library runs 2B
- * rows, [x; x] with labels [y; num_classes], and writes e(null) + s (e(y) - e(null)).
+ * rows, [x; x] with labels [y; num_classes], and writes e(null) + s (e(y) - e(null))
+ * on every output channel (or on the first n only, see DIT_OPT_CFG_CHANNELS).
  * Otherwise it runs B rows and writes e(y).  1 <= B <= max_batch.
  * One forward may be in flight per handle (the handle owns one workspace); the
  * handle is not thread-safe.  Buffers must stay valid until the stream reaches
