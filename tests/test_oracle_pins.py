@@ -185,9 +185,28 @@ def test_sincos_2d_invariants():
     assert abs(pe[tok(0, 1), d // 2] - math.sin(1.0)) < 1e-15               # w_0 = 1
 
 
+def test_token_coords_follow_the_patchify_token_order():
+    """Each token's (frame, row, col) on the patch grid, fixed by the tokenisation itself: a
+    latent whose channels hold each element's own frame, row and column index is patchified
+    (patchify is pinned to a Conv3d with kernel = stride = patch below), and token tau's patch
+    must start at (frame, row, col) = patch extent x token_coords(tau)."""
+    for (pt, ph, pw), (F_, H, W) in (((1, 2, 2), (3, 8, 6)), ((2, 1, 3), (4, 5, 9)), ((1, 4, 4), (1, 16, 8))):
+        f, i, j = np.meshgrid(np.arange(F_), np.arange(H), np.arange(W), indexing="ij")
+        x = np.stack([f, i, j]).astype(np.float64)[None]          # [1, 3, F, H, W]
+        v = O.patchify(x, pt, ph, pw)[0]                           # [T, 3 * pt * ph * pw]
+        n = pt * ph * pw
+        start = np.stack([v[:, 0], v[:, n], v[:, 2 * n]], axis=1)  # first element of each channel
+        grid = (F_ // pt, H // ph, W // pw)
+        assert np.array_equal(O.token_coords(grid) * np.array([pt, ph, pw]), start)
+    # a frame/row swap is caught whenever the two extents differ
+    swapped = O.token_coords((2, 3, 4))[:, [1, 0, 2]]
+    assert not np.array_equal(swapped, O.token_coords((2, 3, 4)))
+
+
 def test_rope_invariants():
     rng = np.random.default_rng(6)
-    coords = O.token_coords((2, 3, 4))
+    # explicit (frame, row, col) triples, independent of token_coords
+    coords = np.array([[f, r, c] for f in range(2) for r in range(3) for c in range(4)])
     q = rng.standard_normal((24, 72))
     k = rng.standard_normal((24, 72))
     rq = O.rope_3d(q, coords)
@@ -196,9 +215,11 @@ def test_rope_invariants():
     shifted = coords + np.array([3, -2, 5])
     assert np.allclose(O.rope_3d(q, coords) @ O.rope_3d(k, coords).T,
                        O.rope_3d(q, shifted) @ O.rope_3d(k, shifted).T)
-    # first pair of the time slice turns by exactly the frame index (theta_0 = 1)
-    ang = math.atan2(rq[12, 1], rq[12, 0]) - math.atan2(q[12, 1], q[12, 0])
-    assert abs(math.remainder(ang - coords[12, 0], 2 * math.pi)) < 1e-12
+    # the first pair of each slice (theta_0 = 1) turns by exactly that axis' coordinate:
+    # token 23 is (frame 1, row 2, col 3)
+    for a, want in enumerate((1, 2, 3)):
+        ang = math.atan2(rq[23, 24 * a + 1], rq[23, 24 * a]) - math.atan2(q[23, 24 * a + 1], q[23, 24 * a])
+        assert abs(math.remainder(ang - want, 2 * math.pi)) < 1e-12
 
 
 def test_patchify_is_conv_and_unpatchify_is_rearrange():
@@ -346,6 +367,23 @@ _PLANTS = {
     "ln_eps": ("layernorm", lambda x, eps=1e-6: O.__dict__["_orig_layernorm"](x, eps=1e-2)),
     "attn_scale": ("attention", None),
 }
+
+
+def test_oracle_catches_a_frame_row_swap_in_token_coords(monkeypatch):
+    """The torch-layer cross-check derives each token's RoPE coordinates from the Conv3d
+    output layout, not from the oracle, so swapping frame and row in token_coords shows."""
+    from torch_reference import reference_forward
+    cfg = small_video()
+    assert cfg.grid[0] != cfg.grid[1]
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    Wd = S.weight_dict(cfg, W)
+    inp = S.make_inputs(cfg)
+    want = reference_forward(cfg, Wd, inp["x"], inp["t"], inp["y"])
+    orig = O.token_coords
+    monkeypatch.setattr(O, "token_coords", lambda grid: orig(grid)[:, [1, 0, 2]])
+    got = O.forward(cfg, Wd, inp["x"], inp["t"], inp["y"])
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    assert rel > 1e-7, rel
 
 
 @pytest.mark.parametrize("plant", sorted(_PLANTS))

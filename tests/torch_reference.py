@@ -8,7 +8,8 @@ LayerNorm is ``nn.LayerNorm(elementwise_affine=False, eps=1e-6)``, the FFN uses
 ``nn.GELU(approximate="tanh")``, unpatchify is an einops rearrangement of the
 literal p x p x C_out token vector.  The fixed tables (timestep sinusoid, 2D
 sin-cos positions, RoPE rotation) are taken from the oracle because each is
-pinned on its own by invariants in test_oracle_pins.py.
+pinned on its own by invariants in test_oracle_pins.py; the tokens' RoPE
+coordinates are derived here from the patch layout, not taken from the oracle.
 """
 from __future__ import annotations
 
@@ -87,6 +88,20 @@ class RefBlock(nn.Module):
         return x + g2[:, None] * self.mlp(h)
 
 
+def conv_token_coords(cfg, extent):
+    """(frame, row, col) of every token, read off the tokenisation itself: three planes holding
+    each latent element's own frame, row and column index go through the same stride-p
+    pooling and flatten(2) as the patch tokens, so token tau gets the coordinate of the patch it
+    came from (divided by the patch extent)."""
+    F_, H, W = (int(e) for e in extent)
+    axes = torch.meshgrid(torch.arange(F_, dtype=T64), torch.arange(H, dtype=T64), torch.arange(W, dtype=T64),
+                          indexing="ij")
+    k = (cfg.patch_t, cfg.patch_h, cfg.patch_w)
+    pooled = F.avg_pool3d(torch.stack(axes)[None], k, stride=k).flatten(2)[0]   # [3, T] patch centres
+    low = pooled - (torch.tensor(k, dtype=T64)[:, None] - 1) / 2                 # patch start
+    return (low / torch.tensor(k, dtype=T64)[:, None]).round().to(torch.int64).T.numpy()
+
+
 def reference_forward(cfg, weights_by_name, x, t, y, cfg_scale=None, force_guidance=False):
     W = weights_by_name
     d = cfg.hidden
@@ -125,7 +140,7 @@ def reference_forward(cfg, weights_by_name, x, t, y, cfg_scale=None, force_guida
         else:
             c = c + _t(y)
 
-        coords = O.token_coords(cfg.grid) if cfg.pos_kind == 1 else None
+        coords = conv_token_coords(cfg, x.shape[2:]) if cfg.pos_kind == 1 else None
         for i in range(cfg.depth):
             blk = RefBlock(d, cfg.heads, cfg.mlp_hidden, cfg.qk_norm).to(T64)
             blk.load(W, f"blocks.{i}.")
