@@ -26,6 +26,8 @@ import numpy as np
 DTYPE_F32, DTYPE_BF16 = 0, 1
 POS_SINCOS2D, POS_ROPE3D = 0, 1
 COND_CLASS, COND_VECTOR = 0, 1
+# how the condition enters the blocks (the four designs of the DiT paper's comparison)
+BLOCK_ADALN_ZERO, BLOCK_IN_CONTEXT, BLOCK_CROSS_ATTN, BLOCK_ADALN = 0, 1, 2, 3
 
 
 @dataclass(frozen=True)
@@ -55,6 +57,7 @@ class DiTConfig:
     batch: int
     cfg_scale: float
     index: int = -1  # position in the standard workload list (seeds); -1 = ad hoc
+    block_kind: int = BLOCK_ADALN_ZERO
 
     # ---- derived shapes (no arithmetic of the method) ----
     @property
@@ -65,6 +68,21 @@ class DiTConfig:
     def tokens(self) -> int:
         g = self.grid
         return g[0] * g[1] * g[2]
+
+    @property
+    def cond_tokens(self) -> int:
+        """Condition tokens ahead of the patch tokens in each row (in-context design: 2)."""
+        return 2 if self.block_kind == BLOCK_IN_CONTEXT else 0
+
+    @property
+    def seq_tokens(self) -> int:
+        """Tokens per row inside the blocks."""
+        return self.tokens + self.cond_tokens
+
+    @property
+    def mod_per_block(self) -> int:
+        """Modulation vectors regressed per block: 6 (adaLN-Zero), 4 (adaLN), 0 (others)."""
+        return {BLOCK_ADALN_ZERO: 6, BLOCK_ADALN: 4}.get(self.block_kind, 0)
 
     @property
     def head_dim(self) -> int:
@@ -143,11 +161,13 @@ def inputs_seed(cfg: DiTConfig) -> int:
 def weight_specs(cfg: DiTConfig) -> List[Tuple[str, Tuple[int, ...], str]]:
     """(name, shape, init) for every weight, in the library's fixed order.
 
-    Linear weights are row-major [out, in].  ``init`` is "normal" (N(0, std)) or
-    "one" (filled with 1.0, used for the QK-RMSNorm gains).
+    Linear weights are row-major [out, in].  ``init`` is "normal" (N(0, std)), "one"
+    (filled with 1.0, used for the QK-RMSNorm gains) or "gain" (1 + N(0, 0.1), the learned
+    LayerNorm gains of the in-context and cross-attention designs).
     """
     d, f, m = cfg.hidden, cfg.freq_dim, cfg.mlp_hidden
     dh = cfg.head_dim
+    kind = cfg.block_kind
     s: List[Tuple[str, Tuple[int, ...], str]] = [
         ("pe.w", (d, cfg.patch_dim), "normal"), ("pe.b", (d,), "normal"),
         ("t.w1", (d, f), "normal"), ("t.b1", (d,), "normal"),
@@ -155,17 +175,32 @@ def weight_specs(cfg: DiTConfig) -> List[Tuple[str, Tuple[int, ...], str]]:
     ]
     if cfg.cond_kind == COND_CLASS:
         s.append(("y.table", (cfg.num_classes + 1, d), "normal"))
+    modulated = kind in (BLOCK_ADALN_ZERO, BLOCK_ADALN)
     for i in range(cfg.depth):
         p = f"blocks.{i}."
-        s += [(p + "ada.w", (6 * d, d), "normal"), (p + "ada.b", (6 * d,), "normal"),
-              (p + "qkv.w", (3 * d, d), "normal"), (p + "qkv.b", (3 * d,), "normal")]
+        if modulated:
+            nm = cfg.mod_per_block
+            s += [(p + "ada.w", (nm * d, d), "normal"), (p + "ada.b", (nm * d,), "normal")]
+        else:
+            s += [(p + "ln1.g", (d,), "gain"), (p + "ln1.b", (d,), "normal")]
+        s += [(p + "qkv.w", (3 * d, d), "normal"), (p + "qkv.b", (3 * d,), "normal")]
         if cfg.qk_norm:
             s += [(p + "q_norm.g", (dh,), "one"), (p + "k_norm.g", (dh,), "one")]
-        s += [(p + "proj.w", (d, d), "normal"), (p + "proj.b", (d,), "normal"),
-              (p + "fc1.w", (m, d), "normal"), (p + "fc1.b", (m,), "normal"),
+        s += [(p + "proj.w", (d, d), "normal"), (p + "proj.b", (d,), "normal")]
+        if kind == BLOCK_CROSS_ATTN:
+            s += [(p + "xln.g", (d,), "gain"), (p + "xln.b", (d,), "normal"),
+                  (p + "xq.w", (d, d), "normal"), (p + "xq.b", (d,), "normal"),
+                  (p + "xkv.w", (2 * d, d), "normal"), (p + "xkv.b", (2 * d,), "normal"),
+                  (p + "xo.w", (d, d), "normal"), (p + "xo.b", (d,), "normal")]
+        if not modulated:
+            s += [(p + "ln2.g", (d,), "gain"), (p + "ln2.b", (d,), "normal")]
+        s += [(p + "fc1.w", (m, d), "normal"), (p + "fc1.b", (m,), "normal"),
               (p + "fc2.w", (d, m), "normal"), (p + "fc2.b", (d,), "normal")]
-    s += [("final.ada.w", (2 * d, d), "normal"), ("final.ada.b", (2 * d,), "normal"),
-          ("dec.w", (cfg.out_dim, d), "normal"), ("dec.b", (cfg.out_dim,), "normal")]
+    if modulated:
+        s += [("final.ada.w", (2 * d, d), "normal"), ("final.ada.b", (2 * d,), "normal")]
+    else:
+        s += [("final.ln.g", (d,), "gain"), ("final.ln.b", (d,), "normal")]
+    s += [("dec.w", (cfg.out_dim, d), "normal"), ("dec.b", (cfg.out_dim,), "normal")]
     return s
 
 
@@ -176,6 +211,8 @@ def make_weights(cfg: DiTConfig, seed: int | None = None, std: float = 0.02) -> 
     for _, shape, init in weight_specs(cfg):
         if init == "one":
             a = np.ones(shape, dtype=np.float32)
+        elif init == "gain":
+            a = np.float32(1.0) + np.float32(0.1) * rng.standard_normal(shape, dtype=np.float32)
         else:
             a = rng.standard_normal(shape, dtype=np.float32)
             a *= np.float32(std)
@@ -198,6 +235,12 @@ def set_adaln(cfg: DiTConfig, weights: List[np.ndarray], *, zero: bool = False,
     d = cfg.hidden
     out = [w.copy() for w in weights]
     names = [n for n, _, _ in weight_specs(cfg)]
+    if cfg.block_kind != BLOCK_ADALN_ZERO:
+        if cfg.block_kind == BLOCK_ADALN and zero:
+            for i in range(cfg.depth):
+                out[names.index(f"blocks.{i}.ada.w")][...] = 0.0
+                out[names.index(f"blocks.{i}.ada.b")][...] = 0.0
+        return out   # gates exist only in the adaLN-Zero design
     for i in range(cfg.depth):
         wi = names.index(f"blocks.{i}.ada.w")
         bi = names.index(f"blocks.{i}.ada.b")

@@ -98,6 +98,13 @@ def rmsnorm(x, gain, eps: float = 1e-6):
     return x / np.sqrt((x ** 2).mean(axis=-1, keepdims=True) + eps) * np.asarray(gain, dtype=F64)
 
 
+def layernorm_affine(x, gain, bias, eps: float = 1e-6):
+    """LayerNorm with its learned per-feature scale and shift, the normalisation of the
+    in-context and cross-attention designs ([DiT-wiki] "조건 주입 방식": adaLN replaces
+    exactly these learned constants with values regressed from t + c)."""
+    return layernorm(x, eps) * np.asarray(gain, dtype=F64) + np.asarray(bias, dtype=F64)
+
+
 def modulate(x, shift, scale):
     """x * (1 + scale) + shift, shift/scale broadcast over the token axis
     ([DiT-wiki] "adaLN-Zero": LN(x)(1 + gamma) + beta)."""
@@ -220,19 +227,26 @@ def unpatchify(z, c_out: int, grid, pt: int, ph: int, pw: int):
 # --------------------------------------------------------------------------- #
 # condition and guidance
 # --------------------------------------------------------------------------- #
-def condition(cfg, W: Dict[str, np.ndarray], t, y):
-    """c = MLP(sinusoid(t)) + e(y): the timestep embedding summed with the class
-    embedding ([DiT-wiki] "adaLN-Zero": c is the sum of the time and class
-    embeddings; "조건 주입 방식": gamma, beta regressed from t + c).  For the
-    text-conditioned video model e(y) is the pooled text vector itself."""
+def condition_parts(cfg, W: Dict[str, np.ndarray], t, y):
+    """The two condition embeddings: e_t = MLP(sinusoid(t)) (a two-layer SiLU MLP on the
+    timestep features) and e_y = the class embedding (a row of the label table), or for the
+    text-conditioned video model the pooled text vector itself."""
     e = timestep_embedding(t, cfg.freq_dim, cfg.t_scale)
     hid = silu(linear(e, W["t.w1"], W["t.b1"]))
-    c = linear(hid, W["t.w2"], W["t.b2"])
+    et = linear(hid, W["t.w2"], W["t.b2"])
     if cfg.cond_kind == 0:
-        c = c + np.asarray(W["y.table"], dtype=F64)[np.asarray(y, dtype=np.int64)]
+        ey = np.asarray(W["y.table"], dtype=F64)[np.asarray(y, dtype=np.int64)]
     else:
-        c = c + np.asarray(y, dtype=F64)
-    return c
+        ey = np.asarray(y, dtype=F64)
+    return et, ey
+
+
+def condition(cfg, W: Dict[str, np.ndarray], t, y):
+    """c = e_t + e_y: the timestep embedding summed with the class embedding ([DiT-wiki]
+    "adaLN-Zero": c is the sum of the time and class embeddings; "조건 주입 방식": gamma,
+    beta regressed from t + c)."""
+    et, ey = condition_parts(cfg, W, t, y)
+    return et + ey
 
 
 def cfg_combine(eps_cond, eps_uncond, s: float, channels: Optional[int] = None):
@@ -300,6 +314,56 @@ def dit_block(x, sc, W: Dict[str, np.ndarray], prefix: str, heads: int, coords=N
     return x + g2[:, None, :] * f
 
 
+def cross_attention(u, ctx, wq, bq, wkv, bkv, wo, bo, heads: int):
+    """Multi-head cross-attention of the tokens u [R, T, d] onto the condition sequence
+    ctx [R, S, d] ([DiT-wiki] "조건 주입 방식": t and c embeddings kept as a separate
+    sequence, a cross-attention layer added to every block; [Sora-DiT]: a multi-head
+    cross-attention layer after the self-attention layer): queries from u, keys and values
+    from ctx, per-head softmax attention, heads concatenated, output projection."""
+    r, t, d = u.shape
+    dh = d // heads
+    q = linear(u, wq, bq)
+    kv = linear(ctx, wkv, bkv)
+    k, v = kv[..., :d], kv[..., d:]
+    o = np.zeros((r, t, d), dtype=F64)
+    for i in range(r):
+        for hd in range(heads):
+            sl = slice(hd * dh, (hd + 1) * dh)
+            o[i, :, sl] = attention(q[i, :, sl], k[i, :, sl], v[i, :, sl])
+    return linear(o, wo, bo)
+
+
+def plain_block(x, W: Dict[str, np.ndarray], prefix: str, heads: int, coords=None, ctx=None):
+    """The block of the in-context and cross-attention designs: a pre-norm transformer block
+    with learned LayerNorm affines and no modulation or gate.
+        x <- x + Attn(LN1(x));  [x <- x + CrossAttn(LNx(x), ctx)];  x <- x + FFN(LN2(x))."""
+    qn = W.get(prefix + "q_norm.g")
+    kn = W.get(prefix + "k_norm.g")
+    u = layernorm_affine(x, W[prefix + "ln1.g"], W[prefix + "ln1.b"])
+    x = x + self_attention(u, W[prefix + "qkv.w"], W[prefix + "qkv.b"], W[prefix + "proj.w"],
+                           W[prefix + "proj.b"], heads, qn, kn, coords)
+    if ctx is not None:
+        u = layernorm_affine(x, W[prefix + "xln.g"], W[prefix + "xln.b"])
+        x = x + cross_attention(u, ctx, W[prefix + "xq.w"], W[prefix + "xq.b"], W[prefix + "xkv.w"],
+                                W[prefix + "xkv.b"], W[prefix + "xo.w"], W[prefix + "xo.b"], heads)
+    u = layernorm_affine(x, W[prefix + "ln2.g"], W[prefix + "ln2.b"])
+    return x + ffn(u, W[prefix + "fc1.w"], W[prefix + "fc1.b"], W[prefix + "fc2.w"], W[prefix + "fc2.b"])
+
+
+def adaln_block(x, sc, W: Dict[str, np.ndarray], prefix: str, heads: int, coords=None):
+    """The adaLN design ([DiT-wiki] "조건 주입 방식": LN's scale and shift regressed from the
+    t + c embedding instead of learned constants; no residual gate):
+        (b1, g1, b2, g2) = Linear(SiLU(c));  x <- x + Attn(LN(x)(1+g1)+b1);  x <- x + FFN(LN(x)(1+g2)+b2)."""
+    sh1, sc1, sh2, sc2 = adaln_chunks(sc, W[prefix + "ada.w"], W[prefix + "ada.b"], 4)
+    qn = W.get(prefix + "q_norm.g")
+    kn = W.get(prefix + "k_norm.g")
+    u = modulate(layernorm(x), sh1, sc1)
+    x = x + self_attention(u, W[prefix + "qkv.w"], W[prefix + "qkv.b"], W[prefix + "proj.w"],
+                           W[prefix + "proj.b"], heads, qn, kn, coords)
+    u = modulate(layernorm(x), sh2, sc2)
+    return x + ffn(u, W[prefix + "fc1.w"], W[prefix + "fc1.b"], W[prefix + "fc2.w"], W[prefix + "fc2.b"])
+
+
 def final_layer(x, sc, W):
     """Final modulated LN and linear decoder to pt*ph*pw*C_out per token."""
     shift, scale = adaln_chunks(sc, W["final.ada.w"], W["final.ada.b"], 2)
@@ -351,16 +415,41 @@ def forward(cfg, weights: Sequence[np.ndarray] | Dict[str, np.ndarray], x, t, y,
         x5 = np.concatenate([x5, x5], axis=0)
         t = np.concatenate([t, t], axis=0)
         y = np.concatenate([np.asarray(y), np.full(b, cfg.num_classes, dtype=np.int64)], axis=0)
+    kind = getattr(cfg, "block_kind", 0)
     h = embed(cfg, W, x5)
-    sc = silu(condition(cfg, W, t, y))
+    et, ey = condition_parts(cfg, W, t, y)
+    sc = silu(et + ey)
     coords = token_coords(cfg.grid) if cfg.pos_kind == 1 else None
+    ctx = None
+    if kind == 1:
+        # in-context: the two condition embeddings become two extra tokens in front of the
+        # patch tokens ([DiT-wiki] "조건 주입 방식": appended like ViT's cls token); they carry
+        # no position (3D RoPE, when used, gives them coordinate 0, an identity rotation)
+        h = np.concatenate([et[:, None, :], ey[:, None, :], h], axis=1)
+        if coords is not None:
+            coords = np.concatenate([np.zeros((2, 3), dtype=coords.dtype), coords], axis=0)
+    elif kind == 2:
+        ctx = np.stack([et, ey], axis=1)   # the separate length-two condition sequence
     if stop_after_block == 0:
         return h
     for i in range(cfg.depth):
-        h = dit_block(h, sc, W, f"blocks.{i}.", cfg.heads, coords)
+        p = f"blocks.{i}."
+        if kind == 0:
+            h = dit_block(h, sc, W, p, cfg.heads, coords)
+        elif kind == 3:
+            h = adaln_block(h, sc, W, p, cfg.heads, coords)
+        else:
+            h = plain_block(h, W, p, cfg.heads, coords, ctx)
         if stop_after_block is not None and i + 1 == stop_after_block:
             return h
-    z = final_layer(h, sc, W)
+    if kind in (1, 2):
+        # the condition tokens leave the sequence after the last block; final LN (learned
+        # affine) and the linear decoder ([DiT-wiki] "잠재 공간과 패치화": final layer norm,
+        # then the linear decoder)
+        h = h[:, 2:] if kind == 1 else h
+        z = linear(layernorm_affine(h, W["final.ln.g"], W["final.ln.b"]), W["dec.w"], W["dec.b"])
+    else:
+        z = final_layer(h, sc, W)
     img = unpatchify(z, cfg.out_channels, cfg.grid, cfg.patch_t, cfg.patch_h, cfg.patch_w)
     if guided:
         img = cfg_combine(img[:b], img[b:], s, cfg_channels)

@@ -55,6 +55,17 @@ def test_mac_counter_reproduces_printed_gflops(row):
     assert abs(g - float(printed)) <= 0.1, (size, g, printed)
 
 
+@pytest.mark.parametrize("row", _rows("gflops_conditioning.txt"))
+def test_mac_counter_reproduces_conditioning_table(row):
+    """The four conditioning designs' printed DiT-XL/2 Gflops: in-context adds two tokens to
+    every row, cross-attention adds a query and an output projection per token and block, and
+    neither keeps the per-block modulation MLP (with it, 119.58 and 137.83 would be off)."""
+    name, kind, printed = row
+    cfg = S.DIT_XL2_CFG256.with_(block_kind=int(kind))
+    g = O.count_forward_macs(cfg) / 1e9
+    assert abs(g - float(printed)) <= 0.1, (name, g, printed)
+
+
 def test_mac_counter_range_ends():
     rng = dict((r[0], float(r[1])) for r in _rows("gflops_range.txt"))
     low = O.count_forward_macs(S.DIT_S8_F32) / 1e9
@@ -358,6 +369,94 @@ def test_forward_matches_torch_layers(kind):
     want = reference_forward(cfg, S.weight_dict(cfg, W), inp["x"], inp["t"], inp["y"])
     assert got.shape == want.shape == cfg.out_shape()
     assert np.allclose(got, want, rtol=1e-9, atol=1e-10), np.abs(got - want).max()
+
+
+@pytest.mark.parametrize("kind,video", [(1, False), (2, False), (3, False), (1, True), (2, True)],
+                         ids=["in_context", "cross_attn", "adaln", "in_context_video", "cross_attn_video"])
+def test_conditioning_designs_match_torch_layers(kind, video):
+    """The in-context, cross-attention and adaLN designs against stock torch layers
+    (LayerNorm with affine, nn.MultiheadAttention for the cross-attention)."""
+    from torch_reference import reference_forward
+    cfg = (small_video() if video else small_image(cfg_scale=1.5)).with_(block_kind=kind)
+    W = S.make_weights(cfg)
+    inp = S.make_inputs(cfg)
+    got = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    want = reference_forward(cfg, S.weight_dict(cfg, W), inp["x"], inp["t"], inp["y"])
+    assert got.shape == want.shape == cfg.out_shape()
+    assert np.allclose(got, want, rtol=1e-9, atol=1e-10), np.abs(got - want).max()
+
+
+def test_cross_attention_closed_forms():
+    """Two equal keys weigh both values 1/2; queries identical across tokens give identical
+    outputs; a zero output projection makes the sublayer vanish."""
+    rng = np.random.default_rng(21)
+    d, heads = 8, 2
+    u = rng.standard_normal((1, 5, d))
+    ctx = rng.standard_normal((1, 2, d))
+    wq, bq = rng.standard_normal((d, d)), rng.standard_normal(d)
+    wkv, bkv = rng.standard_normal((2 * d, d)), rng.standard_normal(2 * d)
+    wo, bo = np.eye(d), np.zeros(d)
+    same = np.repeat(ctx[:, :1], 2, axis=1)
+    k0v = O.linear(same, wkv, bkv)[0, 0, d:]
+    out = O.cross_attention(u, same, wq, bq, wkv, bkv, wo, bo, heads)
+    assert np.allclose(out[0], np.broadcast_to(k0v, (5, d)), rtol=1e-12, atol=1e-12)
+    v = O.linear(ctx, wkv, bkv)[0, :, d:]
+    out = O.cross_attention(u, ctx, wq, bq, wkv, bkv, wo, bo, heads)
+    for hd in range(heads):   # each head's output is a convex mix of the two values
+        sl = slice(hd * 4, hd * 4 + 4)
+        lam = (out[0, :, sl] - v[1, sl]) / (v[0, sl] - v[1, sl])
+        assert np.allclose(lam, lam[:, :1], rtol=1e-9, atol=1e-9) and np.all((lam > 0) & (lam < 1))
+    assert np.array_equal(O.cross_attention(u, ctx, wq, bq, wkv, bkv, 0 * wo, bo, heads), np.zeros((1, 5, d)))
+
+
+def test_in_context_tokens_are_dropped_and_blocks_see_them():
+    """In-context: the residual stream carries T + 2 tokens, the first two being e_t and e_y
+    before any block; the output has the patch tokens only, and the condition reaches it."""
+    cfg = small_image(cfg_scale=1.0, block_kind=1)
+    W = S.weight_dict(cfg, S.make_weights(cfg))
+    inp = S.make_inputs(cfg)
+    h0 = O.forward(cfg, W, inp["x"], inp["t"], inp["y"], stop_after_block=0)
+    et, ey = O.condition_parts(cfg, W, inp["t"], inp["y"])
+    assert h0.shape == (cfg.batch, cfg.tokens + 2, cfg.hidden)
+    assert np.array_equal(h0[:, 0], et) and np.array_equal(h0[:, 1], ey)
+    out = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    other = O.forward(cfg, W, inp["x"], inp["t"], (inp["y"] + 1) % cfg.num_classes)
+    assert out.shape == cfg.out_shape() and not np.allclose(out, other)
+
+
+@pytest.mark.parametrize("plant", ["kv_swapped", "ln_gain_dropped", "ctx_from_c", "adaln_gate_kept"])
+def test_conditioning_cross_check_catches_planted_mistakes(plant, monkeypatch):
+    """Slips in the other conditioning designs (keys and values swapped in the cross-attention,
+    the learned LN gain dropped, the summed c used as both condition tokens, a gate applied in
+    the gateless adaLN block) make the torch-layer cross-check fail."""
+    from torch_reference import reference_forward
+    kind = {"kv_swapped": 2, "ln_gain_dropped": 1, "ctx_from_c": 2, "adaln_gate_kept": 3}[plant]
+    cfg = small_image(cfg_scale=1.5, block_kind=kind)
+    Wd = S.weight_dict(cfg, S.make_weights(cfg))
+    inp = S.make_inputs(cfg)
+    want = reference_forward(cfg, Wd, inp["x"], inp["t"], inp["y"])
+    if plant == "kv_swapped":
+        orig = O.cross_attention
+        d = cfg.hidden
+        monkeypatch.setattr(O, "cross_attention", lambda u, ctx, wq, bq, wkv, bkv, wo, bo, h: orig(
+            u, ctx, wq, bq, np.concatenate([wkv[d:], wkv[:d]]), np.concatenate([bkv[d:], bkv[:d]]), wo, bo, h))
+    elif plant == "ln_gain_dropped":
+        orig = O.layernorm_affine
+        monkeypatch.setattr(O, "layernorm_affine", lambda x, g, b, eps=1e-6: orig(x, np.ones_like(g), b, eps))
+    elif plant == "ctx_from_c":
+        orig = O.condition_parts
+        monkeypatch.setattr(O, "condition_parts", lambda c_, W_, t_, y_: (lambda a: (a[0] + a[1], a[0] + a[1]))(
+            orig(c_, W_, t_, y_)))
+    else:
+        orig = O.adaln_block
+
+        def gated(x, sc, W_, prefix, heads, coords=None):
+            g = O.silu(sc) * 0.5 + 0.25    # any gate other than 1
+            return x + g[:, None, :] * (orig(x, sc, W_, prefix, heads, coords) - x)
+        monkeypatch.setattr(O, "adaln_block", gated)
+    got = O.forward(cfg, Wd, inp["x"], inp["t"], inp["y"])
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    assert rel > 1e-7, rel
 
 
 _PLANTS = {

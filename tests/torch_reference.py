@@ -29,22 +29,44 @@ def _t(a):
 
 
 class RefBlock(nn.Module):
-    def __init__(self, d, heads, mlp, qk_norm):
+    """kind 0: adaLN-Zero (six modulation vectors incl. gates); 3: adaLN (four, no gates);
+    1: in-context and 2: cross-attention (learned LayerNorm affines, no modulation)."""
+
+    def __init__(self, d, heads, mlp, qk_norm, kind=0):
         super().__init__()
         self.heads = heads
         self.qk_norm = qk_norm
-        self.norm1 = nn.LayerNorm(d, elementwise_affine=False, eps=1e-6)
-        self.norm2 = nn.LayerNorm(d, elementwise_affine=False, eps=1e-6)
+        self.kind = kind
+        affine = kind in (1, 2)
+        self.norm1 = nn.LayerNorm(d, elementwise_affine=affine, eps=1e-6)
+        self.norm2 = nn.LayerNorm(d, elementwise_affine=affine, eps=1e-6)
         self.attn = nn.MultiheadAttention(d, heads, batch_first=True)
         self.mlp = nn.Sequential(nn.Linear(d, mlp), nn.GELU(approximate="tanh"), nn.Linear(mlp, d))
-        self.ada = nn.Sequential(nn.SiLU(), nn.Linear(d, 6 * d))
+        if kind in (0, 3):
+            self.ada = nn.Sequential(nn.SiLU(), nn.Linear(d, (6 if kind == 0 else 4) * d))
+        if kind == 2:
+            self.normx = nn.LayerNorm(d, eps=1e-6)
+            self.xattn = nn.MultiheadAttention(d, heads, batch_first=True)
         self.qg = None
         self.kg = None
 
     def load(self, W, p):
         with torch.no_grad():
-            self.ada[1].weight.copy_(_t(W[p + "ada.w"]))
-            self.ada[1].bias.copy_(_t(W[p + "ada.b"]))
+            if self.kind in (0, 3):
+                self.ada[1].weight.copy_(_t(W[p + "ada.w"]))
+                self.ada[1].bias.copy_(_t(W[p + "ada.b"]))
+            else:
+                self.norm1.weight.copy_(_t(W[p + "ln1.g"]))
+                self.norm1.bias.copy_(_t(W[p + "ln1.b"]))
+                self.norm2.weight.copy_(_t(W[p + "ln2.g"]))
+                self.norm2.bias.copy_(_t(W[p + "ln2.b"]))
+            if self.kind == 2:
+                self.normx.weight.copy_(_t(W[p + "xln.g"]))
+                self.normx.bias.copy_(_t(W[p + "xln.b"]))
+                self.xattn.in_proj_weight.copy_(torch.cat([_t(W[p + "xq.w"]), _t(W[p + "xkv.w"])]))
+                self.xattn.in_proj_bias.copy_(torch.cat([_t(W[p + "xq.b"]), _t(W[p + "xkv.b"])]))
+                self.xattn.out_proj.weight.copy_(_t(W[p + "xo.w"]))
+                self.xattn.out_proj.bias.copy_(_t(W[p + "xo.b"]))
             self.attn.in_proj_weight.copy_(_t(W[p + "qkv.w"]))
             self.attn.in_proj_bias.copy_(_t(W[p + "qkv.b"]))
             self.attn.out_proj.weight.copy_(_t(W[p + "proj.w"]))
@@ -80,12 +102,21 @@ class RefBlock(nn.Module):
         o = o.transpose(1, 2).reshape(r, t, d)
         return self.attn.out_proj(o)
 
-    def forward(self, x, c, coords=None):
-        sh1, sc1, g1, sh2, sc2, g2 = self.ada(c).chunk(6, dim=1)
-        h = self.norm1(x) * (1 + sc1[:, None]) + sh1[:, None]
-        x = x + g1[:, None] * self._attend(h, coords)
-        h = self.norm2(x) * (1 + sc2[:, None]) + sh2[:, None]
-        return x + g2[:, None] * self.mlp(h)
+    def forward(self, x, c, coords=None, ctx=None):
+        if self.kind == 0:
+            sh1, sc1, g1, sh2, sc2, g2 = self.ada(c).chunk(6, dim=1)
+            h = self.norm1(x) * (1 + sc1[:, None]) + sh1[:, None]
+            x = x + g1[:, None] * self._attend(h, coords)
+            h = self.norm2(x) * (1 + sc2[:, None]) + sh2[:, None]
+            return x + g2[:, None] * self.mlp(h)
+        if self.kind == 3:
+            sh1, sc1, sh2, sc2 = self.ada(c).chunk(4, dim=1)
+            x = x + self._attend(self.norm1(x) * (1 + sc1[:, None]) + sh1[:, None], coords)
+            return x + self.mlp(self.norm2(x) * (1 + sc2[:, None]) + sh2[:, None])
+        x = x + self._attend(self.norm1(x), coords)
+        if self.kind == 2:
+            x = x + self.xattn(self.normx(x), ctx, ctx, need_weights=False)[0]
+        return x + self.mlp(self.norm2(x))
 
 
 def conv_token_coords(cfg, extent):
@@ -132,27 +163,41 @@ def reference_forward(cfg, weights_by_name, x, t, y, cfg_scale=None, force_guida
         tmlp = nn.Sequential(nn.Linear(cfg.freq_dim, d), nn.SiLU(), nn.Linear(d, d)).to(T64)
         tmlp[0].weight.copy_(_t(W["t.w1"])); tmlp[0].bias.copy_(_t(W["t.b1"]))
         tmlp[2].weight.copy_(_t(W["t.w2"])); tmlp[2].bias.copy_(_t(W["t.b2"]))
-        c = tmlp(_t(O.timestep_embedding(t, cfg.freq_dim, cfg.t_scale)))
+        et = tmlp(_t(O.timestep_embedding(t, cfg.freq_dim, cfg.t_scale)))
         if cfg.cond_kind == 0:
             emb = nn.Embedding(cfg.num_classes + 1, d).to(T64)
             emb.weight.copy_(_t(W["y.table"]))
-            c = c + emb(torch.as_tensor(np.asarray(y, dtype=np.int64)))
+            ey = emb(torch.as_tensor(np.asarray(y, dtype=np.int64)))
         else:
-            c = c + _t(y)
+            ey = _t(y)
+        c = et + ey
+        kind = cfg.block_kind
 
         coords = conv_token_coords(cfg, x.shape[2:]) if cfg.pos_kind == 1 else None
+        ctx = None
+        if kind == 1:    # two condition tokens in front, without position
+            h = torch.cat([et[:, None], ey[:, None], h], dim=1)
+            if coords is not None:
+                coords = np.concatenate([np.zeros((2, 3), dtype=coords.dtype), coords])
+        elif kind == 2:  # a separate two-token condition sequence
+            ctx = torch.stack([et, ey], dim=1)
         for i in range(cfg.depth):
-            blk = RefBlock(d, cfg.heads, cfg.mlp_hidden, cfg.qk_norm).to(T64)
+            blk = RefBlock(d, cfg.heads, cfg.mlp_hidden, cfg.qk_norm, kind).to(T64)
             blk.load(W, f"blocks.{i}.")
-            h = blk(h, c, coords)
+            h = blk(h, c, coords, ctx)
 
-        fada = nn.Sequential(nn.SiLU(), nn.Linear(d, 2 * d)).to(T64)
-        fada[1].weight.copy_(_t(W["final.ada.w"])); fada[1].bias.copy_(_t(W["final.ada.b"]))
-        shift, scale = fada(c).chunk(2, dim=1)
-        norm = nn.LayerNorm(d, elementwise_affine=False, eps=1e-6)
         dec = nn.Linear(d, cfg.out_dim).to(T64)
         dec.weight.copy_(_t(W["dec.w"])); dec.bias.copy_(_t(W["dec.b"]))
-        z = dec(norm(h) * (1 + scale[:, None]) + shift[:, None])
+        if kind in (1, 2):
+            norm = nn.LayerNorm(d, eps=1e-6).to(T64)
+            norm.weight.copy_(_t(W["final.ln.g"])); norm.bias.copy_(_t(W["final.ln.b"]))
+            z = dec(norm(h[:, 2:] if kind == 1 else h))
+        else:
+            fada = nn.Sequential(nn.SiLU(), nn.Linear(d, 2 * d)).to(T64)
+            fada[1].weight.copy_(_t(W["final.ada.w"])); fada[1].bias.copy_(_t(W["final.ada.b"]))
+            shift, scale = fada(c).chunk(2, dim=1)
+            norm = nn.LayerNorm(d, elementwise_affine=False, eps=1e-6)
+            z = dec(norm(h) * (1 + scale[:, None]) + shift[:, None])
         gf, gh, gw = cfg.grid
         img = einops.rearrange(z, "n (f h w) (a p q c) -> n c (f a) (h p) (w q)", f=gf, h=gh, w=gw,
                                a=cfg.patch_t, p=cfg.patch_h, q=cfg.patch_w, c=cfg.out_channels)
