@@ -288,7 +288,64 @@ def self_attention(u, wqkv, bqkv, wo, bo, heads: int, qn=None, kn=None, coords=N
 
 def ffn(u, w1, b1, w2, b2):
     """Linear(d, 4d) -> tanh-GELU -> Linear(4d, d) ([DiT-wiki] "구현")."""
+    if _STATE.get("ffn_fp8"):
+        return ffn_e4m3(u, w1, b1, w2, b2)
     return linear(gelu_tanh(linear(u, w1, b1)), w2, b2)
+
+
+# --------------------------------------------------------------------------- #
+# FP8 (E4M3) feed-forward: a reading, not the pages' ([DiT-wiki] "U-Net과 비교" names
+# mixed precision among the techniques that carry over from language models; the pages fix
+# no format, so this is the quantised computation the FP8 path is held to)
+# --------------------------------------------------------------------------- #
+E4M3_MAX = 448.0
+
+
+def round_e4m3(x):
+    """Nearest FP8 E4M3 value (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits:
+    normal magnitudes 2^-6 .. 448 in binades of 8 steps, subnormal steps of 2^-9 below 2^-6),
+    ties to the even mantissa, magnitudes past 448 saturated to 448."""
+    x = np.asarray(x, dtype=F64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))   # binade of each magnitude
+    e = np.maximum(e, -6.0)                            # one step size below 2^-6
+    step = np.exp2(e - 3.0)                            # 8 steps per binade
+    q = np.minimum(np.round(a / step) * step, E4M3_MAX)   # np.round: ties to even
+    return np.sign(x) * q
+
+
+def quantize_rows(a, scale):
+    """s * Q(a / s) row by row: the value an E4M3 operand with per-row scale s stands for."""
+    s = np.asarray(scale, dtype=F64)[..., None]
+    return round_e4m3(np.asarray(a, dtype=F64) / s) * s
+
+
+def amax_scale(a):
+    """Per-row scale amax(|a|) / 448 (1 for an all-zero row), so that a row's largest
+    magnitude maps onto the largest E4M3 value."""
+    m = np.abs(np.asarray(a, dtype=F64)).max(axis=-1)
+    return np.where(m > 0, m / E4M3_MAX, 1.0)
+
+
+def linear_e4m3(x, w, b, x_scale=None):
+    """y = x W^T + b with both operands in E4M3: x with a per-row (token) scale (amax unless
+    given), W with a per-output-channel scale; products accumulated exactly."""
+    x = np.asarray(x, dtype=F64)
+    sx = amax_scale(x) if x_scale is None else np.asarray(x_scale, dtype=F64)
+    wq = quantize_rows(w, amax_scale(w))
+    return linear(quantize_rows(x, sx), wq, b)
+
+
+def ffn_e4m3(u, w1, b1, w2, b2):
+    """The feed-forward with both matmuls in E4M3.  The hidden activation g = GELU(z) gets a
+    per-token scale from a bound known before z is formed: |g| <= |z| <= ||u||_2 max_n ||W1_n||_2
+    + max |b1| (Cauchy-Schwarz), so g's scale is that bound / 448."""
+    u = np.asarray(u, dtype=F64)
+    z = linear_e4m3(u, w1, b1)
+    g = gelu_tanh(z)
+    w1 = np.asarray(w1, dtype=F64)
+    bound = np.linalg.norm(u, axis=-1) * np.linalg.norm(w1, axis=1).max() + np.abs(np.asarray(b1, F64)).max()
+    return linear_e4m3(g, w2, b2, x_scale=np.where(bound > 0, bound / E4M3_MAX, 1.0))
 
 
 def adaln_chunks(sc, w, b, n: int):
@@ -390,7 +447,18 @@ def embed(cfg, W, x5):
 
 def forward(cfg, weights: Sequence[np.ndarray] | Dict[str, np.ndarray], x, t, y,
             cfg_scale: Optional[float] = None, force_guidance: bool = False,
-            stop_after_block: Optional[int] = None, cfg_channels: Optional[int] = None):
+            stop_after_block: Optional[int] = None, cfg_channels: Optional[int] = None,
+            ffn_fp8: bool = False):
+    """ffn_fp8: every block's feed-forward in E4M3 (ffn_e4m3) instead of exact arithmetic."""
+    prev = _STATE.get("ffn_fp8", False)
+    _STATE["ffn_fp8"] = bool(ffn_fp8)
+    try:
+        return _forward(cfg, weights, x, t, y, cfg_scale, force_guidance, stop_after_block, cfg_channels)
+    finally:
+        _STATE["ffn_fp8"] = prev
+
+
+def _forward(cfg, weights, x, t, y, cfg_scale, force_guidance, stop_after_block, cfg_channels):
     """Denoiser output for a batch.
 
     Returns the guided prediction [B, C_out, (F,) H, W] (float64), or, when
