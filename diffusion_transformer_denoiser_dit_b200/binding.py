@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdit_b200
 DIT_OK, DIT_ERR_INVALID_ARG, DIT_ERR_UNSUPPORTED, DIT_ERR_OOM, DIT_ERR_CUDA = 0, 1, 2, 3, 4
 DIT_ERR_DEVICE_TIMEOUT, DIT_ERR_BAD_LABEL, DIT_ERR_NO_DEVICE = 5, 6, 7
 DIT_OPT_FORCE_GUIDANCE, DIT_OPT_USE_GRAPH, DIT_OPT_OVERLAP_LAUNCH, DIT_OPT_CFG_CHANNELS = 1, 2, 3, 4
+DIT_OPT_REPEAT_KIND = 5
 DIT_SAMPLER_DDIM, DIT_SAMPLER_EULER = 0, 1
 
 # every exported symbol declared in include/dit.h
@@ -26,6 +27,7 @@ EXPORTS = [
     "dit_status_string", "dit_destroy", "dit_set_option", "dit_debug_residual", "dit_debug_condition",
     "dit_debug_wait_probe", "dit_op_linear_bf16", "dit_forward_launch_count", "dit_profile_enable",
     "dit_profile_read", "dit_condition_static", "dit_op_linear_bf16_pair", "dit_sampler_step", "dit_sample",
+    "dit_op_attention_bf16", "dit_debug_attention_rescales", "dit_op_linear_e4m3",
 ]
 
 KERNEL_KINDS = ["cond", "adaln", "patch", "ln", "qkv", "attn", "proj", "fc1", "fc2", "decode", "sampler"]
@@ -36,7 +38,7 @@ class DitConfig(ctypes.Structure):
                 ("patch_t", c_int), ("patch_h", c_int), ("patch_w", c_int), ("hidden", c_int), ("depth", c_int),
                 ("heads", c_int), ("mlp_hidden", c_int), ("learn_sigma", c_int), ("pos_kind", c_int),
                 ("qk_norm", c_int), ("cond_kind", c_int), ("num_classes", c_int), ("freq_dim", c_int),
-                ("max_batch", c_int), ("t_scale", c_float)]
+                ("max_batch", c_int), ("t_scale", c_float), ("block_kind", c_int), ("ffn_fp8", c_int)]
 
 
 class DitError(RuntimeError):
@@ -79,6 +81,9 @@ def load() -> ctypes.CDLL:
         "dit_profile_read": (c_int, [P, POINTER(c_float), POINTER(c_int)]),
         "dit_condition_static": (c_int, [P, P, c_int, c_int, P, P, P, P, P, c_int, c_int, c_int, c_int, c_float,
                                          P, P, P]),
+        "dit_op_attention_bf16": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, P, P]),
+        "dit_debug_attention_rescales": (c_int, [P, POINTER(ctypes.c_longlong)]),
+        "dit_op_linear_e4m3": (c_int, [P, P, P, P, P, P, c_int, c_int, c_int, c_int, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -93,7 +98,8 @@ def make_config(cfg, max_batch: Optional[int] = None) -> DitConfig:
     mb = max_batch if max_batch is not None else cfg.batch
     return DitConfig(cfg.dtype, cfg.in_channels, cfg.frames, cfg.height, cfg.width, cfg.patch_t, cfg.patch_h,
                      cfg.patch_w, cfg.hidden, cfg.depth, cfg.heads, cfg.mlp_hidden, cfg.learn_sigma, cfg.pos_kind,
-                     cfg.qk_norm, cfg.cond_kind, cfg.num_classes, cfg.freq_dim, mb, float(cfg.t_scale))
+                     cfg.qk_norm, cfg.cond_kind, cfg.num_classes, cfg.freq_dim, mb, float(cfg.t_scale),
+                     int(getattr(cfg, "block_kind", 0)), int(getattr(cfg, "ffn_fp8", 0)))
 
 
 def status_string(code: int) -> str:
@@ -169,7 +175,8 @@ class DiT:
         import torch
         B = x.shape[0]
         R = self.rows(B, cfg_scale) if not getattr(self, "_force", False) else 2 * B
-        h = torch.empty((R, self.cfg.tokens, self.cfg.hidden), dtype=torch.float32, device=x.device)
+        h = torch.empty((R, getattr(self.cfg, "seq_tokens", self.cfg.tokens), self.cfg.hidden), dtype=torch.float32,
+                        device=x.device)
         rc = self.lib.dit_debug_residual(self.h, _ptr(x), _ptr(t), _ptr(y), B, float(cfg_scale), after_block, _ptr(h),
                                          _stream(stream))
         self._check(rc, "dit_debug_residual")
@@ -219,11 +226,19 @@ class DiT:
     def wait_probe(self, timeout_us: int, stream=None):
         self._check(self.lib.dit_debug_wait_probe(self.h, timeout_us, _stream(stream)), "dit_debug_wait_probe")
 
+    def attention_rescales(self) -> int:
+        """Attention reference-maximum moves (per warp of 32 query rows) since the last read."""
+        n = ctypes.c_longlong(0)
+        self._check(self.lib.dit_debug_attention_rescales(self.h, ctypes.byref(n)), "dit_debug_attention_rescales")
+        return int(n.value)
+
     def launch_count(self, B: int, cfg_scale: float) -> int:
         return self.lib.dit_forward_launch_count(self.h, B, float(cfg_scale))
 
-    def profile(self, enable: bool):
-        self._check(self.lib.dit_profile_enable(self.h, int(enable)), "dit_profile_enable")
+    def profile(self, enable: bool, kind: Optional[str] = None):
+        """Per-launch event timing on (every kind, or only `kind`, one of KERNEL_KINDS) or off."""
+        mode = 0 if not enable else (1 if kind is None else 2 + KERNEL_KINDS.index(kind))
+        self._check(self.lib.dit_profile_enable(self.h, mode), "dit_profile_enable")
 
     def profile_read(self):
         """{kind: (total_ms, launches)} of the launches recorded since the last read."""
@@ -257,4 +272,30 @@ def linear_bf16(x, w, b, block_n: int = 128, stream=None, pair: bool = False):
     rc = fn(_ptr(x), _ptr(w), _ptr(b), _ptr(y), M, N, K, block_n, _stream(stream))
     if rc != DIT_OK:
         raise DitError(rc, f"dit_op_linear_bf16: {status_string(rc)}")
+    return y
+
+
+def attention_bf16(q, k, v, o, R: int, H: int, T: int, dh: int, counters=None, stream=None):
+    """The bf16 tensor-core attention kernel on the forward's workspace layouts (see
+    dit_op_attention_bf16 in include/dit.h): q, k [R*H, Tpad, DP], v [R*H, DP, Tpad] and
+    o [R*T, H*dh], torch bf16 CUDA tensors; counters an int32 CUDA tensor of 2 or None."""
+    lib = load()
+    rc = lib.dit_op_attention_bf16(_ptr(q), _ptr(k), _ptr(v), _ptr(o), R, H, T, dh, _ptr(counters), _stream(stream))
+    if rc != DIT_OK:
+        raise DitError(rc, f"dit_op_attention_bf16: {status_string(rc)}")
+    return o
+
+
+def linear_e4m3(x8, w8, sx, sw, b, block_n: int = 128, stream=None):
+    """y = sx[m] sw[n] (x8 w8^T)[m, n] + b[n] on the FP8 tensor-core GEMM (x8, w8: uint8 CUDA
+    tensors of E4M3 bytes; sx, sw, b: float32 CUDA tensors, b may be None)."""
+    import torch
+    lib = load()
+    M, K = x8.shape
+    N = w8.shape[0]
+    y = torch.empty((M, N), dtype=torch.float32, device=x8.device)
+    rc = lib.dit_op_linear_e4m3(_ptr(x8), _ptr(w8), _ptr(sx), _ptr(sw), _ptr(b), _ptr(y), M, N, K, block_n,
+                                _stream(stream))
+    if rc != DIT_OK:
+        raise DitError(rc, f"dit_op_linear_e4m3: {status_string(rc)}")
     return y

@@ -17,9 +17,12 @@
 //             into registers (then S is released), online softmax in base 2 with lazy
 //             O rescaling (only when the running max grows by more than 2^8), P as bf16 in
 //             128B-swizzled shared memory, and at the end of an item O / l through a
-//             shared-memory staging tile and one TMA store (O is released as soon as it is
-//             in registers).
-// Every mbarrier wait is bounded.
+//             shared-memory staging tile (the start of the group's P buffer, free once the
+//             item's last P V is done) and one TMA store (O is released as soon as it is in
+//             registers).  Q is double-buffered, so the next item's Q arrives while the
+//             current item computes.
+// Every mbarrier wait is bounded.  status[0] receives DIT_ERR_DEVICE_TIMEOUT if one runs
+// out; status[1] counts the warps that moved their reference maximum (lazy rescales).
 //
 // Layouts: q, k [R*H, Tpad, DP] bf16 (rows of one head contiguous, head dim padded with
 // zeros to DP = 80 for dh = 72); v transposed [R*H, DP, Tpad]; padded key rows are zero
@@ -44,24 +47,27 @@ struct AttnCfg {
   static constexpr int O_ROW = DH * 2;                  // bytes of one output row
   static constexpr bool O_SW128 = O_ROW == 128;         // 128B-swizzled staging (else rows packed)
   static constexpr int O_TILE = (128 * O_ROW + 1023) / 1024 * 1024;
-  static constexpr int OFF_Q = 0;                       // Q of both query tiles of the item
-  static constexpr int OFF_K = OFF_Q + 2 * QK_TILE;     // two K stages
+  static constexpr int Q_BUF = 2 * QK_TILE;             // Q of both query tiles of an item
+  static constexpr int OFF_Q = 0;                       // two Q buffers: items alternate
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BUF;       // two K stages
   static constexpr int OFF_V = OFF_K + 2 * QK_TILE;     // two V^T stages
-  static constexpr int OFF_P = OFF_V + 2 * V_TILE;      // P of both query tiles
-  static constexpr int OFF_O = OFF_P + 2 * P_TILE;      // output staging of both query tiles
-  static constexpr int OFF_BAR = OFF_O + 2 * O_TILE;
+  static constexpr int OFF_P = OFF_V + 2 * V_TILE;      // P of both query tiles; each group's
+                                                        // output staging tile reuses the start of
+                                                        // its P buffer once the item's last P V is done
+  static constexpr int OFF_BAR = OFF_P + 2 * P_TILE;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr int TMEM_COLS = 512;                 // S0, S1, O0, O1 (128 columns each)
   static constexpr int THREADS = 384;                   // warpgroup 0: loads, MMA; 1, 2: softmax
   static constexpr int REG_CTRL = 96, REG_SOFTMAX = 200;
   static constexpr int REG_POOL = 128 * REG_CTRL + 256 * REG_SOFTMAX;  // must fit the launch allocation
-  static_assert(QK_TILE % 1024 == 0 && V_ATOM % 1024 == 0 && OFF_O % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(QK_TILE % 1024 == 0 && V_ATOM % 1024 == 0 && OFF_P % 1024 == 0, "1024-byte aligned tiles");
   static_assert(O_ROW % 16 == 0, "16-byte output rows");
+  static_assert(O_TILE <= P_TILE, "output staging inside the P buffer");
   static_assert(SMEM <= 232448, "shared memory");
 };
 
 enum {
-  B_QF = 0, B_QE,                    // Q of the item loaded / free (all its Q K^T done)
+  B_QF0 = 0, B_QF1, B_QE0, B_QE1,    // Q buffer b loaded / free (all Q K^T of its item done)
   B_KF0, B_KF1, B_KE0, B_KE1,        // K stages full / empty
   B_VF0, B_VF1, B_VE0, B_VE1,        // V^T stages full / empty
   B_S0, B_S1,                        // S_g ready
@@ -69,7 +75,7 @@ enum {
   B_P0, B_P1,                        // P_g written (count 128)
   B_O0, B_O1,                        // P_g V done
   B_OF0, B_OF1,                      // O_g read by the epilogue (count 128)
-  B_OS0, B_OS1,                      // output staging of group g free (previous store read it)
+  B_OS0, B_OS1,                      // group g's last output store has read its staging tile
   B_OW0, B_OW1,                      // output staging of group g written (count 128)
   B_GO,                              // group 0 wrote its first P: group 1 may start (completes once)
   B_COUNT
@@ -104,7 +110,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < B_COUNT; ++i) {
       const bool all = i == B_SF0 || i == B_SF1 || i == B_P0 || i == B_P1 || i == B_OF0 || i == B_OF1 ||
                        i == B_OW0 || i == B_OW1;
-      const bool both_issuers = i == B_QE || i == B_KE0 || i == B_KE1 || i == B_VE0 || i == B_VE1;
+      const bool both_issuers = i == B_QE0 || i == B_QE1 || i == B_KE0 || i == B_KE1 || i == B_VE0 || i == B_VE1;
       mbar_init(BAR(i), all ? 128 : both_issuers ? 2 : 1);
     }
     fence_barrier_init();
@@ -143,14 +149,16 @@ __global__ void __launch_bounds__(384, 1)
       for (int li = 0; li < my_items && ok; ++li) {
         int rh, qt0, ng;
         item_of(li, rh, qt0, ng);
-        // Q of item li once every Q K^T of item li-1 completed
-        if (li > 0 && !mbar_wait(BAR(B_QE), (li - 1) & 1, status)) break;
-        mbar_arrive_expect_tx(BAR(B_QF), ng * C::QK_TILE);
+        // Q of item li into buffer li & 1 once every Q K^T of item li-2 (its last user) completed;
+        // issued after the previous item's K / V tiles, so it arrives while that item computes
+        const int qbuf = li & 1, quse = li >> 1;
+        if (quse > 0 && !mbar_wait(BAR(B_QE0 + qbuf), (quse - 1) & 1, status)) break;
+        mbar_arrive_expect_tx(BAR(B_QF0 + qbuf), ng * C::QK_TILE);
         for (int g = 0; g < ng; ++g) {
           const int row0 = rh * a.Tpad + (qt0 + g) * 128;
-          const uint32_t dst = sbase + C::OFF_Q + g * C::QK_TILE;
-          tma_load_2d(dst, &tmQ, BAR(B_QF), 0, row0);
-          if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmQt, BAR(B_QF), 64, row0);
+          const uint32_t dst = sbase + C::OFF_Q + qbuf * C::Q_BUF + g * C::QK_TILE;
+          tma_load_2d(dst, &tmQ, BAR(B_QF0 + qbuf), 0, row0);
+          if (C::TAIL) tma_load_2d(dst + C::MAIN, &tmQt, BAR(B_QF0 + qbuf), 64, row0);
         }
         for (int j = 0; j < nk; ++j, ++n) {
           const uint32_t st = n & 1, free_parity = ((n >> 1) & 1) ^ 1u;
@@ -184,7 +192,7 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, C::DP);
       // No division in the per-tile path: items and key tiles are followed by cursors, and
       // every descriptor is a constant high word plus base + offset.
-      const uint32_t qb = sdesc_lo(sbase + C::OFF_Q) + g * (C::QK_TILE >> 4);
+      const uint32_t qb0 = sdesc_lo(sbase + C::OFF_Q) + g * (C::QK_TILE >> 4);
       const uint32_t k_lo = sdesc_lo(sbase + C::OFF_K), v_lo = sdesc_lo(sbase + C::OFF_V);
       const uint32_t pb = sdesc_lo(sbase + C::OFF_P) + g * (C::P_TILE >> 4);
       const uint32_t tS = tmem_base + g * 128, tO = tmem_base + 256 + g * 128;
@@ -210,8 +218,10 @@ __global__ void __launch_bounds__(384, 1)
       Cursor cq = first(), cp = first();
       // S_g = Q_g K_n^T (cursor cq is at tile n)
       auto issue_qk = [&](int n) -> bool {
-        if (cq.j == 0 && !mbar_wait(BAR(B_QF), cq.li & 1, status)) return false;
+        const int qbuf = cq.li & 1;
+        if (cq.j == 0 && !mbar_wait(BAR(B_QF0 + qbuf), (cq.li >> 1) & 1, status)) return false;
         if (!mbar_wait(BAR(B_KF0 + (n & 1)), (n >> 1) & 1, status)) return false;
+        const uint32_t qb = qb0 + qbuf * (C::Q_BUF >> 4);
         if (g < cq.ng) {
           // S_g may be overwritten once the softmax of group g has read its previous tile
           if (qk_cnt > 0 && !mbar_wait(BAR(B_SF0 + g), (qk_cnt - 1) & 1, status)) return false;
@@ -228,7 +238,7 @@ __global__ void __launch_bounds__(384, 1)
           ++qk_cnt;
         }
         mma_commit(BAR(B_KE0 + (n & 1)));
-        if (cq.j == nk - 1) mma_commit(BAR(B_QE));
+        if (cq.j == nk - 1) mma_commit(BAR(B_QE0 + qbuf));
         advance(cq);
         return true;
       };
@@ -279,7 +289,7 @@ __global__ void __launch_bounds__(384, 1)
     const float sc = 1.4426950408889634f * rsqrtf(static_cast<float>(DH));
     const uint32_t prow = sbase + C::OFF_P + g * C::P_TILE + r * 128;
     const uint32_t r7 = static_cast<uint32_t>(r & 7);
-    const uint32_t ostage = sbase + C::OFF_O + g * C::O_TILE;
+    const uint32_t ostage = sbase + C::OFF_P + g * C::P_TILE;  // the group's P buffer, between items
     const bool issuer = q == 0 && lane == 0;  // issues this group's output stores
     int cnt = 0;  // tiles of this group processed
     int ne = 0;   // items of this group finished
@@ -330,6 +340,7 @@ __global__ void __launch_bounds__(384, 1)
           rescale = true;
           alpha = ex2_approx(m_ref - m_new);
           m_ref = m_new;
+          if (lane == 0 && status != nullptr) atomicAdd(status + 1, 1);  // diagnostic event count
         }
         // P = 2^(s*sc - m_ref) as packed bf16 in registers (paired f32 scaling and row sums)
         uint32_t pk[64];
@@ -343,9 +354,12 @@ __global__ void __launch_bounds__(384, 1)
           rs2[i & 1] = f2_add(rs2[i & 1], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
-        // the previous P V must be complete before O is rescaled and the P buffer rewritten
+        // the previous P V must be complete before O is rescaled and the P buffer rewritten;
+        // at an item's first key tile the P buffer also held the previous item's output
+        // staging tile, which its TMA store must have finished reading
         if (cnt > 0) {
-          const bool okw = mbar_wait(BAR(B_O0 + g), (cnt - 1) & 1, status);
+          bool okw = mbar_wait(BAR(B_O0 + g), (cnt - 1) & 1, status);
+          if (j == 0 && ne > 0) okw = okw && mbar_wait(BAR(B_OS0 + g), (ne - 1) & 1, status);
           __syncwarp();
           if (__any_sync(0xffffffffu, !okw)) {
             ok = false;
@@ -398,16 +412,7 @@ __global__ void __launch_bounds__(384, 1)
       tmem_ld_wait<C::DP>(o);
       tc_fence_before();
       mbar_arrive(BAR(B_OF0 + g));  // O_g is in registers: the next item may overwrite it
-      if (issuer) {
-        bulk_wait_read_all();  // the previous store has finished reading the staging tile
-        mbar_arrive(BAR(B_OS0 + g));
-      }
-      const bool okf = mbar_wait(BAR(B_OS0 + g), ne & 1, status);
-      __syncwarp();
-      if (__any_sync(0xffffffffu, !okf)) {
-        ok = false;
-        break;
-      }
+      // the last P V has read the P buffer: it becomes this item's output staging tile
       const float inv = 1.0f / l;
       const uint32_t orow = ostage + r * C::O_ROW;
 #pragma unroll
@@ -428,6 +433,8 @@ __global__ void __launch_bounds__(384, 1)
           const int row = rh / a.H, head = rh - row * a.H;
           tma_store_3d(&tmO, ostage, head * DH, (qt0 + g) * 128, row);  // rows past T are clipped
           bulk_commit_group();
+          bulk_wait_read_all();         // the staging tile has been read: P may be written again
+          mbar_arrive(BAR(B_OS0 + g));
         }
       }
       ++ne;
@@ -462,8 +469,11 @@ bool make_attention_maps(AttnMaps* m, const void* q, const void* k, const void* 
 template <int DH>
 static cudaError_t launch_dh(const AttnArgs& a, const AttnMaps& mp, int* status, cudaStream_t st) {
   using C = AttnCfg<DH>;
-  static int num_sms = 0;
-  if (num_sms == 0) {
+  // one-time set-up per device: the shared-memory attribute is a per-device setting
+  static int sms_of[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (sms_of[dev] == 0) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     // the register split (setmaxnreg) must fit in the launch allocation, or it would wait forever
@@ -471,10 +481,12 @@ static cudaError_t launch_dh(const AttnArgs& a, const AttnMaps& mp, int* status,
     e = cudaFuncGetAttributes(&fa, attn_tc_kernel<DH>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * C::THREADS < C::REG_POOL) return cudaErrorInvalidConfiguration;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       return cudaErrorInvalidDevice;
+    sms_of[dev] = n;
   }
+  const int num_sms = sms_of[dev];
   const int nq = a.Tpad / 128;
   const int items = a.R * a.H * ((nq + 1) / 2);
   const int grid = items < num_sms ? items : num_sms;

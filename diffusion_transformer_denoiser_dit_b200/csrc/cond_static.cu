@@ -25,22 +25,44 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-float* g_scratch_dev[kMaxDevices] = {};  // device address of g_cond_scratch, per device
+// Device address of g_cond_scratch, per device, and the context it was resolved in: a
+// device reset tears the primary context down and a new one may place the array
+// elsewhere, so the address is looked up again whenever the current context changes.
+float* g_scratch_dev[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
+
+typedef CUresult (*PFN_ctxGetCurrent_t)(CUcontext*);
+
+CUcontext current_context() {
+  static PFN_ctxGetCurrent_t fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_ctxGetCurrent_t>(p);
+  }
+  CUcontext c = nullptr;
+  return fn(&c) == CUDA_SUCCESS ? c : nullptr;
+}
 
 // Resolves the device address of the scratch array on the current device (once per
-// device).  Host code must not use the array's name as a pointer: on the host it is
-// only a stand-in symbol.
+// device and context).  Host code must not use the array's name as a pointer: on the
+// host it is only a stand-in symbol.
 cudaError_t scratch_address(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_dev[dev] == nullptr) {
+  const CUcontext ctx = current_context();
+  if (g_scratch_dev[dev] == nullptr || ctx == nullptr || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_cond_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_dev[dev] = static_cast<float*>(p);
+    g_scratch_ctx[dev] = current_context();
   }
   *out = g_scratch_dev[dev];
   return cudaSuccess;

@@ -18,13 +18,31 @@ struct BlockW {
   void *qkv_w = nullptr, *proj_w = nullptr, *fc1_w = nullptr, *fc2_w = nullptr;  // bf16 or f32
   float *qkv_b = nullptr, *proj_b = nullptr, *fc1_b = nullptr, *fc2_b = nullptr;
   float *qn = nullptr, *kn = nullptr;
-  CUtensorMap tm_qkv, tm_fc1;          // weights as the B operand (box = tile width rows)
-  CUtensorMap ta_qkv, ta_proj, ta_fc2;  // weights as the A operand of the swapped GEMMs (box 128 rows)
+  // in-context / cross-attention designs: learned LayerNorm affines, stored as (gain - 1, bias)
+  // so that the LN + modulate kernel applies them as a row-independent (scale, shift)
+  float *ln1_s = nullptr, *ln1_b = nullptr, *ln2_s = nullptr, *ln2_b = nullptr, *xln_s = nullptr, *xln_b = nullptr;
+  // cross-attention: query and output projections (the key / value projections of all blocks
+  // are stacked in the handle for one GEMM at the start of the forward)
+  void *xq_w = nullptr, *xo_w = nullptr;
+  float *xq_b = nullptr, *xo_b = nullptr;
+  // FP8 feed-forward: E4M3 weights with per-output-channel scales, and the constants of the
+  // hidden activation's scale bound (max_n ||fc1.w_n||_2, max |fc1.b|)
+  uint8_t *fc1_w8 = nullptr, *fc2_w8 = nullptr;
+  float *fc1_s = nullptr, *fc2_s = nullptr;
+  float g_w = 0.f, g_b = 0.f;
+  CUtensorMap tm_qkv, tm_fc1, tm_xq, tm_fc1_8;  // weights as the B operand (box = tile width rows)
+  CUtensorMap ta_qkv, ta_proj, ta_fc2, ta_xo, ta_fc2_8;  // weights as the A operand of the swapped GEMMs (box 128 rows)
 };
 
 struct Geometry {
   int gf, gh, gw, T, Kp, P, Cout, dh, DP, Tpad, Rmax, RPalloc, Mmax, nmod;
+  int kind;      // DIT_BLOCK_*
+  int Tc, Ts;    // condition tokens in front of the patch tokens; tokens per row inside the blocks
+  int mpb;       // modulation vectors per block (6 adaLN-Zero, 4 adaLN, 0 otherwise)
+  int nkv;       // cross-attention: key / value features of all blocks (depth * 2d)
+  int CTXalloc;  // rows of the condition-sequence buffer (2 Rmax rounded up for 256-row boxes)
   int bn_qkv, bn_fc1;
+  int bn_dec, dec_rows;  // decoder GEMM tile width; decoder weight rows (P padded to whole tiles)
   int headwise;  // 1: QK-RMSNorm / RoPE need whole heads -> two-head tiles for the QKV projection
 };
 
@@ -49,6 +67,8 @@ bool validate(const dit_config* c, std::string& err) {
   if (c->freq_dim <= 0 || (c->freq_dim & 1)) return bad("freq_dim must be positive and even");
   if (c->max_batch <= 0) return bad("max_batch must be positive");
   if (!isfinite(c->t_scale)) return bad("t_scale must be finite");
+  if (c->block_kind < DIT_BLOCK_ADALN_ZERO || c->block_kind > DIT_BLOCK_ADALN) return bad("unknown block_kind");
+  if (c->ffn_fp8 != 0 && c->ffn_fp8 != 1) return bad("ffn_fp8 must be 0 or 1");
   return true;
 }
 
@@ -77,6 +97,10 @@ bool supported(const dit_config* c, std::string& err) {
       return false;
     }
   }
+  if (c->ffn_fp8 && c->dtype != DIT_DTYPE_BF16) {
+    err = "the FP8 feed-forward runs on the bf16 tensor-core path only";
+    return false;
+  }
   const long long kp = 1LL * c->in_channels * c->patch_t * c->patch_h * c->patch_w;
   if (kp * 16 * 4 > 200 * 1024) {
     err = "patch vector too long";
@@ -91,16 +115,22 @@ Geometry geometry(const dit_config* c) {
   g.gh = c->height / c->patch_h;
   g.gw = c->width / c->patch_w;
   g.T = g.gf * g.gh * g.gw;
+  g.kind = c->block_kind;
+  g.Tc = g.kind == DIT_BLOCK_IN_CONTEXT ? 2 : 0;
+  g.Ts = g.T + g.Tc;
+  g.mpb = g.kind == DIT_BLOCK_ADALN_ZERO ? 6 : g.kind == DIT_BLOCK_ADALN ? 4 : 0;
   g.Kp = c->in_channels * c->patch_t * c->patch_h * c->patch_w;
   g.Cout = c->learn_sigma ? 2 * c->in_channels : c->in_channels;
   g.P = c->patch_t * c->patch_h * c->patch_w * g.Cout;
   g.dh = c->hidden / c->heads;
   g.DP = (g.dh + 15) / 16 * 16;
-  g.Tpad = (g.T + 127) / 128 * 128;
+  g.Tpad = (g.Ts + 127) / 128 * 128;
   g.Rmax = c->cond_kind == DIT_COND_CLASS ? 2 * c->max_batch : c->max_batch;
   g.RPalloc = (g.Rmax + 255) / 256 * 256;
-  g.Mmax = g.Rmax * g.T;
-  g.nmod = (6 * c->depth + 2) * c->hidden;
+  g.Mmax = g.Rmax * g.Ts;
+  g.nmod = g.mpb > 0 ? (g.mpb * c->depth + 2) * c->hidden : 0;
+  g.nkv = g.kind == DIT_BLOCK_CROSS_ATTN ? 2 * c->depth * c->hidden : 0;
+  g.CTXalloc = (2 * g.Rmax + 255) / 256 * 256;
   // GEMM tiles.  The MMA reads its A and B tiles from shared memory every instruction,
   // so wide (N = 256) tiles keep the tensor cores fed.  proj, fc2 and (without QK norm
   // / RoPE) QKV run with swapped operands — A = weights (features), B = tokens — so the
@@ -108,11 +138,14 @@ Geometry geometry(const dit_config* c) {
   g.headwise = (c->qk_norm || c->pos_kind == DIT_POS_ROPE3D) ? 1 : 0;
   g.bn_qkv = g.headwise ? 2 * g.dh : 256;
   g.bn_fc1 = 256;
+  g.bn_dec = g.P <= 16 ? 16 : g.P <= 32 ? 32 : g.P <= 64 ? 64 : g.P <= 128 ? 128 : 256;
+  g.dec_rows = (g.P + g.bn_dec - 1) / g.bn_dec * g.bn_dec;
   return g;
 }
 
 int weight_count(const dit_config* c) {
-  const int per_block = 10 + (c->qk_norm ? 2 : 0);
+  const int k = c->block_kind;
+  const int per_block = (k == DIT_BLOCK_IN_CONTEXT ? 12 : k == DIT_BLOCK_CROSS_ATTN ? 20 : 10) + (c->qk_norm ? 2 : 0);
   return 6 + (c->cond_kind == DIT_COND_CLASS ? 1 : 0) + c->depth * per_block + 4;
 }
 
@@ -134,36 +167,47 @@ struct dit_handle {
   std::string err;
   std::vector<void*> allocs;
   // weights
-  float *pe_w = nullptr, *pe_b = nullptr, *t_w1 = nullptr, *t_b1 = nullptr, *t_w2 = nullptr, *t_b2 = nullptr;
+  float *pe_w = nullptr, *pe_wt = nullptr, *pe_b = nullptr, *t_w1 = nullptr, *t_b1 = nullptr, *t_w2 = nullptr,
+        *t_b2 = nullptr;
   float* table = nullptr;
   void* ada_w = nullptr;
   float* ada_b = nullptr;
   std::vector<BlockW> blk;
-  float *dec_w = nullptr, *dec_b = nullptr;
+  void* dec_w = nullptr;  // [dec_rows, d] bf16 or f32, rows >= P zero
+  float* dec_b = nullptr;
+  float *fln_s = nullptr, *fln_b = nullptr;  // final LayerNorm affine (gain - 1, bias) of the unmodulated designs
+  float* ones = nullptr;                     // [d] of 1.0: the gate of the ungated designs
+  uint8_t *u8 = nullptr, *g8 = nullptr;      // FP8 feed-forward operands [Mmax, d], [Mmax, mlp]
+  float *su = nullptr, *sg = nullptr;        // their per-token scales [Mmax]
+  void* xkv_w = nullptr;                     // cross-attention key / value weights of all blocks [nkv, d]
+  float *xkv_b = nullptr, *xkv = nullptr;    // their biases [nkv]; keys / values [2 Rmax, nkv] (f32)
+  void* ctx = nullptr;                       // condition sequence [CTXalloc, d]: rows 2r, 2r+1 = e_t, e_y
   float *pos = nullptr, *rope = nullptr;
   // workspace
-  float *E = nullptr, *hid = nullptr, *c = nullptr, *mod = nullptr, *h = nullptr;
+  float *E = nullptr, *hid = nullptr, *c = nullptr, *mod = nullptr, *h = nullptr, *z = nullptr;
   void *sc = nullptr, *u = nullptr, *q = nullptr, *k = nullptr, *v = nullptr, *o = nullptr, *gbuf = nullptr;
   int *status = nullptr, *probe_flag = nullptr;
   float *x_stage = nullptr, *t_stage = nullptr, *out_stage = nullptr;
   void* y_stage = nullptr;
-  CUtensorMap tm_ada, tm_sc[5], tm_u, tm_o, tm_g;
+  CUtensorMap tm_ada, tm_sc[5], tm_u, tm_o, tm_g, tm_dec, tm_xkv, tm_ctx[5];
+  CUtensorMap tm_u8, tb_g8;  // FP8: LN output as fc1's A operand; fc1 output as fc2's B operand
   CUtensorMap tm_g_out, tm_h_red;  // TMA-store targets: GELU output, residual stream
   CUtensorMap tb_u, tb_o, tb_g;     // activations as the B operand of the swapped GEMMs (box 256 rows)
   AttnMaps attn_maps;
   int force_guidance = 0;
   int cfg_channels = 0;  // DIT_OPT_CFG_CHANNELS: guided output channels (0: all)
+  int repeat_kind = -1;  // DIT_OPT_REPEAT_KIND: kernel kind launched twice per use (-1: none)
   // CUDA-graph replay of the whole forward (DIT_OPT_USE_GRAPH): one cached executable graph,
   // valid for the exact pointers and parameters it was captured with
   struct GraphKey {
     const void *x, *t, *y;
     float* out;
-    int B, R, depth, gch;
+    int B, R, depth, gch, rep;
     bool guided, pdl;
     float s;
     bool operator==(const GraphKey& o) const {
       return x == o.x && t == o.t && y == o.y && out == o.out && B == o.B && R == o.R && depth == o.depth &&
-             gch == o.gch && guided == o.guided && pdl == o.pdl && s == o.s;
+             gch == o.gch && rep == o.rep && guided == o.guided && pdl == o.pdl && s == o.s;
     }
   };
   cudaStream_t cap_stream = nullptr;
@@ -178,21 +222,22 @@ struct dit_handle {
     float* x = nullptr;
     const void* y = nullptr;
     const float* t_sched = nullptr;
-    int B = 0, R = 0, kind = 0, steps = 0, gch = 0;
+    int B = 0, R = 0, kind = 0, steps = 0, gch = 0, rep = -1;
     bool guided = false, pdl = false;
     float s = 0.f;
     std::vector<float> levels;
     bool operator==(const SampleKey& o) const {
       return x == o.x && y == o.y && t_sched == o.t_sched && B == o.B && R == o.R && kind == o.kind && gch == o.gch &&
-             steps == o.steps && guided == o.guided && pdl == o.pdl && s == o.s && levels == o.levels;
+             rep == o.rep && steps == o.steps && guided == o.guided && pdl == o.pdl && s == o.s && levels == o.levels;
     }
   };
   cudaGraphExec_t sexec = nullptr;
   SampleKey skey, sseen;
   bool has_sseen = false;
   int use_graph = 0;
-  // per-launch event timing (dit_profile_enable)
+  // per-launch event timing (dit_profile_enable): every kind, or only prof_kind
   bool prof = false;
+  int prof_kind = -1;
   std::vector<cudaEvent_t> ev_pool;
   std::vector<std::pair<int, int>> prof_recs;  // (kind, index of the start event in ev_pool)
 
@@ -308,6 +353,7 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
 
   // ---------------- weights
   ALLOC(H->pe_w, float, (size_t)d * g.Kp * 4);
+  ALLOC(H->pe_wt, float, (size_t)d * g.Kp * 4);
   ALLOC(H->pe_b, float, (size_t)d * 4);
   ALLOC(H->t_w1, float, (size_t)d * cfg->freq_dim * 4);
   ALLOC(H->t_b1, float, (size_t)d * 4);
@@ -316,26 +362,57 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
   if (cfg->cond_kind == DIT_COND_CLASS) ALLOC(H->table, float, (size_t)(cfg->num_classes + 1) * d * 4);
   ALLOC(H->ada_w, void, (size_t)g.nmod * d * es);
   ALLOC(H->ada_b, float, (size_t)g.nmod * 4);
+  const bool modulated = g.mpb > 0, cross = g.kind == DIT_BLOCK_CROSS_ATTN;
+  ALLOC(H->ones, float, (size_t)d * 4);
+  if (!modulated) {
+    ALLOC(H->fln_s, float, (size_t)d * 4);
+    ALLOC(H->fln_b, float, (size_t)d * 4);
+  }
+  if (cross) {
+    ALLOC(H->xkv_w, void, (size_t)g.nkv * d * es);
+    ALLOC(H->xkv_b, float, (size_t)g.nkv * 4);
+  }
   H->blk.resize(N);
   for (int i = 0; i < N; ++i) {
     BlockW& b = H->blk[i];
+    if (!modulated) {
+      ALLOC(b.ln1_s, float, (size_t)d * 4);
+      ALLOC(b.ln1_b, float, (size_t)d * 4);
+      ALLOC(b.ln2_s, float, (size_t)d * 4);
+      ALLOC(b.ln2_b, float, (size_t)d * 4);
+    }
+    if (cross) {
+      ALLOC(b.xln_s, float, (size_t)d * 4);
+      ALLOC(b.xln_b, float, (size_t)d * 4);
+      ALLOC(b.xq_w, void, (size_t)d * d * es);
+      ALLOC(b.xq_b, float, (size_t)d * 4);
+      ALLOC(b.xo_w, void, (size_t)d * d * es);
+      ALLOC(b.xo_b, float, (size_t)d * 4);
+    }
     ALLOC(b.qkv_w, void, (size_t)3 * d * d * es);
     ALLOC(b.qkv_b, float, (size_t)3 * d * 4);
     ALLOC(b.proj_w, void, (size_t)d * d * es);
     ALLOC(b.proj_b, float, (size_t)d * 4);
-    ALLOC(b.fc1_w, void, (size_t)mlp * d * es);
+    if (cfg->ffn_fp8) {
+      ALLOC(b.fc1_w8, uint8_t, (size_t)mlp * d);
+      ALLOC(b.fc1_s, float, (size_t)mlp * 4);
+      ALLOC(b.fc2_w8, uint8_t, (size_t)d * mlp);
+      ALLOC(b.fc2_s, float, (size_t)d * 4);
+    } else {
+      ALLOC(b.fc1_w, void, (size_t)mlp * d * es);
+      ALLOC(b.fc2_w, void, (size_t)d * mlp * es);
+    }
     ALLOC(b.fc1_b, float, (size_t)mlp * 4);
-    ALLOC(b.fc2_w, void, (size_t)d * mlp * es);
     ALLOC(b.fc2_b, float, (size_t)d * 4);
     if (cfg->qk_norm) {
       ALLOC(b.qn, float, (size_t)g.dh * 4);
       ALLOC(b.kn, float, (size_t)g.dh * 4);
     }
   }
-  ALLOC(H->dec_w, float, (size_t)g.P * d * 4);
+  ALLOC(H->dec_w, void, (size_t)g.dec_rows * d * es);
   ALLOC(H->dec_b, float, (size_t)g.P * 4);
   if (cfg->pos_kind == DIT_POS_SINCOS2D) ALLOC(H->pos, float, (size_t)g.T * d * 4);
-  else ALLOC(H->rope, float, (size_t)g.T * g.dh * 4);
+  else ALLOC(H->rope, float, (size_t)g.Ts * g.dh * 4);
 
   // ---------------- workspace
   const size_t R = g.Rmax, M = g.Mmax;
@@ -344,6 +421,10 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
   ALLOC(H->c, float, R * d * 4);
   ALLOC(H->sc, void, (size_t)g.RPalloc * d * es);
   ALLOC(H->mod, float, R * g.nmod * 4);
+  if (cross) {
+    ALLOC(H->ctx, void, (size_t)g.CTXalloc * d * es);
+    ALLOC(H->xkv, float, 2 * R * g.nkv * 4);
+  }
   ALLOC(H->h, float, M * d * 4);
   ALLOC(H->u, void, M * d * es);
   if (H->bf16) {
@@ -352,13 +433,22 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
     ALLOC(H->k, void, qk);
     ALLOC(H->v, void, qk);
   } else {
-    const size_t qk = R * cfg->heads * (size_t)g.T * g.dh * 4;
+    const size_t qk = R * cfg->heads * (size_t)g.Ts * g.dh * 4;
     ALLOC(H->q, void, qk);
     ALLOC(H->k, void, qk);
     ALLOC(H->v, void, qk);
   }
   ALLOC(H->o, void, M * d * es);
-  ALLOC(H->gbuf, void, M * mlp * es);
+  ALLOC(H->z, float, M * g.P * 4);
+  if (cfg->ffn_fp8) {
+    ALLOC(H->u8, uint8_t, M * d);
+    ALLOC(H->g8, uint8_t, M * mlp);
+    ALLOC(H->su, float, M * 4);
+    ALLOC(H->sg, float, M * 4);
+    ALLOC(H->gbuf, void, 16);
+  } else {
+    ALLOC(H->gbuf, void, M * mlp * es);
+  }
   ALLOC(H->status, int, 64);
   ALLOC(H->probe_flag, int, 64);
   const size_t xin = (size_t)cfg->max_batch * cfg->in_channels * cfg->frames * cfg->height * cfg->width;
@@ -371,11 +461,15 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
   // ---------------- upload
   size_t maxn = 0;
   {
-    const size_t cand[] = {(size_t)3 * d * d, (size_t)mlp * d, (size_t)6 * d * d};
+    const size_t cand[] = {(size_t)3 * d * d, (size_t)mlp * d, (size_t)6 * d * d, (size_t)g.dec_rows * d};
     for (size_t v : cand) maxn = v > maxn ? v : maxn;
   }
   float* staging = nullptr;
   if (H->bf16) ALLOC(staging, float, maxn * 4);
+  if (cfg->ffn_fp8 && staging == nullptr) {
+    dit_destroy(H);
+    return DIT_ERR_INVALID_ARG;
+  }
   int wi = 0;
   dit_status st = DIT_OK;
 #define UP(dst, n, tobf)                                                 \
@@ -386,6 +480,16 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
       return st;                                                         \
     }                                                                    \
   } while (0)
+  {  // the patch weights also transposed, [Kp, d], for the embedding kernel's coalesced reads
+    std::vector<float> wt((size_t)d * g.Kp);
+    const float* w = weights[wi];
+    for (int j = 0; j < d; ++j)
+      for (int k = 0; k < g.Kp; ++k) wt[(size_t)k * d + j] = w[(size_t)j * g.Kp + k];
+    if (cudaMemcpy(H->pe_wt, wt.data(), wt.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+      dit_destroy(H);
+      return DIT_ERR_CUDA;
+    }
+  }
   UP(H->pe_w, (size_t)d * g.Kp, false);
   UP(H->pe_b, (size_t)d, false);
   UP(H->t_w1, (size_t)d * cfg->freq_dim, false);
@@ -393,10 +497,27 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
   UP(H->t_w2, (size_t)d * d, false);
   UP(H->t_b2, (size_t)d, false);
   if (cfg->cond_kind == DIT_COND_CLASS) UP(H->table, (size_t)(cfg->num_classes + 1) * d, false);
+  // a learned LayerNorm gain is stored as gain - 1 (the LN kernel applies (1 + scale))
+#define UP_GAIN(dst)                                                        \
+  do {                                                                      \
+    std::vector<float> gm1(weights[wi], weights[wi] + d);                   \
+    for (float& v : gm1) v -= 1.0f;                                         \
+    ++wi;                                                                   \
+    if (cudaMemcpy((dst), gm1.data(), (size_t)d * 4, cudaMemcpyHostToDevice) != cudaSuccess) { \
+      dit_destroy(H);                                                       \
+      return DIT_ERR_CUDA;                                                  \
+    }                                                                       \
+  } while (0)
+  const int mpb = g.mpb;
   for (int i = 0; i < N; ++i) {
     BlockW& b = H->blk[i];
-    UP(static_cast<char*>(H->ada_w) + (size_t)i * 6 * d * d * es, (size_t)6 * d * d, H->bf16);
-    UP(H->ada_b + (size_t)i * 6 * d, (size_t)6 * d, false);
+    if (modulated) {
+      UP(static_cast<char*>(H->ada_w) + (size_t)i * mpb * d * d * es, (size_t)mpb * d * d, H->bf16);
+      UP(H->ada_b + (size_t)i * mpb * d, (size_t)mpb * d, false);
+    } else {
+      UP_GAIN(b.ln1_s);
+      UP(b.ln1_b, (size_t)d, false);
+    }
     UP(b.qkv_w, (size_t)3 * d * d, H->bf16);
     UP(b.qkv_b, (size_t)3 * d, false);
     if (cfg->qk_norm) {
@@ -405,19 +526,77 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
     }
     UP(b.proj_w, (size_t)d * d, H->bf16);
     UP(b.proj_b, (size_t)d, false);
-    UP(b.fc1_w, (size_t)mlp * d, H->bf16);
-    UP(b.fc1_b, (size_t)mlp, false);
-    UP(b.fc2_w, (size_t)d * mlp, H->bf16);
-    UP(b.fc2_b, (size_t)d, false);
+    if (cross) {
+      UP_GAIN(b.xln_s);
+      UP(b.xln_b, (size_t)d, false);
+      UP(b.xq_w, (size_t)d * d, H->bf16);
+      UP(b.xq_b, (size_t)d, false);
+      UP(static_cast<char*>(H->xkv_w) + (size_t)i * 2 * d * d * es, (size_t)2 * d * d, H->bf16);
+      UP(H->xkv_b + (size_t)i * 2 * d, (size_t)2 * d, false);
+      UP(b.xo_w, (size_t)d * d, H->bf16);
+      UP(b.xo_b, (size_t)d, false);
+    }
+    if (!modulated) {
+      UP_GAIN(b.ln2_s);
+      UP(b.ln2_b, (size_t)d, false);
+    }
+    if (cfg->ffn_fp8) {
+      // E4M3 weights, quantised per output channel on the device from the float32 values;
+      // the hidden scale bound's constants from the host copy
+      const float* w1 = weights[wi];
+      double wmax = 0.0;
+      for (int n = 0; n < mlp; ++n) {
+        double ss = 0.0;
+        for (int k = 0; k < d; ++k) ss += (double)w1[(size_t)n * d + k] * w1[(size_t)n * d + k];
+        wmax = ss > wmax ? ss : wmax;
+      }
+      b.g_w = (float)std::sqrt(wmax);
+      if (cudaMemcpy(staging, weights[wi++], (size_t)mlp * d * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+          launch_quantize_rows_e4m3(staging, b.fc1_w8, b.fc1_s, mlp, d, 0) != cudaSuccess ||
+          cudaDeviceSynchronize() != cudaSuccess) {
+        dit_destroy(H);
+        return DIT_ERR_CUDA;
+      }
+      const float* b1 = weights[wi];
+      float bmax = 0.f;
+      for (int n = 0; n < mlp; ++n) bmax = fabsf(b1[n]) > bmax ? fabsf(b1[n]) : bmax;
+      b.g_b = bmax;
+      UP(b.fc1_b, (size_t)mlp, false);
+      if (cudaMemcpy(staging, weights[wi++], (size_t)d * mlp * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+          launch_quantize_rows_e4m3(staging, b.fc2_w8, b.fc2_s, d, mlp, 0) != cudaSuccess ||
+          cudaDeviceSynchronize() != cudaSuccess) {
+        dit_destroy(H);
+        return DIT_ERR_CUDA;
+      }
+      UP(b.fc2_b, (size_t)d, false);
+    } else {
+      UP(b.fc1_w, (size_t)mlp * d, H->bf16);
+      UP(b.fc1_b, (size_t)mlp, false);
+      UP(b.fc2_w, (size_t)d * mlp, H->bf16);
+      UP(b.fc2_b, (size_t)d, false);
+    }
   }
-  UP(static_cast<char*>(H->ada_w) + (size_t)N * 6 * d * d * es, (size_t)2 * d * d, H->bf16);
-  UP(H->ada_b + (size_t)N * 6 * d, (size_t)2 * d, false);
-  UP(H->dec_w, (size_t)g.P * d, false);
+  if (modulated) {
+    UP(static_cast<char*>(H->ada_w) + (size_t)N * mpb * d * d * es, (size_t)2 * d * d, H->bf16);
+    UP(H->ada_b + (size_t)N * mpb * d, (size_t)2 * d, false);
+  } else {
+    UP_GAIN(H->fln_s);
+    UP(H->fln_b, (size_t)d, false);
+  }
+#undef UP_GAIN
+  {
+    std::vector<float> one((size_t)d, 1.0f);
+    if (cudaMemcpy(H->ones, one.data(), (size_t)d * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+      dit_destroy(H);
+      return DIT_ERR_CUDA;
+    }
+  }
+  UP(H->dec_w, (size_t)g.P * d, H->bf16);
   UP(H->dec_b, (size_t)g.P, false);
 #undef UP
 #undef ALLOC
 
-  if (launch_pos_tables(H->pos, H->rope, g.gf, g.gh, g.gw, d, g.dh, 0) != cudaSuccess ||
+  if (launch_pos_tables(H->pos, H->rope, g.gf, g.gh, g.gw, d, g.dh, g.Tc, 0) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess) {
     dit_destroy(H);
     return DIT_ERR_CUDA;
@@ -425,25 +604,42 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
 
   // ---------------- tensor maps (bf16 path)
   if (H->bf16) {
-    bool ok = make_tmap_bf16_kmajor(&H->tm_ada, H->ada_w, g.nmod, d, 128);
+    bool ok = g.nmod == 0 || make_tmap_bf16_kmajor(&H->tm_ada, H->ada_w, g.nmod, d, 128);
     const int bns[5] = {16, 32, 64, 128, 256};
     for (int i = 0; i < 5; ++i) ok = ok && make_tmap_bf16_kmajor(&H->tm_sc[i], H->sc, g.RPalloc, d, bns[i]);
+    if (cross) {
+      ok = ok && make_tmap_bf16_kmajor(&H->tm_xkv, H->xkv_w, g.nkv, d, 128);
+      for (int i = 0; i < 5; ++i) ok = ok && make_tmap_bf16_kmajor(&H->tm_ctx[i], H->ctx, g.CTXalloc, d, bns[i]);
+    }
     ok = ok && make_tmap_bf16_kmajor(&H->tm_u, H->u, g.Mmax, d, 128);
     ok = ok && make_tmap_bf16_kmajor(&H->tm_o, H->o, g.Mmax, d, 128);
-    ok = ok && make_tmap_bf16_kmajor(&H->tm_g, H->gbuf, g.Mmax, mlp, 128);
-    ok = ok && make_tmap_bf16(&H->tm_g_out, H->gbuf, g.Mmax, mlp, 32, 32, 64);
+    if (cfg->ffn_fp8) {
+      ok = ok && make_tmap_e4m3_kmajor(&H->tm_u8, H->u8, g.Mmax, d, 128) &&
+           make_tmap_e4m3_kmajor(&H->tb_g8, H->g8, g.Mmax, mlp, 256);
+    } else {
+      ok = ok && make_tmap_bf16_kmajor(&H->tm_g, H->gbuf, g.Mmax, mlp, 128) &&
+           make_tmap_bf16(&H->tm_g_out, H->gbuf, g.Mmax, mlp, 32, 32, 64) &&
+           make_tmap_bf16_kmajor(&H->tb_g, H->gbuf, g.Mmax, mlp, 256);
+    }
+    ok = ok && make_tmap_bf16_kmajor(&H->tm_dec, H->dec_w, g.dec_rows, d, g.bn_dec);
     ok = ok && make_tmap_f32(&H->tm_h_red, H->h, g.Mmax, d, 32, 16, 128);
     ok = ok && make_tmap_bf16_kmajor(&H->tb_u, H->u, g.Mmax, d, 256);
     ok = ok && make_tmap_bf16_kmajor(&H->tb_o, H->o, g.Mmax, d, 256);
-    ok = ok && make_tmap_bf16_kmajor(&H->tb_g, H->gbuf, g.Mmax, mlp, 256);
-    ok = ok && make_attention_maps(&H->attn_maps, H->q, H->k, H->v, H->o, g.Rmax, cfg->heads, g.T, g.Tpad, g.dh, g.DP, d);
+    ok = ok && make_attention_maps(&H->attn_maps, H->q, H->k, H->v, H->o, g.Rmax, cfg->heads, g.Ts, g.Tpad, g.dh, g.DP, d);
     for (int i = 0; i < N && ok; ++i) {
       BlockW& b = H->blk[i];
       ok = make_tmap_bf16_kmajor(&b.tm_qkv, b.qkv_w, 3 * d, d, g.headwise ? g.bn_qkv : 128) &&
-           make_tmap_bf16_kmajor(&b.tm_fc1, b.fc1_w, mlp, d, g.bn_fc1) &&
            make_tmap_bf16_kmajor(&b.ta_qkv, b.qkv_w, 3 * d, d, 128) &&
-           make_tmap_bf16_kmajor(&b.ta_proj, b.proj_w, d, d, 128) &&
-           make_tmap_bf16_kmajor(&b.ta_fc2, b.fc2_w, d, mlp, 128);
+           make_tmap_bf16_kmajor(&b.ta_proj, b.proj_w, d, d, 128);
+      if (cfg->ffn_fp8)
+        ok = ok && make_tmap_e4m3_kmajor(&b.tm_fc1_8, b.fc1_w8, mlp, d, g.bn_fc1) &&
+             make_tmap_e4m3_kmajor(&b.ta_fc2_8, b.fc2_w8, d, mlp, 128);
+      else
+        ok = ok && make_tmap_bf16_kmajor(&b.tm_fc1, b.fc1_w, mlp, d, g.bn_fc1) &&
+             make_tmap_bf16_kmajor(&b.ta_fc2, b.fc2_w, d, mlp, 128);
+      if (cross)
+        ok = ok && make_tmap_bf16_kmajor(&b.tm_xq, b.xq_w, d, d, 2 * g.dh) &&
+             make_tmap_bf16_kmajor(&b.ta_xo, b.xo_w, d, d, 128);
     }
     if (!ok) {
       dit_destroy(H);
@@ -458,8 +654,11 @@ int dit_forward_launch_count(const dit_handle* H, int B, float cfg_scale) {
   if (H == nullptr) return 0;
   (void)B;
   (void)cfg_scale;
-  const int per_block = 7 + ((!H->bf16 && (H->cfg.qk_norm || H->cfg.pos_kind == DIT_POS_ROPE3D)) ? 1 : 0);
-  return 3 + 1 + 1 + H->cfg.depth * per_block + 1 + 1;
+  const Geometry& g = H->g;
+  int per_block = 7 + ((!H->bf16 && (H->cfg.qk_norm || H->cfg.pos_kind == DIT_POS_ROPE3D)) ? 1 : 0);
+  if (g.kind == DIT_BLOCK_CROSS_ATTN) per_block += H->bf16 ? 3 : 4;
+  const int front = 3 + (g.nmod > 0 ? 1 : 0) + (g.nkv > 0 ? 1 : 0) + 1;  // condition, projections, embedding
+  return front + H->cfg.depth * per_block + 1 + 2;
 }
 
 }  // extern "C"
@@ -481,13 +680,15 @@ dit_status check_run(dit_handle* H, const void* x, const void* t, const void* y,
   p.B = B;
   p.guided = H->cfg.cond_kind == DIT_COND_CLASS && (s != 1.0f || H->force_guidance);
   p.R = p.guided ? 2 * B : B;
-  p.M = p.R * H->g.T;
+  p.M = p.R * H->g.Ts;
   p.s = s;
   return DIT_OK;
 }
 
+bool prof_on(const dit_handle* H, int kind) { return H->prof && (H->prof_kind < 0 || H->prof_kind == kind); }
+
 void prof_begin(dit_handle* H, int kind, cudaStream_t st) {
-  if (!H->prof) return;
+  if (!prof_on(H, kind)) return;
   const size_t i = H->prof_recs.size() * 2;
   while (H->ev_pool.size() < i + 2) {
     cudaEvent_t e;
@@ -498,20 +699,24 @@ void prof_begin(dit_handle* H, int kind, cudaStream_t st) {
   cudaEventRecord(H->ev_pool[i], st);
 }
 
-void prof_end(dit_handle* H, cudaStream_t st) {
-  if (!H->prof || H->prof_recs.empty()) return;
+void prof_end(dit_handle* H, int kind, cudaStream_t st) {
+  if (!prof_on(H, kind) || H->prof_recs.empty()) return;
   cudaEventRecord(H->ev_pool[H->prof_recs.back().second + 1], st);
 }
 
-#define DIT_LAUNCH(H, kind, st, call, where) \
-  do {                                      \
-    prof_begin(H, kind, st);                \
-    DIT_CK(H, call, where);                 \
-    prof_end(H, st);                        \
+// Launches `call` once (twice when DIT_OPT_REPEAT_KIND names its kind: a timing
+// diagnostic, the step time grows by the kind's in-pipeline cost).
+#define DIT_LAUNCH(H, kind, st, call, where)           \
+  do {                                                \
+    prof_begin(H, kind, st);                          \
+    DIT_CK(H, call, where);                           \
+    if (H->repeat_kind == (kind)) DIT_CK(H, call, where); \
+    prof_end(H, kind, st);                            \
   } while (0)
 
 dit_status run_condition(dit_handle* H, const float* t, const void* y, const RunPlan& p, cudaStream_t st) {
   const dit_config& c = H->cfg;
+  const Geometry& g = H->g;
   CondArgs a;
   a.t = t;
   a.y = y;
@@ -531,12 +736,25 @@ dit_status run_condition(dit_handle* H, const float* t, const void* y, const Run
   a.E = H->E;
   a.hid = H->hid;
   a.c = H->c;
-  a.sc = H->sc;
+  a.sc = g.mpb > 0 ? H->sc : nullptr;  // SiLU(c) feeds the modulation GEMM
   a.sc_bf16 = H->bf16;
   a.status = H->status;
+  if (g.kind == DIT_BLOCK_IN_CONTEXT) {  // e_t, e_y as the first two tokens of every row
+    a.tok_h = H->h;
+    a.tok_ld = (size_t)g.Ts * c.hidden;
+  } else if (g.kind == DIT_BLOCK_CROSS_ATTN) {  // e_t, e_y as the condition sequence
+    a.ctx = H->ctx;
+    a.ctx_bf16 = H->bf16;
+  }
   DIT_LAUNCH(H, DIT_KERNEL_COND, st, launch_condition(a, st), "condition");
   return DIT_OK;
 }
+
+// Row-independent (scale, shift) or per-row modulation vectors of one normalisation.
+struct Norm {
+  const float *shift, *scale;
+  int ld;
+};
 
 // Runs the forward through `stop_after` blocks (depth => the whole network, with
 // the final layer when out != nullptr).
@@ -544,12 +762,12 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
                        float* out, cudaStream_t st) {
   const dit_config& c = H->cfg;
   const Geometry& g = H->g;
-  const int d = c.hidden, mlp = c.mlp_hidden, T = g.T;
+  const int d = c.hidden, mlp = c.mlp_hidden, Ts = g.Ts;
   dit_status s = run_condition(H, t, y, p, st);
   if (s != DIT_OK) return s;
 
-  // modulation vectors of every block and the final layer: mod[r, (6N+2) d]
-  {
+  // modulation vectors of every block and the final layer: mod[r, nmod] (modulated designs)
+  if (g.nmod > 0) {
     EpiArgs ea = {};
     ea.M = g.nmod;
     ea.N = p.R;
@@ -567,10 +785,33 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
              "adaLN gemm");
     }
   }
+  // cross-attention keys and values of every block from the two condition tokens:
+  // xkv[2r + s, blk * 2d + (0: k | d: v)]
+  if (g.nkv > 0) {
+    EpiArgs ea = {};
+    ea.M = g.nkv;
+    ea.N = 2 * p.R;
+    ea.bias = H->xkv_b;
+    ea.out = H->xkv;
+    ea.ldo = g.nkv;
+    ea.status = H->status;
+    if (H->bf16) {
+      const int bn = adaln_bn(2 * p.R);
+      const int idx = bn == 16 ? 0 : bn == 32 ? 1 : bn == 64 ? 2 : bn == 128 ? 3 : 4;
+      DIT_LAUNCH(H, DIT_KERNEL_ADALN, st, launch_gemm_tc(EPI_ADALN, bn, &H->tm_xkv, &H->tm_ctx[idx], d, ea, H->num_sms, st),
+                 "condition key / value gemm");
+    } else {
+      DIT_LAUNCH(H, DIT_KERNEL_ADALN, st,
+                 launch_gemm_simt(EPI_ADALN, static_cast<const float*>(H->xkv_w), static_cast<const float*>(H->ctx),
+                                  g.nkv, 2 * p.R, d, ea, st),
+                 "condition key / value gemm");
+    }
+  }
   {
     PatchArgs a;
     a.x = x;
     a.w = H->pe_w;
+    a.wt = H->pe_wt;
     a.b = H->pe_b;
     a.pos = H->pos;
     a.h = H->h;
@@ -584,23 +825,78 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
     a.ph = c.patch_h;
     a.pw = c.patch_w;
     a.d = d;
+    a.Trow = Ts;
+    a.tok0 = g.Tc;
     DIT_LAUNCH(H, DIT_KERNEL_PATCH, st, launch_patch_embed(a, st), "patch embed");
   }
-  const int nblk = stop_after < c.depth ? stop_after : c.depth;
-  for (int i = 0; i < nblk; ++i) {
-    BlockW& b = H->blk[i];
-    const float* mb = H->mod + (size_t)i * 6 * d;
+  auto run_ln = [&](const Norm& n, const char* where) -> dit_status {
     LnArgs ln;
     ln.h = H->h;
     ln.u = H->u;
     ln.u_bf16 = H->bf16;
-    ln.ld_mod = g.nmod;
+    ln.ld_mod = n.ld;
     ln.M = p.M;
-    ln.T = T;
+    ln.T = Ts;
     ln.d = d;
-    ln.shift = mb;
-    ln.scale = mb + d;
-    DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "ln1");
+    ln.shift = n.shift;
+    ln.scale = n.scale;
+    DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), where);
+    return DIT_OK;
+  };
+  // gated residual update h += gate[row] * (A W^T + b) on the tensor cores (swapped operands)
+  // or the SIMT GEMM
+  auto run_resid = [&](int kind, const CUtensorMap* ta, const CUtensorMap* tb, const void* A, const void* W, int K,
+                       const float* bias, const float* gate, int ld_gate, const char* where) -> dit_status {
+    EpiArgs pa = {};
+    pa.M = p.M;
+    pa.N = d;
+    pa.bias = bias;
+    pa.h = H->h;
+    pa.ldh = d;
+    pa.gate = gate;
+    pa.ld_gate = ld_gate;
+    pa.T = Ts;
+    pa.status = H->status;
+    if (H->bf16) {
+      EpiArgs pt = pa;  // swapped: rows = d output features, columns = tokens
+      pt.M = d;
+      pt.N = p.M;
+      DIT_LAUNCH(H, kind, st, launch_gemm_tc(EPI_RESID_T, 256, ta, tb, K, pt, H->num_sms, st, &H->tm_h_red), where);
+    } else {
+      DIT_LAUNCH(H, kind, st,
+                 launch_gemm_simt(EPI_RESID, static_cast<const float*>(A), static_cast<const float*>(W), p.M, d, K, pa, st),
+                 where);
+    }
+    return DIT_OK;
+  };
+#define DIT_TRY(call)               \
+  do {                              \
+    const dit_status s_ = (call);   \
+    if (s_ != DIT_OK) return s_;    \
+  } while (0)
+
+  const bool modulated = g.mpb > 0;
+  const int nblk = stop_after < c.depth ? stop_after : c.depth;
+  for (int i = 0; i < nblk; ++i) {
+    BlockW& b = H->blk[i];
+    const float* mb = modulated ? H->mod + (size_t)i * g.mpb * d : nullptr;
+    Norm n1, n2;
+    const float *gate1 = H->ones, *gate2 = H->ones;
+    int ld_gate = 0;
+    if (g.kind == DIT_BLOCK_ADALN_ZERO) {  // (shift1, scale1, gate1, shift2, scale2, gate2)
+      n1 = {mb, mb + d, g.nmod};
+      n2 = {mb + 3 * d, mb + 4 * d, g.nmod};
+      gate1 = mb + 2 * d;
+      gate2 = mb + 5 * d;
+      ld_gate = g.nmod;
+    } else if (g.kind == DIT_BLOCK_ADALN) {  // (shift1, scale1, shift2, scale2), no gates
+      n1 = {mb, mb + d, g.nmod};
+      n2 = {mb + 2 * d, mb + 3 * d, g.nmod};
+    } else {  // learned LayerNorm affines, the same for every row
+      n1 = {b.ln1_b, b.ln1_s, 0};
+      n2 = {b.ln2_b, b.ln2_s, 0};
+    }
+    DIT_TRY(run_ln(n1, "ln1"));
 
     EpiArgs qa = {};
     qa.M = p.M;
@@ -614,7 +910,7 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
     qa.dh = g.dh;
     qa.DP = g.DP;
     qa.Tpad = g.Tpad;
-    qa.T = T;
+    qa.T = Ts;
     qa.qn = b.qn;
     qa.kn = b.kn;
     qa.rope = H->rope;
@@ -626,32 +922,12 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
     aa.o = H->o;
     aa.R = p.R;
     aa.H = c.heads;
-    aa.T = T;
+    aa.T = Ts;
     aa.dh = g.dh;
     aa.DP = g.DP;
     aa.Tpad = g.Tpad;
     aa.d = d;
     aa.bf16 = H->bf16;
-    EpiArgs pa = {};
-    pa.M = p.M;
-    pa.N = d;
-    pa.bias = b.proj_b;
-    pa.h = H->h;
-    pa.ldh = d;
-    pa.gate = mb + 2 * d;
-    pa.ld_gate = g.nmod;
-    pa.T = T;
-    pa.status = H->status;
-    EpiArgs f1 = {};
-    f1.M = p.M;
-    f1.N = mlp;
-    f1.bias = b.fc1_b;
-    f1.out = H->gbuf;
-    f1.ldo = mlp;
-    f1.status = H->status;
-    EpiArgs f2 = pa;
-    f2.bias = b.fc2_b;
-    f2.gate = mb + 5 * d;
 
     if (H->bf16) {
       if (g.headwise) {
@@ -665,12 +941,6 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
                    "qkv gemm");
       }
       DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_tc(aa, H->attn_maps, H->status, st), "attention");
-      EpiArgs pt = pa;  // swapped: rows = d output features, columns = tokens
-      pt.M = d;
-      pt.N = p.M;
-      DIT_LAUNCH(H, DIT_KERNEL_PROJ, st,
-                 launch_gemm_tc(EPI_RESID_T, 256, &b.ta_proj, &H->tb_o, d, pt, H->num_sms, st, &H->tm_h_red),
-                 "proj gemm");
     } else {
       DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_simt(EPI_QKV, static_cast<const float*>(H->u), static_cast<const float*>(b.qkv_w), p.M,
                                  3 * d, d, qa, st),
@@ -683,71 +953,170 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
         qn.kn = b.kn;
         qn.rope = H->rope;
         qn.RH = p.R * c.heads;
-        qn.T = T;
+        qn.T = Ts;
         qn.dh = g.dh;
         DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_qknorm_rope_f32(qn, st), "qk norm");
       }
       DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_simt(aa, st), "attention");
-      DIT_LAUNCH(H, DIT_KERNEL_PROJ, st, launch_gemm_simt(EPI_RESID, static_cast<const float*>(H->o), static_cast<const float*>(b.proj_w), p.M, d,
-                                 d, pa, st),
-             "proj gemm");
     }
-    ln.shift = mb + 3 * d;
-    ln.scale = mb + 4 * d;
-    DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "ln2");
+    DIT_TRY(run_resid(DIT_KERNEL_PROJ, &b.ta_proj, &H->tb_o, H->o, b.proj_w, d, b.proj_b, gate1, ld_gate, "proj gemm"));
+
+    if (g.kind == DIT_BLOCK_CROSS_ATTN) {  // h += CrossAttn(LNx(h), [e_t, e_y])
+      DIT_TRY(run_ln(Norm{b.xln_b, b.xln_s, 0}, "cross-attention ln"));
+      const float* xkv = H->xkv + (size_t)i * 2 * d;
+      if (H->bf16) {
+        EpiArgs xa = {};
+        xa.M = p.M;
+        xa.N = d;
+        xa.bias = b.xq_b;
+        xa.xkv = xkv;
+        xa.ld_xkv = g.nkv;
+        xa.xo = H->o;
+        xa.d = d;
+        xa.T = Ts;
+        xa.status = H->status;
+        DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_gemm_tc(EPI_XATTN, 2 * g.dh, &H->tm_u, &b.tm_xq, d, xa, H->num_sms, st),
+                   "cross-attention query gemm");
+      } else {
+        EpiArgs xa = {};
+        xa.M = p.M;
+        xa.N = d;
+        xa.bias = b.xq_b;
+        xa.out = H->q;  // [M, d] float32 queries (the q buffer is free until the next block)
+        xa.ldo = d;
+        xa.status = H->status;
+        DIT_LAUNCH(H, DIT_KERNEL_ATTN, st,
+                   launch_gemm_simt(EPI_F32, static_cast<const float*>(H->u), static_cast<const float*>(b.xq_w), p.M, d,
+                                    d, xa, st),
+                   "cross-attention query gemm");
+        XAttnArgs xk;
+        xk.q = static_cast<const float*>(H->q);
+        xk.xkv = xkv;
+        xk.ld_xkv = g.nkv;
+        xk.o = static_cast<float*>(H->o);
+        xk.M = p.M;
+        xk.T = Ts;
+        xk.d = d;
+        xk.H = c.heads;
+        xk.dh = g.dh;
+        DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_xattn_f32(xk, st), "cross-attention");
+      }
+      DIT_TRY(run_resid(DIT_KERNEL_PROJ, &b.ta_xo, &H->tb_o, H->o, b.xo_w, d, b.xo_b, H->ones, 0,
+                        "cross-attention output gemm"));
+    }
+
+    if (c.ffn_fp8) {  // feed-forward with E4M3 operands on the tensor cores (kind::f8f6f4)
+      LnArgs ln;
+      ln.h = H->h;
+      ln.u = H->u;
+      ln.u_bf16 = 1;
+      ln.u8 = H->u8;
+      ln.su = H->su;
+      ln.sg = H->sg;
+      ln.g_w = b.g_w;
+      ln.g_b = b.g_b;
+      ln.ld_mod = n2.ld;
+      ln.M = p.M;
+      ln.T = Ts;
+      ln.d = d;
+      ln.shift = n2.shift;
+      ln.scale = n2.scale;
+      DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "ln2 (fp8)");
+      EpiArgs f1 = {};
+      f1.M = p.M;
+      f1.N = mlp;
+      f1.bias = b.fc1_b;
+      f1.out = H->g8;
+      f1.ldo = mlp;
+      f1.sa = H->su;
+      f1.sb = b.fc1_s;
+      f1.sg = H->sg;
+      f1.status = H->status;
+      DIT_LAUNCH(H, DIT_KERNEL_FC1, st, launch_gemm_tc(EPI_GELU8, 256, &H->tm_u8, &b.tm_fc1_8, d, f1, H->num_sms, st),
+                 "fc1 gemm (fp8)");
+      EpiArgs f2 = {};
+      f2.M = d;
+      f2.N = p.M;
+      f2.bias = b.fc2_b;
+      f2.h = H->h;
+      f2.ldh = d;
+      f2.gate = gate2;
+      f2.ld_gate = ld_gate;
+      f2.T = Ts;
+      f2.sa = b.fc2_s;
+      f2.sb = H->sg;
+      f2.status = H->status;
+      DIT_LAUNCH(H, DIT_KERNEL_FC2, st,
+                 launch_gemm_tc(EPI_RESID_T8, 256, &b.ta_fc2_8, &H->tb_g8, mlp, f2, H->num_sms, st, &H->tm_h_red),
+                 "fc2 gemm (fp8)");
+      continue;
+    }
+    DIT_TRY(run_ln(n2, "ln2"));
+    EpiArgs f1 = {};
+    f1.M = p.M;
+    f1.N = mlp;
+    f1.bias = b.fc1_b;
+    f1.out = H->gbuf;
+    f1.ldo = mlp;
+    f1.status = H->status;
     if (H->bf16) {
       DIT_LAUNCH(H, DIT_KERNEL_FC1, st,
                  launch_gemm_tc(EPI_GELU, g.bn_fc1, &H->tm_u, &b.tm_fc1, d, f1, H->num_sms, st, &H->tm_g_out),
                  "fc1 gemm");
-      EpiArgs ft = f2;  // swapped: rows = d output features, columns = tokens
-      ft.M = d;
-      ft.N = p.M;
-      DIT_LAUNCH(H, DIT_KERNEL_FC2, st,
-                 launch_gemm_tc(EPI_RESID_T, 256, &b.ta_fc2, &H->tb_g, mlp, ft, H->num_sms, st, &H->tm_h_red),
-                 "fc2 gemm");
     } else {
       DIT_LAUNCH(H, DIT_KERNEL_FC1, st, launch_gemm_simt(EPI_GELU, static_cast<const float*>(H->u), static_cast<const float*>(b.fc1_w), p.M,
                                  mlp, d, f1, st),
              "fc1 gemm");
-      DIT_LAUNCH(H, DIT_KERNEL_FC2, st, launch_gemm_simt(EPI_RESID, static_cast<const float*>(H->gbuf), static_cast<const float*>(b.fc2_w), p.M,
-                                 d, mlp, f2, st),
-             "fc2 gemm");
     }
+    DIT_TRY(run_resid(DIT_KERNEL_FC2, &b.ta_fc2, &H->tb_g, H->gbuf, b.fc2_w, mlp, b.fc2_b, gate2, ld_gate, "fc2 gemm"));
   }
   if (out == nullptr) return DIT_OK;
 
-  LnArgs ln;
-  ln.h = H->h;
-  ln.u = H->u;
-  ln.u_bf16 = H->bf16;
-  ln.ld_mod = g.nmod;
-  ln.M = p.M;
-  ln.T = T;
-  ln.d = d;
-  ln.shift = H->mod + (size_t)c.depth * 6 * d;
-  ln.scale = ln.shift + d;
-  DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "final ln");
-  DecodeArgs da;
-  da.u = H->u;
-  da.u_bf16 = H->bf16;
-  da.w = H->dec_w;
-  da.b = H->dec_b;
-  da.out = out;
-  da.B = p.B;
-  da.T = T;
-  da.d = d;
-  da.P = g.P;
-  da.Cout = g.Cout;
-  da.F = c.frames;
-  da.H = c.height;
-  da.W = c.width;
-  da.pt = c.patch_t;
-  da.ph = c.patch_h;
-  da.pw = c.patch_w;
-  da.guided = p.guided;
-  da.s = p.s;
-  da.gch = H->cfg_channels;
-  DIT_LAUNCH(H, DIT_KERNEL_DECODE, st, launch_decode_cfg(da, st), "decode");
+  // final layer: modulated (adaLN designs) or learned-affine LayerNorm
+  if (modulated) {
+    const float* fm = H->mod + (size_t)c.depth * g.mpb * d;
+    DIT_TRY(run_ln(Norm{fm, fm + d, g.nmod}, "final ln"));
+  } else {
+    DIT_TRY(run_ln(Norm{H->fln_b, H->fln_s, 0}, "final ln"));
+  }
+#undef DIT_TRY
+  // linear decoder z = u W_dec^T + b_dec [M, P] (tensor cores on the bf16 path), then the
+  // guidance combine and unpatchify (condition tokens are skipped)
+  EpiArgs de = {};
+  de.M = p.M;
+  de.N = g.P;
+  de.bias = H->dec_b;
+  de.out = H->z;
+  de.ldo = g.P;
+  de.status = H->status;
+  if (H->bf16) {
+    DIT_LAUNCH(H, DIT_KERNEL_DECODE, st, launch_gemm_tc(EPI_F32, g.bn_dec, &H->tm_u, &H->tm_dec, d, de, H->num_sms, st),
+               "decoder gemm");
+  } else {
+    DIT_LAUNCH(H, DIT_KERNEL_DECODE, st,
+               launch_gemm_simt(EPI_F32, static_cast<const float*>(H->u), static_cast<const float*>(H->dec_w), p.M, g.P,
+                                d, de, st),
+               "decoder gemm");
+  }
+  UnpatchArgs ua;
+  ua.z = H->z;
+  ua.out = out;
+  ua.B = p.B;
+  ua.T = g.T;
+  ua.P = g.P;
+  ua.Cout = g.Cout;
+  ua.F = c.frames;
+  ua.H = c.height;
+  ua.W = c.width;
+  ua.pt = c.patch_t;
+  ua.ph = c.patch_h;
+  ua.pw = c.patch_w;
+  ua.guided = p.guided;
+  ua.s = p.s;
+  ua.gch = H->cfg_channels;
+  ua.Trow = Ts;
+  ua.tok0 = g.Tc;
+  DIT_LAUNCH(H, DIT_KERNEL_DECODE, st, launch_cfg_unpatchify(ua, H->num_sms, st), "guidance + unpatchify");
   return DIT_OK;
 }
 
@@ -760,7 +1129,7 @@ dit_status run_forward_cached(dit_handle* H, const float* x, const float* t, con
                               float* out, cudaStream_t st) {
   const int depth = H->cfg.depth;
   if (!H->use_graph || H->prof) return run_forward(H, x, t, y, p, depth, out, st);
-  dit_handle::GraphKey k{x, t, y, out, p.B, p.R, depth, H->cfg_channels, p.guided, g_pdl, p.s};
+  dit_handle::GraphKey k{x, t, y, out, p.B, p.R, depth, H->cfg_channels, H->repeat_kind, p.guided, g_pdl, p.s};
   if (H->gexec != nullptr && k == H->gkey) {
     DIT_CK(H, cudaGraphLaunch(H->gexec, st), "graph launch");
     return DIT_OK;
@@ -863,6 +1232,11 @@ dit_status dit_set_option(dit_handle* H, int option, int value) {
     H->cfg_channels = value;
     return DIT_OK;
   }
+  if (option == DIT_OPT_REPEAT_KIND) {
+    if (value < -1 || value >= DIT_KERNEL_COUNT) return fail(H, DIT_ERR_INVALID_ARG, "unknown kernel kind");
+    H->repeat_kind = value;
+    return DIT_OK;
+  }
 
   return fail(H, DIT_ERR_INVALID_ARG, "unknown option");
 }
@@ -923,6 +1297,7 @@ dit_status dit_sample(dit_handle* H, int kind, float* x, const void* y, int B, f
   k.kind = kind;
   k.steps = steps;
   k.gch = H->cfg_channels;
+  k.rep = H->repeat_kind;
   k.guided = p.guided;
   k.pdl = g_pdl;
   k.s = p.s;
@@ -1026,7 +1401,9 @@ dit_status dit_debug_wait_probe(dit_handle* H, int timeout_us, dit_stream_t stre
 
 dit_status dit_profile_enable(dit_handle* H, int enable) {
   if (H == nullptr) return DIT_ERR_INVALID_ARG;
+  if (enable < 0 || enable >= 2 + DIT_KERNEL_COUNT) return fail(H, DIT_ERR_INVALID_ARG, "bad profiling mode");
   H->prof = enable != 0;
+  H->prof_kind = enable >= 2 ? enable - 2 : -1;
   return DIT_OK;
 }
 
@@ -1070,6 +1447,68 @@ static dit_status op_linear(const uint16_t* x, const uint16_t* w, const float* b
   const cudaError_t e = pair ? launch_gemm_tc2(EPI_F32, block_n, &ta, &tb, K, ea, sms, st)
                              : launch_gemm_tc(EPI_F32, block_n, &ta, &tb, K, ea, sms, st);
   return e == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+dit_status dit_op_linear_e4m3(const uint8_t* x, const uint8_t* w, const float* sx, const float* sw, const float* b,
+                              float* y, int M, int N, int K, int block_n, dit_stream_t stream) {
+  if (x == nullptr || w == nullptr || sx == nullptr || sw == nullptr || y == nullptr || M < 0 || N <= 0 || K <= 0 ||
+      (K % 16) != 0)
+    return DIT_ERR_INVALID_ARG;
+  if (block_n != 64 && block_n != 128 && block_n != 256) return DIT_ERR_INVALID_ARG;
+  if (M == 0) return DIT_OK;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return DIT_ERR_NO_DEVICE;
+  CUtensorMap ta, tb;
+  if (!make_tmap_e4m3_kmajor(&ta, x, M, K, 128) || !make_tmap_e4m3_kmajor(&tb, w, N, K, block_n))
+    return DIT_ERR_INVALID_ARG;
+  EpiArgs ea = {};
+  ea.M = M;
+  ea.N = N;
+  ea.bias = b;
+  ea.out = y;
+  ea.ldo = N;
+  ea.sa = sx;
+  ea.sb = sw;
+  return launch_gemm_tc(EPI_F32_8, block_n, &ta, &tb, K, ea, sms, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? DIT_OK
+             : DIT_ERR_CUDA;
+}
+
+dit_status dit_op_attention_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int R, int H,
+                                 int T, int dh, int* counters, dit_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || R < 0 || H <= 0 || T <= 0)
+    return DIT_ERR_INVALID_ARG;
+  if (dh != 64 && dh != 72) return DIT_ERR_UNSUPPORTED;
+  if (R == 0) return DIT_OK;
+  const int DP = (dh + 15) / 16 * 16, Tpad = (T + 127) / 128 * 128, d = H * dh;
+  AttnMaps maps;
+  if (!make_attention_maps(&maps, q, k, v, o, R, H, T, Tpad, dh, DP, d)) return DIT_ERR_INVALID_ARG;
+  AttnArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.R = R;
+  a.H = H;
+  a.T = T;
+  a.dh = dh;
+  a.DP = DP;
+  a.Tpad = Tpad;
+  a.d = d;
+  a.bf16 = 1;
+  return launch_attention_tc(a, maps, counters, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? DIT_OK
+                                                                                                         : DIT_ERR_CUDA;
+}
+
+dit_status dit_debug_attention_rescales(dit_handle* H, long long* count) {
+  if (H == nullptr || count == nullptr) return DIT_ERR_INVALID_ARG;
+  DIT_CK(H, cudaDeviceSynchronize(), "sync");
+  int v = 0;
+  DIT_CK(H, cudaMemcpy(&v, H->status + 1, 4, cudaMemcpyDeviceToHost), "counter read");
+  DIT_CK(H, cudaMemset(H->status + 1, 0, 4), "counter clear");
+  *count = v;
+  return DIT_OK;
 }
 
 dit_status dit_op_linear_bf16_pair(const uint16_t* x, const uint16_t* w, const float* b, float* y, int M, int N, int K,

@@ -53,6 +53,11 @@ __device__ __forceinline__ void epilogue_chunk(const EpiArgs& ea, const uint32_t
     } else {
       for (int i = 0; i < W && n + i < ea.N; ++i) o[i] = __uint_as_float(r[i]) + (ea.bias ? __ldg(ea.bias + n + i) : 0.f);
     }
+  } else if constexpr (EPI == EPI_F32_8) {
+    const float sm = __ldg(ea.sa + m);
+    float* o = static_cast<float*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n;
+    for (int i = 0; i < W && n + i < ea.N; ++i)
+      o[i] = __uint_as_float(r[i]) * sm * __ldg(ea.sb + n + i) + (ea.bias ? __ldg(ea.bias + n + i) : 0.f);
   } else if constexpr (EPI == EPI_GELU) {
     uint16_t* o = static_cast<uint16_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n;
     if (full) {
@@ -181,6 +186,48 @@ __device__ __forceinline__ void epilogue_head(const EpiArgs& ea, const uint32_t*
   }
 }
 
+// Cross-attention of one token onto the two condition tokens of its row, for one head,
+// fused into the query projection: q = acc + bias over the head's DH columns (n is the
+// head's first column, a multiple of DH), scores s_k = q . key_k / sqrt(DH) for k = 0, 1,
+// softmax, and o = p_0 value_0 + p_1 value_1 written as bf16 to xo[m, n .. n + DH).
+template <int DH>
+__device__ __forceinline__ void epilogue_xattn(const EpiArgs& ea, const uint32_t* r, int m, int n) {
+  if (n >= ea.N || m >= ea.M) return;
+  const int row = m / ea.T;
+  const float4* k0 = reinterpret_cast<const float4*>(ea.xkv + static_cast<size_t>(2 * row) * ea.ld_xkv + n);
+  const float4* k1 = reinterpret_cast<const float4*>(ea.xkv + static_cast<size_t>(2 * row + 1) * ea.ld_xkv + n);
+  const float4* v0 = k0 + ea.d / 4;
+  const float4* v1 = k1 + ea.d / 4;
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int j4 = 0; j4 < DH / 4; ++j4) {
+    const float4 b4 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + j4);
+    const float4 a = __ldg(k0 + j4), b = __ldg(k1 + j4);
+    const float q0 = __uint_as_float(r[4 * j4 + 0]) + b4.x, q1 = __uint_as_float(r[4 * j4 + 1]) + b4.y;
+    const float q2 = __uint_as_float(r[4 * j4 + 2]) + b4.z, q3 = __uint_as_float(r[4 * j4 + 3]) + b4.w;
+    s0 = fmaf(q0, a.x, fmaf(q1, a.y, fmaf(q2, a.z, fmaf(q3, a.w, s0))));
+    s1 = fmaf(q0, b.x, fmaf(q1, b.y, fmaf(q2, b.z, fmaf(q3, b.w, s1))));
+  }
+  const float sc = rsqrtf(static_cast<float>(DH));
+  s0 *= sc;
+  s1 *= sc;
+  const float mx = fmaxf(s0, s1);
+  const float e0 = expf(s0 - mx), e1 = expf(s1 - mx);
+  const float inv = 1.0f / (e0 + e1);
+  const float p0 = e0 * inv, p1 = e1 * inv;
+  uint16_t* dst = static_cast<uint16_t*>(ea.xo) + static_cast<size_t>(m) * ea.d + n;
+#pragma unroll
+  for (int c = 0; c < DH / 8; ++c) {
+    const float4 a0 = __ldg(v0 + 2 * c), a1 = __ldg(v0 + 2 * c + 1);
+    const float4 b0 = __ldg(v1 + 2 * c), b1 = __ldg(v1 + 2 * c + 1);
+    *reinterpret_cast<uint4*>(dst + c * 8) =
+        make_uint4(pack_bf16x2(p0 * a0.x + p1 * b0.x, p0 * a0.y + p1 * b0.y),
+                   pack_bf16x2(p0 * a0.z + p1 * b0.z, p0 * a0.w + p1 * b0.w),
+                   pack_bf16x2(p0 * a1.x + p1 * b1.x, p0 * a1.y + p1 * b1.y),
+                   pack_bf16x2(p0 * a1.z + p1 * b1.z, p0 * a1.w + p1 * b1.w));
+  }
+}
+
 // The columns [n0 + c0, n0 + c0 + NC) of a tile for output row m; tacc addresses
 // column 0 of the tile in this warp's TMEM lanes.
 template <int NC, int EPI, bool HEADWISE>
@@ -192,7 +239,10 @@ __device__ __forceinline__ void epilogue_cols(const EpiArgs& ea, uint32_t tacc, 
 #pragma unroll
     for (int c = 0; c < NC / 8; ++c) DIT_TMEM_LD_X8(tacc + c0 + c * 8, (r + c * 8));
     tmem_ld_wait<NC>(r);
-    epilogue_head<NC>(ea, r, m, n0 + c0);
+    if constexpr (EPI == EPI_XATTN)
+      epilogue_xattn<NC>(ea, r, m, n0 + c0);
+    else
+      epilogue_head<NC>(ea, r, m, n0 + c0);
   } else {
     constexpr int W = NC % 32 == 0 ? 32 : (NC % 16 == 0 ? 16 : 8);
     constexpr int NCH = NC / W;
@@ -208,14 +258,15 @@ __device__ __forceinline__ void epilogue_cols(const EpiArgs& ea, uint32_t tacc, 
   }
 }
 
-// Epilogues that write through shared memory: each warp turns a 32-row x 32-column
-// chunk into a swizzled box in its own 4 KB staging buffer and one lane hands it to
-// the TMA unit (GELU: bf16 store; RESID: float32 reduce-add into the residual
-// stream, so the SM never reads the stream back).  Stores leave as whole rows
-// instead of 32 scattered row pieces per instruction.
+// Epilogues that write through shared memory, each warp in its own 4 KB staging
+// buffer: GELU stages a 32-row x 32-column bf16 chunk and writes it back out with plain
+// coalesced 16-byte stores (whole 64-byte row segments instead of 32 scattered pieces
+// per instruction); RESID_T stages [token][feature] boxes that one lane hands to the
+// TMA unit as a float32 reduce-add into the residual stream, so the SM never reads the
+// stream back.
 template <int EPI>
 __host__ __device__ constexpr bool epi_staged() {
-  return EPI == EPI_GELU || EPI == EPI_RESID_T;
+  return EPI == EPI_GELU || EPI == EPI_RESID_T || EPI == EPI_RESID_T8;
 }
 constexpr int kStageBytesPerWarp = 4096;
 constexpr int kEpilogueWarps = 8;
@@ -277,7 +328,9 @@ __device__ __forceinline__ void epilogue_cols_staged(const EpiArgs& ea, const CU
 // buffers, written one token row per instruction by the 32 lanes, and added into the
 // residual stream by the TMA unit (cp.reduce.async.bulk .add), so the SM never reads
 // the stream back.
-template <int NC>
+// FP8 = true: E4M3 operands, the accumulator is first scaled by the weight row's scale sa[f]
+// and each token's scale sb[tok].
+template <int NC, bool FP8 = false>
 __device__ __forceinline__ void epilogue_resid_t(const EpiArgs& ea, const CUtensorMap* tmC, uint32_t tacc, int f_base,
                                                  int lane, int n0, int c0, uint8_t* stg) {
   static_assert(NC % 32 == 0, "32-token chunks");
@@ -285,6 +338,7 @@ __device__ __forceinline__ void epilogue_resid_t(const EpiArgs& ea, const CUtens
   const int f = f_base + lane;
   const bool fok = f < ea.M;
   const float bf = fok ? __ldg(ea.bias + f) : 0.f;
+  const float sf = (FP8 && fok) ? __ldg(ea.sa + f) : 1.f;
   uint32_t r[2][32];
   tmem_ld_chunk<32>(tacc + c0, r[0]);
   tmem_ld_wait<32>(r[0]);
@@ -297,6 +351,8 @@ __device__ __forceinline__ void epilogue_resid_t(const EpiArgs& ea, const CUtens
       const int last = min(tok0 + 31, ea.N - 1);
       const int r0 = tok0 / ea.T, r1 = last / ea.T;
       const float g0 = fok ? __ldg(ea.gate + static_cast<size_t>(r0) * ea.ld_gate + f) : 0.f;
+      // FP8: lane l holds token tok0 + l's scale, handed to every lane below
+      const float st_l = FP8 ? (tok0 + lane < ea.N ? __ldg(ea.sb + tok0 + lane) : 0.f) : 1.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {  // 16 tokens per box, alternating 2 KB buffers
         uint8_t* buf = stg + half * 2048;
@@ -310,9 +366,11 @@ __device__ __forceinline__ void epilogue_resid_t(const EpiArgs& ea, const CUtens
             const int rt = min(tok0 + t, ea.N - 1) / ea.T;
             g = fok ? __ldg(ea.gate + static_cast<size_t>(rt) * ea.ld_gate + f) : 0.f;
           }
+          float acc = __uint_as_float(v[t]);
+          if constexpr (FP8) acc *= sf * __shfl_sync(0xffffffffu, st_l, t);
           // [token][feature] float32 rows of 128 bytes, 128B swizzle
           *reinterpret_cast<float*>(buf + tt * 128 + ((((lane >> 2) ^ (tt & 7)) << 4) | ((lane & 3) << 2))) =
-              g * (__uint_as_float(v[t]) + bf);
+              g * (acc + bf);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -321,6 +379,45 @@ __device__ __forceinline__ void epilogue_resid_t(const EpiArgs& ea, const CUtens
           bulk_commit_group();
         }
       }
+    }
+    if (c + 1 < NCH) tmem_ld_wait<32>(r[(c + 1) & 1]);
+  }
+}
+
+// FP8 feed-forward hidden layer: for output row m and columns [n0 + c0, n0 + c0 + NC),
+// z = sa[m] sb[n] acc + bias[n], g = gelu_tanh(z), stored as E4M3 g / sg[m] (one byte per
+// column; 32 columns leave as two 16-byte stores per thread).
+template <int NC>
+__device__ __forceinline__ void epilogue_gelu8(const EpiArgs& ea, uint32_t tacc, int m, int n0, int c0) {
+  static_assert(NC % 32 == 0, "32-column chunks");
+  constexpr int NCH = NC / 32;
+  const bool mok = m < ea.M;
+  const float sm = mok ? __ldg(ea.sa + m) : 0.f;
+  const float inv = mok ? 1.0f / __ldg(ea.sg + m) : 0.f;
+  uint32_t r[2][32];
+  tmem_ld_chunk<32>(tacc + c0, r[0]);
+  tmem_ld_wait<32>(r[0]);
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    if (c + 1 < NCH) tmem_ld_chunk<32>(tacc + c0 + (c + 1) * 32, r[(c + 1) & 1]);
+    const int n = n0 + c0 + c * 32;
+    const uint32_t* v = r[c & 1];
+    if (mok && n < ea.N) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int i4 = 0; i4 < 8; ++i4) {
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(ea.sb + n) + i4);
+        const float4 b4 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + i4);
+        const float z0 = fmaf(__uint_as_float(v[4 * i4 + 0]) * sm, s4.x, b4.x);
+        const float z1 = fmaf(__uint_as_float(v[4 * i4 + 1]) * sm, s4.y, b4.y);
+        const float z2 = fmaf(__uint_as_float(v[4 * i4 + 2]) * sm, s4.z, b4.z);
+        const float z3 = fmaf(__uint_as_float(v[4 * i4 + 3]) * sm, s4.w, b4.w);
+        pk[i4] = pack_e4m3x4(gelu_tanh_fast(z0) * inv, gelu_tanh_fast(z1) * inv, gelu_tanh_fast(z2) * inv,
+                             gelu_tanh_fast(z3) * inv);
+      }
+      uint4* o = reinterpret_cast<uint4*>(static_cast<uint8_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n);
+      o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
     if (c + 1 < NCH) tmem_ld_wait<32>(r[(c + 1) & 1]);
   }

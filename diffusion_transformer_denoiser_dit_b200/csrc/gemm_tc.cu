@@ -1,17 +1,20 @@
 // Tensor-core GEMM for sm_100a: D[M, N] = A[M, K] * B[N, K]^T, bf16 operands,
 // float32 accumulation in tensor memory, with the DiT epilogues fused in.
 //
-// Design (one persistent CTA per SM, 192 threads):
+// Design (one persistent CTA per SM, 320 threads = 10 warps):
 //   warp 0      TMA producer: 128x64 A tile + BNx64 B tile per stage, 128-byte
 //               swizzle, STAGES-deep ring guarded by full/empty mbarriers.
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
 //               (M=128, N=BN, K=16, four per 64-wide stage) into one of two TMEM
 //               accumulators and commits stage releases / accumulator hand-off.
-//   warps 2..5  epilogue: tcgen05.ld of its 32 TMEM lanes (one output row per
-//               thread), bias / GELU / gated residual / head-major scatter with
-//               QK-RMSNorm and 3D RoPE, stores to global memory.  Two accumulators
-//               let the epilogue of tile i overlap the main loop of tile i+1.
-// Every mbarrier wait is bounded (common.cuh); no TMA multicast is used.
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (one output row per
+//               thread) and one half of the tile's columns (warps 2-5 the first half,
+//               6-9 the second); bias / GELU / gated residual / head-major scatter with
+//               QK-RMSNorm and 3D RoPE, stores to global memory.  Two accumulators let
+//               the epilogue of tile i overlap the main loop of tile i+1.
+// Every mbarrier wait is bounded (common.cuh); no TMA multicast is used.  When a wait
+// runs out, the producer and the MMA issuer first wait (bounded again) for the copies
+// and MMAs they already issued before the CTA frees its TMEM and exits.
 #include "common.cuh"
 #include "gemm_epilogue.cuh"
 #include "internal.h"
@@ -20,9 +23,10 @@ namespace dit {
 
 template <int BN, int EPI>
 struct TcCfg {
-  static constexpr int BM = 128, BK = 64;
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr bool F8 = epi_fp8<EPI>();            // E4M3 operands (one byte per element)
+  static constexpr int BM = 128, BK = F8 ? 128 : 64;    // K elements per 128-byte stage row
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGING = epi_staged<EPI>() ? kEpilogueWarps * kStageBytesPerWarp : 0;
   static constexpr int BAR_BYTES = 256;
@@ -47,19 +51,20 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(staging + C::STAGING);
-  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 4);
+  uint32_t* holder = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
   const uint32_t bar0 = smem_u32(bars);
   // barrier addresses: full[s], empty[s], tmem_full[a], tmem_empty[a]
 #define FULL_BAR(s) (bar0 + 8u * (s))
 #define EMPTY_BAR(s) (bar0 + 8u * (C::STAGES + (s)))
 #define TFULL_BAR(a) (bar0 + 8u * (2 * C::STAGES + (a)))
 #define TEMPTY_BAR(a) (bar0 + 8u * (2 * C::STAGES + 2 + (a)))
+#define DRAIN_BAR (bar0 + 8u * (2 * C::STAGES + 4))
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m_tiles = (ea.M + 127) / 128;
   const int n_tiles = (ea.N + BN - 1) / BN;
   const int num_tiles = m_tiles * n_tiles;
-  const int kblocks = (K + 63) / 64;
+  const int kblocks = (K + C::BK - 1) / C::BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -70,6 +75,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(TFULL_BAR(a), 1);
       mbar_init(TEMPTY_BAR(a), 256);  // 8 epilogue warps
     }
+    mbar_init(DRAIN_BAR, 1);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -93,6 +99,7 @@ __global__ void __launch_bounds__(320, 1)
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
+      uint32_t armed = 0;  // bit s: stage s has been filled at least once
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m0 = (tile % m_tiles) * 128, n0 = (tile / m_tiles) * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -102,18 +109,25 @@ __global__ void __launch_bounds__(320, 1)
           }
           const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
           mbar_arrive_expect_tx(FULL_BAR(s), C::STAGE_BYTES);
-          tma_load_2d(sa, &tmA, FULL_BAR(s), kb * 64, m0);
-          tma_load_2d(sa + C::A_BYTES, &tmB, FULL_BAR(s), kb * 64, n0);
+          tma_load_2d(sa, &tmA, FULL_BAR(s), kb * C::BK, m0);
+          tma_load_2d(sa + C::A_BYTES, &tmB, FULL_BAR(s), kb * C::BK, n0);
+          armed |= 1u << s;
           if (++s == C::STAGES) {
             s = 0;
             ph ^= 1u;
           }
         }
       }
+      if (!ok) {
+        // a wait ran out: let every copy already issued land before shared memory is
+        // released (the last fill of stage j used parity ph for j < s, ph ^ 1 for j >= s)
+        for (int j = 0; j < C::STAGES; ++j)
+          if (armed & (1u << j)) mbar_wait(FULL_BAR(j), j < s ? ph : ph ^ 1u, ea.status);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---------------- MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+      constexpr uint32_t idesc = C::F8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN);
       int s = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -133,8 +147,12 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(dt, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {  // four 32-byte K steps per 128-byte row
+            if constexpr (C::F8)
+              mma_e4m3_ss(dt, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              mma_bf16_ss(dt, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           mma_commit(EMPTY_BAR(s));
           if (++s == C::STAGES) {
             s = 0;
@@ -142,6 +160,11 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
         if (ok) mma_commit(TFULL_BAR(a));
+      }
+      if (!ok) {
+        // a wait ran out: the MMAs already issued must finish before TMEM is freed
+        mma_commit(DRAIN_BAR);
+        mbar_wait(DRAIN_BAR, 0, ea.status);
       }
     }
   } else {  // ------------------------ epilogue warps 2..9
@@ -156,16 +179,19 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       const int m0 = (tile % m_tiles) * 128, n0 = (tile / m_tiles) * BN;
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a * C::ACC_COLS;
-      if constexpr (EPI == EPI_RESID_T)
-        epilogue_resid_t<BN / 2>(ea, &tmC, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
-                                 staging + (warp - 2) * kStageBytesPerWarp);
+      if constexpr (EPI == EPI_RESID_T || EPI == EPI_RESID_T8)
+        epilogue_resid_t<BN / 2, EPI == EPI_RESID_T8>(ea, &tmC, tacc, m0 + q * 32, lane, n0,
+                                                       ((warp - 2) >> 2) * (BN / 2),
+                                                       staging + (warp - 2) * kStageBytesPerWarp);
+      else if constexpr (EPI == EPI_GELU8)
+        epilogue_gelu8<BN / 2>(ea, tacc, m0 + q * 32 + lane, n0, ((warp - 2) >> 2) * (BN / 2));
       else if constexpr (EPI == EPI_QKV_T)
         epilogue_qkv_t<BN / 2>(ea, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2));
       else if constexpr (epi_staged<EPI>())
         epilogue_cols_staged<BN / 2, EPI>(ea, &tmC, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
                                           staging + (warp - 2) * kStageBytesPerWarp);
       else
-        epilogue_cols<BN / 2, (EPI == EPI_QKV_HEAD ? EPI_QKV : EPI), EPI == EPI_QKV_HEAD>(
+        epilogue_cols<BN / 2, (EPI == EPI_QKV_HEAD ? EPI_QKV : EPI), EPI == EPI_QKV_HEAD || EPI == EPI_XATTN>(
             ea, tacc, m0 + q * 32 + lane, n0, ((warp - 2) >> 2) * (BN / 2));
       tc_fence_before();
       mbar_arrive(TEMPTY_BAR(a));
@@ -183,6 +209,7 @@ __global__ void __launch_bounds__(320, 1)
 #undef EMPTY_BAR
 #undef TFULL_BAR
 #undef TEMPTY_BAR
+#undef DRAIN_BAR
 }
 
 // ------------------------------------------------------------------------- host side
@@ -252,6 +279,10 @@ bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, ui
   return make_tmap_bf16(map, base, rows, K, 64, box_rows, 128);
 }
 
+bool make_tmap_e4m3_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows) {
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, K, 128, box_rows, 128);
+}
+
 template <int BN, int EPI>
 static cudaError_t launch_bn(const CUtensorMap* tA, const CUtensorMap* tB, const CUtensorMap* tC, int K,
                              const EpiArgs& ea, int num_sms, cudaStream_t st) {
@@ -276,7 +307,7 @@ int gemm_tc_supported_bn(int bn) {
 
 cudaError_t launch_gemm_tc(int epi, int bn, const CUtensorMap* tA, const CUtensorMap* tB, int K, const EpiArgs& ea,
                            int num_sms, cudaStream_t st, const CUtensorMap* tC) {
-  if ((epi == EPI_GELU || epi == EPI_RESID_T) && tC == nullptr) return cudaErrorInvalidValue;
+  if ((epi == EPI_GELU || epi == EPI_RESID_T || epi == EPI_RESID_T8) && tC == nullptr) return cudaErrorInvalidValue;
 #define DIT_BN_CASE(BNV, EPIV) \
   if (bn == BNV) return launch_bn<BNV, EPIV>(tA, tB, tC, K, ea, num_sms, st);
   switch (epi) {
@@ -299,6 +330,14 @@ cudaError_t launch_gemm_tc(int epi, int bn, const CUtensorMap* tA, const CUtenso
       DIT_BN_CASE(256, EPI_RESID_T) break;
     case EPI_QKV_T:
       DIT_BN_CASE(256, EPI_QKV_T) break;
+    case EPI_XATTN:
+      DIT_BN_CASE(128, EPI_XATTN) DIT_BN_CASE(144, EPI_XATTN) break;
+    case EPI_F32_8:
+      DIT_BN_CASE(64, EPI_F32_8) DIT_BN_CASE(128, EPI_F32_8) DIT_BN_CASE(256, EPI_F32_8) break;
+    case EPI_GELU8:
+      DIT_BN_CASE(256, EPI_GELU8) break;
+    case EPI_RESID_T8:
+      DIT_BN_CASE(256, EPI_RESID_T8) break;
     default:
       break;
   }

@@ -9,9 +9,9 @@
 // work on the tile, each reading its own A rows and both halves of B, and each SM's
 // TMEM receives its 128 rows of the accumulator.  The MMA completion is committed to
 // the "empty" barrier of both CTAs (the stage may be refilled) and, at the end of a
-// tile, to the "tmem full" barrier of both CTAs (their epilogues may read).  Each
-// CTA's four epilogue warps release the accumulator by arriving on the leader's
-// "tmem empty" barrier.  Per SM and stage this moves 16 KB of A and BN*64 bytes of B
+// tile, to the "tmem full" barrier of both CTAs (their epilogues may read), one commit
+// per CTA.  Each CTA's eight epilogue warps release the accumulator by arriving on the
+// leader's "tmem empty" barrier.  Per SM and stage this moves 16 KB of A and BN*64 bytes of B
 // for 128 x BN x 64 multiply-adds, half the B traffic of a one-SM tile.
 // Persistent: one cluster per SM pair, tiles strided over clusters, two TMEM
 // accumulators so the epilogue of one tile overlaps the main loop of the next.
@@ -152,13 +152,17 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_bf16_pair(dt, sdesc_k_sw128(sa + k * 32), sdesc_k_sw128(sb + k * 32), idesc, (kb | k) != 0 ? 1u : 0u);
-          mma_commit_pair(EMPTY_BAR(s), 0x3);
+          mma_commit_pair(EMPTY_BAR(s));
+          mma_commit_pair(mapa_shared(EMPTY_BAR(s), 1));
           if (++s == C::STAGES) {
             s = 0;
             ph ^= 1u;
           }
         }
-        if (ok) mma_commit_pair(TFULL_BAR(a), 0x3);
+        if (ok) {
+          mma_commit_pair(TFULL_BAR(a));
+          mma_commit_pair(mapa_shared(TFULL_BAR(a), 1));
+        }
       }
       // accumulator tail: every epilogue release (including the partner CTA's remote
       // arrivals) has landed before this CTA may leave
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(320, 1)
         epilogue_cols_staged<BN / 2, EPI>(ea, &tmC, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
                                           staging + (warp - 2) * kStageBytesPerWarp);
       else
-        epilogue_cols<BN / 2, (EPI == EPI_QKV_HEAD ? EPI_QKV : EPI), EPI == EPI_QKV_HEAD>(
+        epilogue_cols<BN / 2, (EPI == EPI_QKV_HEAD ? EPI_QKV : EPI), EPI == EPI_QKV_HEAD || EPI == EPI_XATTN>(
             ea, tacc, m0 + q * 32 + lane, n0, ((warp - 2) >> 2) * (BN / 2));
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(TEMPTY_BAR(a), 0));

@@ -20,7 +20,20 @@ enum Epi : int {
   // GEMM columns are tokens; ea.M = features, ea.N = tokens):
   EPI_RESID_T = 6,   // h[tok, f] += gate[row(tok), f] * (acc + bias[f])   (TMA reduce-add)
   EPI_QKV_T = 7,     // q, k, v^T scatter, column by column
+  // Cross-attention onto a two-token condition sequence, fused into the query projection:
+  // tile = 2 heads; each thread holds one token's query for one head, scores it against the
+  // two keys, and writes the softmax mix of the two values to o [M, d] (bf16).
+  EPI_XATTN = 8,
+  // FP8 E4M3 operands (kind::f8f6f4): the accumulator is scaled by the per-row scale sa[m] of
+  // the A operand and the per-column scale sb[n] of the B operand before the epilogue proper.
+  EPI_F32_8 = 9,     // out[m, n] = sa[m] sb[n] acc + bias[n]                  (float32)
+  EPI_GELU8 = 10,    // g = gelu(sa[m] sb[n] acc + bias[n]) stored as E4M3 g / sg[m] (bytes [M, ldo])
+  EPI_RESID_T8 = 11, // swapped: h[tok, f] += gate * (sa[f] sb[tok] acc + bias[f]) (TMA reduce-add)
 };
+template <int EPI>
+__host__ __device__ constexpr bool epi_fp8() {
+  return EPI == EPI_F32_8 || EPI == EPI_GELU8 || EPI == EPI_RESID_T8;
+}
 
 struct EpiArgs {
   int M, N;             // logical output extent (rows of A, rows of B)
@@ -41,6 +54,15 @@ struct EpiArgs {
   const float* qn;      // [dh] RMSNorm gains or nullptr
   const float* kn;
   const float* rope;    // [T, dh/2, 2] (cos, sin) or nullptr
+  // EPI_XATTN: keys and values of the condition tokens of row r at
+  // xkv + (2r + s) * ld_xkv + {0: k, d: v} + head * dh (s = 0, 1), float32
+  const float* xkv;
+  int ld_xkv;
+  void* xo;             // bf16 [M, d] attention output
+  // FP8 operand scales (per A row, per B row) and the E4M3 output scale of EPI_GELU8
+  const float* sa;
+  const float* sb;
+  const float* sg;
   int* status;
 };
 
@@ -69,6 +91,8 @@ inline int current_device() {
   return dev;
 }
 bool make_tmap_bf16_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
+// FP8 (one byte per element) K-major map: rows x K, box = box_rows x 128, 128-byte swizzle.
+bool make_tmap_e4m3_kmajor(CUtensorMap* map, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows);
 // 3-d bf16 map: dims d0 (innermost) x d1 x d2, box box0 x box1 x 1, 128B swizzle or none.
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
                        uint32_t box1, int swizzle_bytes);
@@ -95,26 +119,41 @@ struct CondArgs {
   float* E;              // scratch [R, freq]
   float* hid;            // scratch [R, d]
   float* c;              // [R, d]   (optional, may be null)
-  void* sc;              // SiLU(c): bf16 [*, d] or f32 [R, d]
+  void* sc;              // SiLU(c): bf16 [*, d] or f32 [R, d] (optional, may be null)
   int sc_bf16;
   int* status;
+  // the two condition embeddings e_t (timestep MLP) and e_y (label row / text vector) as
+  // tokens: in the residual stream at tok_h + r * tok_ld (e_t) and + d (e_y), and / or as
+  // rows 2r, 2r + 1 of a condition sequence ctx [2R, d] (bf16 or f32)
+  float* tok_h = nullptr;
+  size_t tok_ld = 0;
+  void* ctx = nullptr;
+  int ctx_bf16 = 0;
 };
 cudaError_t launch_condition(const CondArgs& a, cudaStream_t st);
 
 struct PatchArgs {
   const float* x;        // [B, C, F, H, W]
   const float* w;        // [d, Kp]
+  const float* wt;       // the same weights transposed, [Kp, d]
   const float* b;        // [d]
   const float* pos;      // [T, d] or nullptr
-  float* h;              // [R*T, d]
+  float* h;              // [R*Trow, d]: patch token tau of row r at row r * Trow + tok0 + tau
   int B, R, C, F, H, W, pt, ph, pw, d;
+  int Trow = 0, tok0 = 0;  // tokens per row in h (0: the patch count) and the first patch token
 };
 cudaError_t launch_patch_embed(const PatchArgs& a, cudaStream_t st);
 
 struct LnArgs {
   const float* h;        // [M, d]
-  void* u;               // bf16 or f32 [M, d]
+  void* u;               // bf16 or f32 [M, d] (E4M3 bytes when u8 is set)
   int u_bf16;
+  // FP8 output: u as E4M3 with a per-row scale su[m] = amax_m / 448, and the per-row scale
+  // sg[m] = (||u_m||_2 * g_w + g_b) / 448 of the next matmul's GELU output (a bound on it)
+  uint8_t* u8 = nullptr;
+  float* su = nullptr;
+  float* sg = nullptr;
+  float g_w = 0.f, g_b = 0.f;
   const float* shift;    // row r vector at shift + r * ld_mod
   const float* scale;
   int ld_mod;
@@ -147,17 +186,20 @@ struct QkNormArgs {   // f32 path: RMSNorm + RoPE applied in place to q, k [R*H,
 };
 cudaError_t launch_qknorm_rope_f32(const QkNormArgs& a, cudaStream_t st);
 
-struct DecodeArgs {
-  const void* u;         // [R*T, d] bf16 or f32
-  int u_bf16;
-  const float* w;        // [P, d]
-  const float* b;        // [P]
+// Classifier-free guidance combine and unpatchify of the decoder output z:
+// out[b, c, f*pt+it, i*ph+ih, j*pw+iw] = z_null + s (z_cond - z_null) at token (f, i, j) and
+// vector index ((it*ph + ih)*pw + iw)*Cout + c (z_cond alone when not guided, and on channels
+// c >= gch when gch > 0).
+struct UnpatchArgs {
+  const float* z;        // [R*Trow, P], rows [cond; uncond] when guided; patch token tau of row r
+                         // at row r * Trow + tok0 + tau
   float* out;            // [B, Cout, F, H, W]
-  int B, T, d, P, Cout, F, H, W, pt, ph, pw, guided;
+  int B, T, P, Cout, F, H, W, pt, ph, pw, guided;
   int gch;               // guided channels: c < gch are guided, the rest keep z_cond (0: all)
   float s;
+  int Trow = 0, tok0 = 0;
 };
-cudaError_t launch_decode_cfg(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_cfg_unpatchify(const UnpatchArgs& a, int num_sms, cudaStream_t st);
 
 // Sampler update x_next = c0 * x + c1 * pred, pred = the first n_sample values of each
 // sample's ld_pred-long block of the denoiser output (its first C channels).
@@ -171,8 +213,26 @@ struct SamplerArgs {
 };
 cudaError_t launch_sampler_step(const SamplerArgs& a, int num_sms, cudaStream_t st);
 
-cudaError_t launch_pos_tables(float* pos, float* rope, int gf, int gh, int gw, int d, int dh, cudaStream_t st);
+// rope rows tok0 .. tok0 + gf*gh*gw - 1 hold the patch tokens' rotations; rows < tok0
+// (condition tokens) the identity (cos 1, sin 0)
+cudaError_t launch_pos_tables(float* pos, float* rope, int gf, int gh, int gw, int d, int dh, int tok0,
+                              cudaStream_t st);
+
+// float32 cross-attention onto the two condition tokens (the fp32 path's unfused form of
+// EPI_XATTN): o[m, head] = softmax over s of q[m, head] . k_s / sqrt(dh), mixing v_s.
+struct XAttnArgs {
+  const float* q;        // [M, d]
+  const float* xkv;      // as EpiArgs::xkv
+  int ld_xkv;
+  float* o;              // [M, d]
+  int M, T, d, H, dh;
+};
+cudaError_t launch_xattn_f32(const XAttnArgs& a, cudaStream_t st);
 cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaStream_t st);
+// Row-wise E4M3 quantisation of a float32 matrix [rows, cols]: scale[r] = amax_r / 448 (1 for a
+// zero row), dst[r, c] = E4M3(src[r, c] / scale[r]).
+cudaError_t launch_quantize_rows_e4m3(const float* src, uint8_t* dst, float* scale, int rows, int cols,
+                                      cudaStream_t st);
 cudaError_t launch_wait_probe(int* flag, int* status, long long limit_ns, cudaStream_t st);
 
 }  // namespace dit

@@ -1,6 +1,6 @@
 // CUDA-core kernels of the DiT forward: condition MLP, patch embedding, fused
-// LayerNorm + modulate, the float32 GEMM / attention of the fp32 path, the decoder
-// fused with unpatchify and classifier-free guidance, and set-up tables.
+// LayerNorm + modulate, the float32 GEMM / attention of the fp32 path, classifier-free
+// guidance fused with unpatchify, and set-up tables.
 #include <math.h>
 
 #include "common.cuh"
@@ -28,88 +28,111 @@ __global__ void cond_sinusoid_kernel(const float* __restrict__ t, int B, int R, 
   }
 }
 
-// out[r, j] = act(sum_i W[j, i] in[r, i] + b[j]) (+ e(y_r) for the condition's second
-// layer).  One warp per (output feature j, group of kRowsPerWarp rows): lanes split the
-// K-long dot products, so the weight row is read once per row group.
-constexpr int kRowsPerWarp = 8;
+// The condition MLP's two layers, out[r, j] = W[j] . in[r] + b[j] for all sample rows r:
+// a block of 8 warps owns 8 output features (one per warp) and a group of up to 32 rows
+// (lane = row).  The rows' inputs are staged in shared memory in K-chunks of 128, read once
+// per block; each lane loads 32 consecutive weights of its warp's feature at a time and hands
+// them round with shuffles, so a multiply-add costs a shuffle, a shared load and an FMA.
+constexpr int kCondK = 128;  // K-chunk staged per pass
+constexpr int kCondRows = 32;
 
-__device__ __forceinline__ void rows_dot(const float* __restrict__ w, const float* __restrict__ in, int K, int r0,
-                                         int nr, int lane, float (&acc)[kRowsPerWarp]) {
+__device__ __forceinline__ float cond_dot(const float* __restrict__ w, const float* __restrict__ in, int K, int r0,
+                                          int nr, float* stage, int lane) {
+  float acc = 0.f;
+  for (int k0 = 0; k0 < K; k0 += kCondK) {
+    const int kn = min(kCondK, K - k0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nr * kn; i += blockDim.x) {
+      const int rr = i / kn, kk = i - rr * kn;
+      stage[rr * (kCondK + 1) + kk] = in[static_cast<size_t>(r0 + rr) * K + k0 + kk];
+    }
+    __syncthreads();
+    for (int kb = 0; kb < kn; kb += 32) {
+      const float wl = kb + lane < kn ? __ldg(w + k0 + kb + lane) : 0.f;
+      const float* srow = stage + lane * (kCondK + 1) + kb;
+      const int kc = min(32, kn - kb);
+      if (kc == 32) {
 #pragma unroll
-  for (int q = 0; q < kRowsPerWarp; ++q) acc[q] = 0.f;
-  for (int i = lane; i < K; i += 32) {
-    const float wi = __ldg(w + i);
-#pragma unroll
-    for (int q = 0; q < kRowsPerWarp; ++q)
-      if (q < nr) acc[q] = fmaf(wi, in[static_cast<size_t>(r0 + q) * K + i], acc[q]);
-  }
-#pragma unroll
-  for (int q = 0; q < kRowsPerWarp; ++q) acc[q] = warp_sum(acc[q]);
-}
-
-template <bool SILU>
-__global__ void rows_linear_kernel(const float* __restrict__ in, const float* __restrict__ W,
-                                   const float* __restrict__ b, float* __restrict__ out, int R, int K, int N) {
-  pdl_trigger();
-  pdl_wait();
-  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const int groups = (R + kRowsPerWarp - 1) / kRowsPerWarp;
-  if (gw >= N * groups) return;
-  const int j = gw / groups, r0 = (gw - j * groups) * kRowsPerWarp;
-  const int nr = min(kRowsPerWarp, R - r0);
-  float acc[kRowsPerWarp];
-  rows_dot(W + static_cast<size_t>(j) * K, in, K, r0, nr, lane, acc);
-  if (lane == 0) {
-#pragma unroll
-    for (int q = 0; q < kRowsPerWarp; ++q)
-      if (q < nr) {
-        const float v = acc[q] + b[j];
-        out[static_cast<size_t>(r0 + q) * N + j] = SILU ? silu_f(v) : v;
-      }
-  }
-}
-
-// c[r, j] = W2 hid[r] + b2 + e(y_r);  sc = SiLU(c) (bf16 or f32).
-// Rows r >= B of a guided batch take the null label num_classes.
-__global__ void cond_out_kernel(CondArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const int groups = (a.R + kRowsPerWarp - 1) / kRowsPerWarp;
-  if (gw >= a.d * groups) return;
-  const int j = gw / groups, r0 = (gw - j * groups) * kRowsPerWarp;
-  const int nr = min(kRowsPerWarp, a.R - r0);
-  float acc[kRowsPerWarp];
-  rows_dot(a.w2 + static_cast<size_t>(j) * a.d, a.hid, a.d, r0, nr, lane, acc);
-  if (lane == 0) {
-#pragma unroll
-    for (int q = 0; q < kRowsPerWarp; ++q) {
-      if (q >= nr) continue;
-      const int r = r0 + q;
-      float v = acc[q] + a.b2[j];
-      if (a.cond_kind == DIT_COND_CLASS) {
-        int lab;
-        if (r < a.B) {
-          lab = static_cast<const int*>(a.y)[r];
-          if (lab < 0 || lab > a.num_classes) {
-            record_status(a.status, DIT_ERR_BAD_LABEL);
-            lab = lab < 0 ? 0 : a.num_classes;
-          }
-        } else {
-          lab = a.num_classes;
-        }
-        v += a.table[static_cast<size_t>(lab) * a.d + j];
+        for (int q = 0; q < 32; ++q) acc = fmaf(__shfl_sync(0xffffffffu, wl, q), srow[q], acc);
       } else {
-        v += static_cast<const float*>(a.y)[static_cast<size_t>(r % a.B) * a.d + j];
+        for (int q = 0; q < kc; ++q) acc = fmaf(__shfl_sync(0xffffffffu, wl, q), srow[q], acc);
       }
-      if (a.c) a.c[static_cast<size_t>(r) * a.d + j] = v;
+    }
+  }
+  return acc;
+}
+
+// hid[r, j] = SiLU(W1[j] . E[r] + b1[j])
+__global__ void __launch_bounds__(256) cond_hidden_kernel(const float* __restrict__ E, const float* __restrict__ W1,
+                                                          const float* __restrict__ b1, float* __restrict__ hid, int R,
+                                                          int K, int N) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float stage[kCondRows * (kCondK + 1)];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * 8 + warp;
+  const int jc = j < N ? j : N - 1;  // every warp takes part in the block's staging barriers
+  for (int r0 = blockIdx.y * kCondRows; r0 < R; r0 += gridDim.y * kCondRows) {
+    const int nr = min(kCondRows, R - r0);
+    const float v = cond_dot(W1 + static_cast<size_t>(jc) * K, E, K, r0, nr, stage, lane);
+    if (j < N && lane < nr) hid[static_cast<size_t>(r0 + lane) * N + j] = silu_f(v + b1[j]);
+  }
+}
+
+// c[r, j] = e_t + e_y with e_t = W2[j] . hid[r] + b2[j] and e_y = e(y_r);  sc = SiLU(c) (bf16
+// or f32); optionally e_t and e_y as condition tokens.  Rows r >= B of a guided batch take the
+// null label num_classes.
+__global__ void __launch_bounds__(256) cond_out_kernel(CondArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float stage[kCondRows * (kCondK + 1)];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * 8 + warp;
+  const int jc = j < a.d ? j : a.d - 1;
+  for (int r0 = blockIdx.y * kCondRows; r0 < a.R; r0 += gridDim.y * kCondRows) {
+    const int nr = min(kCondRows, a.R - r0);
+    const float acc = cond_dot(a.w2 + static_cast<size_t>(jc) * a.d, a.hid, a.d, r0, nr, stage, lane);
+    if (j >= a.d || lane >= nr) continue;
+    const int r = r0 + lane;
+    const float et = acc + a.b2[j];  // timestep embedding
+    float ey;                        // class embedding / text vector
+    if (a.cond_kind == DIT_COND_CLASS) {
+      int lab;
+      if (r < a.B) {
+        lab = static_cast<const int*>(a.y)[r];
+        if (lab < 0 || lab > a.num_classes) {
+          record_status(a.status, DIT_ERR_BAD_LABEL);
+          lab = lab < 0 ? 0 : a.num_classes;
+        }
+      } else {
+        lab = a.num_classes;
+      }
+      ey = a.table[static_cast<size_t>(lab) * a.d + j];
+    } else {
+      ey = static_cast<const float*>(a.y)[static_cast<size_t>(r % a.B) * a.d + j];
+    }
+    const float v = et + ey;
+    if (a.c) a.c[static_cast<size_t>(r) * a.d + j] = v;
+    if (a.sc) {
       const float sv = silu_f(v);
       if (a.sc_bf16)
         static_cast<uint16_t*>(a.sc)[static_cast<size_t>(r) * a.d + j] = f32_to_bf16(sv);
       else
         static_cast<float*>(a.sc)[static_cast<size_t>(r) * a.d + j] = sv;
+    }
+    if (a.tok_h) {
+      a.tok_h[r * a.tok_ld + j] = et;
+      a.tok_h[r * a.tok_ld + a.d + j] = ey;
+    }
+    if (a.ctx) {
+      const size_t i0 = static_cast<size_t>(2 * r) * a.d + j, i1 = i0 + a.d;
+      if (a.ctx_bf16) {
+        static_cast<uint16_t*>(a.ctx)[i0] = f32_to_bf16(et);
+        static_cast<uint16_t*>(a.ctx)[i1] = f32_to_bf16(ey);
+      } else {
+        static_cast<float*>(a.ctx)[i0] = et;
+        static_cast<float*>(a.ctx)[i1] = ey;
+      }
     }
   }
 }
@@ -119,12 +142,11 @@ cudaError_t launch_condition(const CondArgs& a, cudaStream_t st) {
   cudaError_t e = launch_kernel(cond_sinusoid_kernel, dim3((n + 255) / 256), dim3(256), 0, st, a.t, a.B, a.R, a.freq,
                                  a.t_scale, a.E);
   if (e != cudaSuccess) return e;
-  const int groups = (a.R + kRowsPerWarp - 1) / kRowsPerWarp;
-  const int warps = a.d * groups;
-  e = launch_kernel(rows_linear_kernel<true>, dim3((warps + 7) / 8), dim3(256), 0, st, (const float*)a.E, a.w1, a.b1,
+  const int rg = (a.R + kCondRows - 1) / kCondRows;
+  e = launch_kernel(cond_hidden_kernel, dim3((a.d + 7) / 8, rg), dim3(256), 0, st, (const float*)a.E, a.w1, a.b1,
                     a.hid, a.R, a.freq, a.d);
   if (e != cudaSuccess) return e;
-  return launch_kernel(cond_out_kernel, dim3((warps + 7) / 8), dim3(256), 0, st, a);
+  return launch_kernel(cond_out_kernel, dim3((a.d + 7) / 8, rg), dim3(256), 0, st, a);
 }
 
 // ============================================================================ patch embed
@@ -166,7 +188,110 @@ __global__ void patch_embed_kernel(PatchArgs a) {
     for (int t = 0; t < ntok; ++t) {
       float v = acc[t] + bj;
       if (a.pos) v += a.pos[static_cast<size_t>(tau0 + t) * a.d + j];
-      a.h[(static_cast<size_t>(r) * T + tau0 + t) * a.d + j] = v;
+      a.h[(static_cast<size_t>(r) * (a.Trow ? a.Trow : T) + a.tok0 + tau0 + t) * a.d + j] = v;
+    }
+  }
+}
+
+// Fast path (Kp <= 256, d <= 1536, d % 4 == 0): one warp per pair of tokens of the B unique
+// samples.  Lane l holds patch elements l, l+32, ... of both tokens and broadcasts them with
+// shuffles; it accumulates output features 4(l + 32i) .. +3 from the transposed weights
+// [Kp, d] (coalesced 16-byte loads, shared by the two tokens), then adds bias and position
+// and stores whole 16-byte groups to row b and, when guided, to row B + b as well.
+constexpr int kPeMaxVec = 12;   // float4 groups per lane: d <= 32 * 4 * 12 = 1536
+constexpr int kPeMaxKv = 8;     // patch elements per lane: Kp <= 256
+__global__ void __launch_bounds__(256) patch_embed_pairs_kernel(PatchArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int gh = a.H / a.ph, gw = a.W / a.pw, gf = a.F / a.pt;
+  const int T = gf * gh * gw;
+  const int Kp = a.C * a.pt * a.ph * a.pw;
+  const int lane = threadIdx.x & 31;
+  const int nvec = (a.d + 127) / 128;
+  const long long units = static_cast<long long>(a.B) * T;  // unique tokens
+  const long long pairs = (units + 1) / 2;
+  const long long gwarp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long pr = gwarp; pr < pairs; pr += nwarps) {
+    float xv[2][kPeMaxKv];
+    int tb[2], ttau[2];
+    bool live[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const long long id = 2 * pr + u;
+      live[u] = id < units;
+      const long long idc = live[u] ? id : units - 1;
+      tb[u] = static_cast<int>(idc / T);
+      ttau[u] = static_cast<int>(idc - static_cast<long long>(tb[u]) * T);
+      const int f = ttau[u] / (gh * gw), i = (ttau[u] / gw) % gh, jj = ttau[u] % gw;
+#pragma unroll
+      for (int kk = 0; kk < kPeMaxKv; ++kk) {
+        const int k = kk * 32 + lane;
+        float v = 0.f;
+        if (k < Kp) {
+          const int iw = k % a.pw, ih = (k / a.pw) % a.ph, it = (k / (a.pw * a.ph)) % a.pt, c = k / (a.pw * a.ph * a.pt);
+          const size_t xi = ((((static_cast<size_t>(tb[u]) * a.C + c) * a.F + f * a.pt + it) * a.H + i * a.ph + ih) *
+                             a.W) + jj * a.pw + iw;
+          v = __ldg(a.x + xi);
+        }
+        xv[u][kk] = v;
+      }
+    }
+    float4 acc[2][kPeMaxVec];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int i = 0; i < kPeMaxVec; ++i) acc[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int kk = 0; kk < kPeMaxKv; ++kk) {
+      if (kk * 32 >= Kp) break;
+      const int kn = min(32, Kp - kk * 32);
+      for (int kl = 0; kl < kn; ++kl) {
+        const float x0 = __shfl_sync(0xffffffffu, xv[0][kk], kl);
+        const float x1 = __shfl_sync(0xffffffffu, xv[1][kk], kl);
+        const float4* wr = reinterpret_cast<const float4*>(a.wt + static_cast<size_t>(kk * 32 + kl) * a.d);
+#pragma unroll
+        for (int i = 0; i < kPeMaxVec; ++i) {
+          const int c4 = lane + 32 * i;
+          if (i < nvec && 4 * c4 < a.d) {
+            const float4 w = __ldg(wr + c4);
+            acc[0][i].x = fmaf(x0, w.x, acc[0][i].x);
+            acc[0][i].y = fmaf(x0, w.y, acc[0][i].y);
+            acc[0][i].z = fmaf(x0, w.z, acc[0][i].z);
+            acc[0][i].w = fmaf(x0, w.w, acc[0][i].w);
+            acc[1][i].x = fmaf(x1, w.x, acc[1][i].x);
+            acc[1][i].y = fmaf(x1, w.y, acc[1][i].y);
+            acc[1][i].z = fmaf(x1, w.z, acc[1][i].z);
+            acc[1][i].w = fmaf(x1, w.w, acc[1][i].w);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!live[u]) continue;
+      const float4* pos = a.pos ? reinterpret_cast<const float4*>(a.pos + static_cast<size_t>(ttau[u]) * a.d) : nullptr;
+      const int Tr = a.Trow ? a.Trow : T;
+      float4* h0 = reinterpret_cast<float4*>(a.h + (static_cast<size_t>(tb[u]) * Tr + a.tok0 + ttau[u]) * a.d);
+      float4* h1 = reinterpret_cast<float4*>(a.h + (static_cast<size_t>(tb[u] + a.B) * Tr + a.tok0 + ttau[u]) * a.d);
+      const bool dup = a.R > a.B;
+#pragma unroll
+      for (int i = 0; i < kPeMaxVec; ++i) {
+        const int c4 = lane + 32 * i;
+        if (i < nvec && 4 * c4 < a.d) {
+          const float4 bb = __ldg(reinterpret_cast<const float4*>(a.b) + c4);
+          float4 v = make_float4(acc[u][i].x + bb.x, acc[u][i].y + bb.y, acc[u][i].z + bb.z, acc[u][i].w + bb.w);
+          if (pos) {
+            const float4 pp = __ldg(pos + c4);
+            v.x += pp.x;
+            v.y += pp.y;
+            v.z += pp.z;
+            v.w += pp.w;
+          }
+          h0[c4] = v;
+          if (dup) h1[c4] = v;
+        }
+      }
     }
   }
 }
@@ -174,6 +299,13 @@ __global__ void patch_embed_kernel(PatchArgs a) {
 cudaError_t launch_patch_embed(const PatchArgs& a, cudaStream_t st) {
   const int T = (a.F / a.pt) * (a.H / a.ph) * (a.W / a.pw);
   const int Kp = a.C * a.pt * a.ph * a.pw;
+  if (a.wt != nullptr && Kp <= 32 * kPeMaxKv && a.d <= 128 * kPeMaxVec && (a.d & 3) == 0 && (a.R == a.B || a.R == 2 * a.B)) {
+    const long long pairs = (static_cast<long long>(a.B) * T + 1) / 2;
+    const long long blocks = (pairs + 7) / 8;
+    const int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
+    if (grid == 0) return cudaSuccess;
+    return launch_kernel(patch_embed_pairs_kernel, dim3(grid), dim3(256), 0, st, a);
+  }
   const size_t smem = static_cast<size_t>(kPatchTok) * Kp * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(patch_embed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -186,32 +318,78 @@ cudaError_t launch_patch_embed(const PatchArgs& a, cudaStream_t st) {
 
 // ============================================================================ LN + modulate
 // u = (h - mean) / sqrt(var + 1e-6) * (1 + scale[r]) + shift[r]  (population variance).
-// One warp per token row, four rows per 128-thread block: the row's float4 loads are
-// all issued before any use, mean and variance are two exact passes over registers,
-// and u leaves as 8-byte (bf16) or 16-byte (f32) stores.  The pass is bound by the
-// memory system: 6 bytes per element for the bf16 output.
-constexpr int kLnMaxVec = 12;  // d <= 1536 (float4 per lane)
-constexpr int kLnRowsPerBlock = 4;
+// A block of 256 threads owns 32 consecutive token rows, so its rows come from at most two
+// sample rows r (when T >= 32); the (shift, scale) vectors of those are staged once in shared
+// memory instead of being re-read for every token.  Each warp normalises 4 rows, two at a
+// time: both rows' float4 loads are in flight before any use, mean and variance are two
+// exact passes over registers, and u leaves as 8-byte (bf16), 16-byte (f32) or 4-byte (E4M3)
+// stores per lane.  Bound by the memory system: 6 bytes per element for the bf16 output.
+constexpr int kLnMaxVec = 12;   // d <= 1536 (float4 per lane)
+constexpr int kLnRows = 32;     // token rows per block
+constexpr int kLnThreads = 256;
 
-template <bool BF16OUT>
-__global__ void __launch_bounds__(32 * kLnRowsPerBlock) ln_modulate_kernel(LnArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  const int m = blockIdx.x * kLnRowsPerBlock + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (m >= a.M) return;
-  const int nv = a.d >> 2;
-  const float4* hp = reinterpret_cast<const float4*>(a.h + static_cast<size_t>(m) * a.d);
-  float4 x[kLnMaxVec];
+// Writes the modulated row; the normalised values replace x (the E4M3 output needs them twice).
+template <int OUT>
+__device__ __forceinline__ void ln_store_row(const LnArgs& a, int m, int lane, int nv, float4 (&x)[kLnMaxVec],
+                                             float mean, float rstd, const float* sh, const float* sc) {
+  float amax = 0.f, ss = 0.f;
+  float4(&o)[kLnMaxVec] = x;
+#pragma unroll
+  for (int k = 0; k < kLnMaxVec; ++k) {
+    const int c = lane + 32 * k;
+    if (c < nv) {
+      const float4 s4 = reinterpret_cast<const float4*>(sc)[c], b4 = reinterpret_cast<const float4*>(sh)[c];
+      o[k].x = (x[k].x - mean) * rstd * (1.f + s4.x) + b4.x;
+      o[k].y = (x[k].y - mean) * rstd * (1.f + s4.y) + b4.y;
+      o[k].z = (x[k].z - mean) * rstd * (1.f + s4.z) + b4.z;
+      o[k].w = (x[k].w - mean) * rstd * (1.f + s4.w) + b4.w;
+      if (OUT == 1) {
+        uint2 p;
+        p.x = pack_bf16x2(o[k].x, o[k].y);
+        p.y = pack_bf16x2(o[k].z, o[k].w);
+        reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.u) + static_cast<size_t>(m) * a.d)[c] = p;
+      } else if (OUT == 0) {
+        reinterpret_cast<float4*>(static_cast<float*>(a.u) + static_cast<size_t>(m) * a.d)[c] = o[k];
+      } else {
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(o[k].x), fabsf(o[k].y)), fmaxf(fabsf(o[k].z), fabsf(o[k].w))));
+        ss += (o[k].x * o[k].x + o[k].y * o[k].y) + (o[k].z * o[k].z + o[k].w * o[k].w);
+      }
+    }
+  }
+  if (OUT == 2) {  // E4M3 with the row's scale, and the bound-based scale of the next GELU output
+    amax = warp_max(amax);
+    ss = warp_sum(ss);
+    const float su = amax > 0.f ? amax * (1.0f / 448.0f) : 1.0f;
+    const float bound = sqrtf(ss) * a.g_w + a.g_b;
+    const float inv = 1.0f / su;
+    if (lane == 0) {
+      a.su[m] = su;
+      a.sg[m] = bound > 0.f ? bound * (1.0f / 448.0f) : 1.0f;
+    }
+    uint32_t* u8 = reinterpret_cast<uint32_t*>(a.u8 + static_cast<size_t>(m) * a.d);
+#pragma unroll
+    for (int k = 0; k < kLnMaxVec; ++k) {
+      const int c = lane + 32 * k;
+      if (c < nv) u8[c] = pack_e4m3x4(o[k].x * inv, o[k].y * inv, o[k].z * inv, o[k].w * inv);
+    }
+  }
+}
+
+__device__ __forceinline__ void ln_load_row(const float* h, int d, int lane, int nv, float4 (&x)[kLnMaxVec]) {
+  const float4* hp = reinterpret_cast<const float4*>(h);
 #pragma unroll
   for (int k = 0; k < kLnMaxVec; ++k) {
     const int c = lane + 32 * k;
     x[k] = c < nv ? hp[c] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+}
+
+__device__ __forceinline__ void ln_stats(const float4 (&x)[kLnMaxVec], int lane, int nv, int d, float& mean,
+                                         float& rstd) {
   float sum = 0.f;
 #pragma unroll
   for (int k = 0; k < kLnMaxVec; ++k) sum += (x[k].x + x[k].y) + (x[k].z + x[k].w);
-  const float mean = warp_sum(sum) / a.d;
+  mean = warp_sum(sum) / d;
   float q = 0.f;
 #pragma unroll
   for (int k = 0; k < kLnMaxVec; ++k) {
@@ -221,39 +399,67 @@ __global__ void __launch_bounds__(32 * kLnRowsPerBlock) ln_modulate_kernel(LnArg
       q += (dx * dx + dy * dy) + (dz * dz + dw * dw);
     }
   }
-  const float rstd = rsqrtf(warp_sum(q) / a.d + 1e-6f);
-  const int r = m / a.T;
-  const float4* sh = reinterpret_cast<const float4*>(a.shift + static_cast<size_t>(r) * a.ld_mod);
-  const float4* sc = reinterpret_cast<const float4*>(a.scale + static_cast<size_t>(r) * a.ld_mod);
-#pragma unroll
-  for (int k = 0; k < kLnMaxVec; ++k) {
-    const int c = lane + 32 * k;
-    if (c < nv) {
-      const float4 s4 = __ldg(sc + c), b4 = __ldg(sh + c);
-      float4 o;
-      o.x = (x[k].x - mean) * rstd * (1.f + s4.x) + b4.x;
-      o.y = (x[k].y - mean) * rstd * (1.f + s4.y) + b4.y;
-      o.z = (x[k].z - mean) * rstd * (1.f + s4.z) + b4.z;
-      o.w = (x[k].w - mean) * rstd * (1.f + s4.w) + b4.w;
-      if (BF16OUT) {
-        uint2 p;
-        p.x = pack_bf16x2(o.x, o.y);
-        p.y = pack_bf16x2(o.z, o.w);
-        reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.u) + static_cast<size_t>(m) * a.d)[c] = p;
-      } else {
-        reinterpret_cast<float4*>(static_cast<float*>(a.u) + static_cast<size_t>(m) * a.d)[c] = o;
-      }
+  rstd = rsqrtf(warp_sum(q) / d + 1e-6f);
+}
+
+// OUT: 0 float32, 1 bf16, 2 FP8 E4M3 with the row's scales (see LnArgs).
+template <int OUT>
+__global__ void __launch_bounds__(kLnThreads) ln_modulate_kernel(LnArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ float ln_mod[];  // [2 sample rows][shift | scale][d]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nv = a.d >> 2;
+  const int m0 = blockIdx.x * kLnRows;
+  // sample rows of this block's first and last token rows; staged when at most two
+  const int rfirst = a.ld_mod ? m0 / a.T : 0;
+  const int rlast = a.ld_mod ? min(m0 + kLnRows - 1, a.M - 1) / a.T : 0;
+  const bool staged = rlast - rfirst <= 1;
+  if (staged) {
+    for (int i = threadIdx.x; i < (rlast - rfirst + 1) * nv; i += blockDim.x) {
+      const int j = i / nv, c = i - j * nv;
+      const size_t off = static_cast<size_t>(rfirst + j) * a.ld_mod;
+      reinterpret_cast<float4*>(ln_mod + (2 * j) * a.d)[c] = __ldg(reinterpret_cast<const float4*>(a.shift + off) + c);
+      reinterpret_cast<float4*>(ln_mod + (2 * j + 1) * a.d)[c] = __ldg(reinterpret_cast<const float4*>(a.scale + off) + c);
+    }
+  }
+  __syncthreads();
+  for (int pr = 0; pr < kLnRows / 8; pr += 2) {  // each warp: rows m0 + 4 warp + {0, 1}, then {2, 3}
+    const int ma = m0 + warp * (kLnRows / 8) + pr, mb = ma + 1;
+    if (ma >= a.M) break;
+    float4 xa[kLnMaxVec], xb[kLnMaxVec];
+    ln_load_row(a.h + static_cast<size_t>(ma) * a.d, a.d, lane, nv, xa);
+    const bool hb = mb < a.M;
+    if (hb) ln_load_row(a.h + static_cast<size_t>(mb) * a.d, a.d, lane, nv, xb);
+    float mean, rstd;
+    ln_stats(xa, lane, nv, a.d, mean, rstd);
+    {
+      const int r = a.ld_mod ? ma / a.T : 0;
+      const float* sh = staged ? ln_mod + 2 * (r - rfirst) * a.d : a.shift + static_cast<size_t>(r) * a.ld_mod;
+      const float* sc = staged ? ln_mod + (2 * (r - rfirst) + 1) * a.d : a.scale + static_cast<size_t>(r) * a.ld_mod;
+      ln_store_row<OUT>(a, ma, lane, nv, xa, mean, rstd, sh, sc);
+    }
+    if (hb) {
+      ln_stats(xb, lane, nv, a.d, mean, rstd);
+      const int r = a.ld_mod ? mb / a.T : 0;
+      const float* sh = staged ? ln_mod + 2 * (r - rfirst) * a.d : a.shift + static_cast<size_t>(r) * a.ld_mod;
+      const float* sc = staged ? ln_mod + (2 * (r - rfirst) + 1) * a.d : a.scale + static_cast<size_t>(r) * a.ld_mod;
+      ln_store_row<OUT>(a, mb, lane, nv, xb, mean, rstd, sh, sc);
     }
   }
 }
 
 cudaError_t launch_ln_modulate(const LnArgs& a, cudaStream_t st) {
   if ((a.d & 3) != 0 || a.d > 4 * 32 * kLnMaxVec) return cudaErrorInvalidValue;
-  const int grid = (a.M + kLnRowsPerBlock - 1) / kLnRowsPerBlock;
+  const int grid = (a.M + kLnRows - 1) / kLnRows;
   if (grid == 0) return cudaSuccess;
-  if (a.u_bf16)
-    return launch_kernel(ln_modulate_kernel<true>, dim3(grid), dim3(32 * kLnRowsPerBlock), 0, st, a);
-  return launch_kernel(ln_modulate_kernel<false>, dim3(grid), dim3(32 * kLnRowsPerBlock), 0, st, a);
+  const size_t smem = 4 * static_cast<size_t>(a.d) * sizeof(float);
+  if (a.u8 != nullptr) {
+    if (a.su == nullptr || a.sg == nullptr) return cudaErrorInvalidValue;
+    return launch_kernel(ln_modulate_kernel<2>, dim3(grid), dim3(kLnThreads), smem, st, a);
+  }
+  if (a.u_bf16) return launch_kernel(ln_modulate_kernel<1>, dim3(grid), dim3(kLnThreads), smem, st, a);
+  return launch_kernel(ln_modulate_kernel<0>, dim3(grid), dim3(kLnThreads), smem, st, a);
 }
 
 // ============================================================================ f32 GEMM
@@ -473,58 +679,44 @@ cudaError_t launch_attention_simt(const AttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// ============================================================================ decoder + unpatchify + CFG
-// One block per (sample b, token tau).  Each warp computes decoder outputs p
-// (stride 8); lanes split the d-long dot products.  Guided: both rows b and b+B
-// are decoded and combined as z_null + s (z_cond - z_null) (on channels c < gch only
-// when gch > 0; the others keep z_cond) before the scatter to
-// out[b, c, f*pt+it, i*ph+ih, j*pw+iw] with p = ((it*ph + ih)*pw + iw)*Cout + c.
-__global__ void decode_cfg_kernel(DecodeArgs a) {
+// ============================================================================ guidance + unpatchify
+// One thread per output element of [B, Cout, F, H, W], in memory order (stores coalesced);
+// the two decoder values it combines sit in rows b and B + b of z at the element's token.
+__global__ void __launch_bounds__(256) cfg_unpatchify_kernel(UnpatchArgs a) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ float su[];  // [2][d]
-  const int tau = blockIdx.x, b = blockIdx.y;
-  const int rows = a.guided ? 2 : 1;
-  for (int idx = threadIdx.x; idx < rows * a.d; idx += blockDim.x) {
-    const int rr = idx / a.d, j = idx - rr * a.d;
-    const size_t m = static_cast<size_t>(b + rr * a.B) * a.T + tau;
-    su[idx] = a.u_bf16 ? bf16_to_f32(static_cast<const uint16_t*>(a.u)[m * a.d + j])
-                       : static_cast<const float*>(a.u)[m * a.d + j];
-  }
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int gw = a.W / a.pw, gh = a.H / a.ph;
-  const int f = tau / (gh * gw), gi = (tau / gw) % gh, gj = tau % gw;
-  for (int p = warp; p < a.P; p += nw) {
-    const float* w = a.w + static_cast<size_t>(p) * a.d;
-    float zc = 0.f, zu = 0.f;
-    for (int j = lane; j < a.d; j += 32) {
-      const float wj = __ldg(w + j);
-      zc = fmaf(wj, su[j], zc);
-      if (a.guided) zu = fmaf(wj, su[a.d + j], zu);
+  const long long total = static_cast<long long>(a.B) * a.Cout * a.F * a.H * a.W;
+  const int gh = a.H / a.ph, gw = a.W / a.pw;
+  for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    long long r = idx;
+    const int ww = static_cast<int>(r % a.W);
+    r /= a.W;
+    const int hh = static_cast<int>(r % a.H);
+    r /= a.H;
+    const int fr = static_cast<int>(r % a.F);
+    r /= a.F;
+    const int c = static_cast<int>(r % a.Cout);
+    const int b = static_cast<int>(r / a.Cout);
+    const int tau = ((fr / a.pt) * gh + hh / a.ph) * gw + ww / a.pw;
+    const int p = (((fr % a.pt) * a.ph + hh % a.ph) * a.pw + ww % a.pw) * a.Cout + c;
+    const int Tr = a.Trow ? a.Trow : a.T;
+    const float zc = __ldg(a.z + (static_cast<size_t>(b) * Tr + a.tok0 + tau) * a.P + p);
+    float v = zc;
+    if (a.guided && (a.gch <= 0 || c < a.gch)) {
+      const float zu = __ldg(a.z + (static_cast<size_t>(b + a.B) * Tr + a.tok0 + tau) * a.P + p);
+      v = zu + a.s * (zc - zu);
     }
-    zc = warp_sum(zc);
-    zu = warp_sum(zu);
-    if (lane == 0) {
-      const int c = p % a.Cout;
-      zc += a.b[p];
-      float val = zc;
-      if (a.guided && (a.gch <= 0 || c < a.gch)) {
-        zu += a.b[p];
-        val = zu + a.s * (zc - zu);
-      }
-      const int iw = (p / a.Cout) % a.pw, ih = (p / (a.Cout * a.pw)) % a.ph, it = p / (a.Cout * a.pw * a.ph);
-      const size_t oi = ((((static_cast<size_t>(b) * a.Cout + c) * a.F + f * a.pt + it) * a.H + gi * a.ph + ih) * a.W) +
-                        gj * a.pw + iw;
-      a.out[oi] = val;
-    }
+    a.out[idx] = v;
   }
 }
 
-cudaError_t launch_decode_cfg(const DecodeArgs& a, cudaStream_t st) {
-  dim3 grid(a.T, a.B);
-  const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float);
-  return launch_kernel(decode_cfg_kernel, grid, dim3(256), smem, st, a);
+cudaError_t launch_cfg_unpatchify(const UnpatchArgs& a, int num_sms, cudaStream_t st) {
+  const long long total = static_cast<long long>(a.B) * a.Cout * a.F * a.H * a.W;
+  if (total == 0) return cudaSuccess;
+  const long long want = (total + 255) / 256;
+  const int grid = static_cast<int>(want < 8LL * num_sms ? want : 8LL * num_sms);
+  return launch_kernel(cfg_unpatchify_kernel, dim3(grid), dim3(256), 0, st, a);
 }
 
 // ============================================================================ sampler step
@@ -573,7 +765,7 @@ cudaError_t launch_sampler_step(const SamplerArgs& a, int num_sms, cudaStream_t 
 // the column; each half [sin(p w_k) | cos(p w_k)], w_k = 10000^(-k/(d/4)).
 // rope[tau, i, :] = (cos, sin) of the angle of pair i: slice a = 2i / (dh/3) picks the
 // axis (frame, row, col), k = (2i mod dh/3) / 2, angle = coord_a * 10000^(-2k/(dh/3)).
-__global__ void pos_tables_kernel(float* pos, float* rope, int gf, int gh, int gw, int d, int dh) {
+__global__ void pos_tables_kernel(float* pos, float* rope, int gf, int gh, int gw, int d, int dh, int tok0) {
   const int T = gf * gh * gw;
   const int q = d / 4;
   if (pos) {
@@ -588,8 +780,14 @@ __global__ void pos_tables_kernel(float* pos, float* rope, int gf, int gh, int g
   }
   if (rope) {
     const int sl = dh / 3;
-    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < T * (dh / 2); idx += gridDim.x * blockDim.x) {
-      const int tau = idx / (dh / 2), i = idx - tau * (dh / 2);
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < (T + tok0) * (dh / 2); idx += gridDim.x * blockDim.x) {
+      const int row = idx / (dh / 2), i = idx - row * (dh / 2);
+      if (row < tok0) {  // condition tokens: no rotation
+        rope[2 * idx] = 1.f;
+        rope[2 * idx + 1] = 0.f;
+        continue;
+      }
+      const int tau = row - tok0;
       const int axis = (2 * i) / sl, k = ((2 * i) % sl) / 2;
       const int coord = axis == 0 ? tau / (gh * gw) : (axis == 1 ? (tau / gw) % gh : tau % gw);
       const double ang = coord * pow(10000.0, -2.0 * k / sl);
@@ -599,9 +797,45 @@ __global__ void pos_tables_kernel(float* pos, float* rope, int gf, int gh, int g
   }
 }
 
-cudaError_t launch_pos_tables(float* pos, float* rope, int gf, int gh, int gw, int d, int dh, cudaStream_t st) {
-  pos_tables_kernel<<<256, 256, 0, st>>>(pos, rope, gf, gh, gw, d, dh);
+cudaError_t launch_pos_tables(float* pos, float* rope, int gf, int gh, int gw, int d, int dh, int tok0,
+                              cudaStream_t st) {
+  pos_tables_kernel<<<256, 256, 0, st>>>(pos, rope, gf, gh, gw, d, dh, tok0);
   return cudaGetLastError();
+}
+
+// ============================================================================ f32 cross-attention
+// One warp per (token, head): lanes split the head dim for the two scores, then write the
+// softmax mix of the two condition values.
+__global__ void xattn_f32_kernel(XAttnArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(a.M) * a.H) return;
+  const int m = static_cast<int>(w / a.H), head = static_cast<int>(w - static_cast<long long>(m) * a.H);
+  const int row = m / a.T;
+  const float* q = a.q + static_cast<size_t>(m) * a.d + head * a.dh;
+  const float* k0 = a.xkv + static_cast<size_t>(2 * row) * a.ld_xkv + head * a.dh;
+  const float* k1 = k0 + a.ld_xkv;
+  float s0 = 0.f, s1 = 0.f;
+  for (int j = lane; j < a.dh; j += 32) {
+    s0 = fmaf(q[j], k0[j], s0);
+    s1 = fmaf(q[j], k1[j], s1);
+  }
+  const float sc = rsqrtf(static_cast<float>(a.dh));
+  s0 = warp_sum(s0) * sc;
+  s1 = warp_sum(s1) * sc;
+  const float mx = fmaxf(s0, s1);
+  const float e0 = expf(s0 - mx), e1 = expf(s1 - mx);
+  const float p0 = e0 / (e0 + e1), p1 = e1 / (e0 + e1);
+  float* o = a.o + static_cast<size_t>(m) * a.d + head * a.dh;
+  for (int j = lane; j < a.dh; j += 32) o[j] = p0 * k0[a.d + j] + p1 * k1[a.d + j];
+}
+
+cudaError_t launch_xattn_f32(const XAttnArgs& a, cudaStream_t st) {
+  const long long warps = static_cast<long long>(a.M) * a.H;
+  if (warps == 0) return cudaSuccess;
+  return launch_kernel(xattn_f32_kernel, dim3(static_cast<unsigned>((warps + 7) / 8)), dim3(256), 0, st, a);
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst, size_t n) {
@@ -612,6 +846,45 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ src, uint16_t* __re
 
 cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaStream_t st) {
   f32_to_bf16_kernel<<<1184, 256, 0, st>>>(src, dst, n);
+  return cudaGetLastError();
+}
+
+// One block per row: the row's largest magnitude, then every element divided by amax / 448
+// and rounded to E4M3 (cols % 4 == 0).
+__global__ void __launch_bounds__(256) quantize_rows_e4m3_kernel(const float* __restrict__ src, uint8_t* __restrict__ dst,
+                                                                 float* __restrict__ scale, int cols) {
+  __shared__ float red[8];
+  const float4* row = reinterpret_cast<const float4*>(src + static_cast<size_t>(blockIdx.x) * cols);
+  const int n4 = cols / 4;
+  float m = 0.f;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = row[i];
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float s = red[0] > 0.f ? red[0] * (1.0f / 448.0f) : 1.0f;
+  if (threadIdx.x == 0) scale[blockIdx.x] = s;
+  const float inv = 1.0f / s;
+  uint32_t* out = reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(blockIdx.x) * cols);
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = row[i];
+    out[i] = pack_e4m3x4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+  }
+}
+
+cudaError_t launch_quantize_rows_e4m3(const float* src, uint8_t* dst, float* scale, int rows, int cols,
+                                      cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (cols % 4) return cudaErrorInvalidValue;
+  quantize_rows_e4m3_kernel<<<rows, 256, 0, st>>>(src, dst, scale, cols);
   return cudaGetLastError();
 }
 

@@ -61,6 +61,20 @@ typedef enum {
 enum { DIT_DTYPE_F32 = 0, DIT_DTYPE_BF16 = 1 };
 enum { DIT_POS_SINCOS2D = 0, DIT_POS_ROPE3D = 1 };
 enum { DIT_COND_CLASS = 0, DIT_COND_VECTOR = 1 };
+/* How the condition enters the blocks: the four designs "확산 트랜스포머" (itwiki.kr) compares
+   in section "조건 주입 방식" (conditioning), and what each block computes:
+   DIT_BLOCK_ADALN_ZERO  (b1,g1,a1,b2,g2,a2) = Linear(SiLU(c));
+                         x += a1 Attn(LN(x)(1+g1)+b1);  x += a2 FFN(LN(x)(1+g2)+b2)
+   DIT_BLOCK_IN_CONTEXT  e_t and e_y become two extra tokens in front of the patch tokens
+                         (no position; removed after the last block); plain pre-norm blocks
+                         x += Attn(LN1(x));  x += FFN(LN2(x)) with learned LN affines
+   DIT_BLOCK_CROSS_ATTN  plain pre-norm blocks with a cross-attention sublayer after the
+                         self-attention: x += CrossAttn(LNx(x), [e_t, e_y])
+   DIT_BLOCK_ADALN       (b1,g1,b2,g2) = Linear(SiLU(c)); the adaLN-Zero block without gates
+   (e_t = timestep MLP output, e_y = label row or text vector, c = e_t + e_y.)  The two
+   unmodulated designs end with a learned-affine LayerNorm before the decoder, the two
+   modulated ones with the adaLN (shift, scale) LayerNorm. */
+enum { DIT_BLOCK_ADALN_ZERO = 0, DIT_BLOCK_IN_CONTEXT = 1, DIT_BLOCK_CROSS_ATTN = 2, DIT_BLOCK_ADALN = 3 };
 
 /* Model and workload description.  Image models use frames = patch_t = 1. */
 typedef struct dit_config {
@@ -82,6 +96,12 @@ typedef struct dit_config {
   int freq_dim;       /* width of the timestep sinusoid (256) */
   int max_batch;      /* largest user batch B; device workspace is sized for 2*max_batch rows */
   float t_scale;      /* the sinusoid sees t * t_scale (1 for integer steps, 1000 for t in [0,1)) */
+  int block_kind;     /* DIT_BLOCK_* (0 = adaLN-Zero, the design of the standard DiT models) */
+  int ffn_fp8;        /* 1: the feed-forward matmuls run on FP8 E4M3 operands (bf16 path only):
+                         fc1.w / fc2.w quantised per output channel (scale amax / 448) at create,
+                         the LN output per token (amax / 448), the hidden activation per token with
+                         the scale (||u||_2 max_n ||fc1.w_n||_2 + max |fc1.b|) / 448, a bound on
+                         |GELU(z)| known before z is formed; accumulation stays float32 */
 } dit_config;
 
 typedef struct dit_handle dit_handle;
@@ -102,6 +122,12 @@ typedef struct dit_handle dit_handle;
  *   final.ada.w [2d, d], final.ada.b [2d], dec.w [P, d], dec.b [P].
  * The ada.w output rows are ordered (shift1, scale1, gate1, shift2, scale2, gate2),
  * the final ones (shift, scale); qkv.w rows are [q | k | v], heads contiguous.
+ * The other block designs change the per-block list and the final layer:
+ *   DIT_BLOCK_ADALN: ada.w [4d, d], ada.b [4d] with rows (shift1, scale1, shift2, scale2);
+ *   DIT_BLOCK_IN_CONTEXT: ln1.g [d], ln1.b [d] replace ada.w, ada.b, and ln2.g [d], ln2.b [d]
+ *       come before fc1.w; DIT_BLOCK_CROSS_ATTN: the same, plus after proj.b: xln.g [d],
+ *       xln.b [d], xq.w [d, d], xq.b [d], xkv.w [2d, d] (rows [k | v]), xkv.b [2d], xo.w [d, d],
+ *       xo.b [d]; for both, final.ln.g [d], final.ln.b [d] replace final.ada.w, final.ada.b.
  * The library copies everything; the caller may free the host arrays on return.
  * Blocks the calling thread until the upload is complete.
  * Returns DIT_ERR_INVALID_ARG / DIT_ERR_UNSUPPORTED before any CUDA call when the
@@ -217,8 +243,14 @@ void dit_destroy(dit_handle* h);
    combines only output channels c < n; the other channels return the conditional
    prediction.  n = 3 is the variant that "확산 트랜스포머" ("ImageNet 클래스 조건 생성")
    attributes to the official code; guidance on every channel is the standard form.
-   A negative n is DIT_ERR_INVALID_ARG. */
-enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2, DIT_OPT_OVERLAP_LAUNCH = 3, DIT_OPT_CFG_CHANNELS = 4 };
+   A negative n is DIT_ERR_INVALID_ARG.
+   DIT_OPT_REPEAT_KIND = k (a DIT_KERNEL_* kind, default -1 = off): a timing diagnostic that
+   launches every kernel of kind k twice where the forward launches it once, so that the step
+   time grows by that kind's in-pipeline cost (the second launch repeats the same work on the
+   same buffers; for the residual kinds DIT_KERNEL_PROJ and DIT_KERNEL_FC2 it adds the update
+   twice, so outputs are meaningless while it is on).  Part of the graph cache key. */
+enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2, DIT_OPT_OVERLAP_LAUNCH = 3, DIT_OPT_CFG_CHANNELS = 4,
+       DIT_OPT_REPEAT_KIND = 5 };
 dit_status dit_set_option(dit_handle* h, int option, int value);
 
 /*
@@ -258,8 +290,10 @@ dit_status dit_op_linear_bf16(const uint16_t* x, const uint16_t* w, const float*
                               int M, int N, int K, int block_n, dit_stream_t stream);
 
 /*
- * Per-step kernel timing.  While enabled, dit_forward brackets each launch with a pair
- * of CUDA events on its stream and files the pair under one of the DIT_KERNEL_* kinds.
+ * Per-step kernel timing.  While enabled, dit_forward brackets launches with a pair of CUDA
+ * events on its stream and files the pair under one of the DIT_KERNEL_* kinds: every launch
+ * (enable = 1) or only the launches of kind k (enable = 2 + k), so that the other kernels
+ * keep their programmatic-dependent-launch overlap.  The graph is bypassed while profiling.
  * dit_profile_read synchronises the device, writes per-kind total milliseconds and
  * launch counts (arrays of at least DIT_KERNEL_COUNT entries) and clears the record.
  */
@@ -288,7 +322,8 @@ dit_status dit_profile_read(dit_handle* h, float* total_ms, int* launches);
  * requests return DIT_ERR_INVALID_ARG before anything is launched.  The array
  * (1.75 MiB) stays resident on every GPU that loaded the library until the process
  * exits.  The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream capture.
+ * device, with that device current; again after a device reset gives the device a new
+ * context); make that first call before any stream capture.
  * All calls share the one array and it keeps the last call's contents; every call
  * rewrites what it reads, so nothing has to start at zero, but calls whose work
  * overlaps on the GPU (different streams, or different threads) race on it.
@@ -306,6 +341,40 @@ dit_status dit_condition_static(const float* t, const void* y, int B, int guided
  */
 dit_status dit_op_linear_bf16_pair(const uint16_t* x, const uint16_t* w, const float* b, float* y,
                                    int M, int N, int K, int block_n, dit_stream_t stream);
+
+/*
+ * dit_op_linear_e4m3 — the FP8 tensor-core GEMM building block (tcgen05.mma kind::f8f6f4):
+ *   y[m, n] = sx[m] sw[n] sum_k x[m, k] w[n, k] + b[n]
+ * x [M, K], w [N, K]: dev FP8 E4M3 bytes, row-major, K % 16 == 0, 16-byte aligned;
+ * sx [M], sw [N]: dev float32 scales; b: dev float32 [N] or NULL; y: dev float32 [M, N].
+ * block_n: 64, 128 or 256.  float32 accumulation.  Asynchronous on `stream`.
+ */
+dit_status dit_op_linear_e4m3(const uint8_t* x, const uint8_t* w, const float* sx, const float* sw, const float* b,
+                              float* y, int M, int N, int K, int block_n, dit_stream_t stream);
+
+/*
+ * dit_op_attention_bf16 — the tensor-core attention kernel of the bf16 forward on its own:
+ *   o[r, tau, h*dh : (h+1)*dh] = softmax(q_{r,h} k_{r,h}^T / sqrt(dh)) v_{r,h}   (full, no mask)
+ * for every sample row r < R and head h < H ("확산 트랜스포머", section "adaLN-Zero": Attn is
+ * multi-head self-attention over all T tokens).  Layouts (dev bf16 bit patterns, the forward's
+ * own workspace layouts; Tpad = T rounded up to a multiple of 128, DP = dh rounded up to a
+ * multiple of 16):
+ *   q, k [R*H, Tpad, DP]  row-major, rows >= T and columns >= dh must hold zeros;
+ *   v    [R*H, DP, Tpad]  V transposed, same zero padding;
+ *   o    [R*T, H*dh]      token-major output.
+ * dh must be 64 or 72 (DIT_ERR_UNSUPPORTED otherwise).  counters: dev int32[2] or NULL;
+ * counters[0] receives DIT_ERR_DEVICE_TIMEOUT if a bounded wait runs out, and counters[1] is
+ * incremented once per warp of 32 query rows each time the online softmax moves its
+ * reference maximum (and rescales its running output) because the row maximum grew by more
+ * than 2^8 — a diagnostic of that code path.  Asynchronous on `stream`.
+ */
+dit_status dit_op_attention_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o, int R, int H,
+                                 int T, int dh, int* counters, dit_stream_t stream);
+
+/* Reads and clears the handle's count of attention reference-maximum moves (the same event
+   as counters[1] of dit_op_attention_bf16), accumulated over every bf16 forward since the
+   last read.  Synchronises the device first. */
+dit_status dit_debug_attention_rescales(dit_handle* h, long long* count);
 
 /* Number of kernel launches one dit_forward enqueues for batch B (graph nodes if a
    graph is replayed). */

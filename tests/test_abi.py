@@ -31,8 +31,9 @@ def test_library_exports_every_declared_function():
 def test_weight_count_matches_generator():
     lib = binding.load()
     for cfg in S.STANDARD:
-        c = binding.make_config(cfg)
-        assert lib.dit_weight_count(ctypes.byref(c)) == len(S.weight_specs(cfg))
+        for kind in (S.BLOCK_ADALN_ZERO, S.BLOCK_IN_CONTEXT, S.BLOCK_CROSS_ATTN, S.BLOCK_ADALN):
+            c = binding.make_config(cfg.with_(block_kind=kind))
+            assert lib.dit_weight_count(ctypes.byref(c)) == len(S.weight_specs(cfg.with_(block_kind=kind)))
 
 
 def _create(cfg, weights=None, n=None):
@@ -52,6 +53,9 @@ def _create(cfg, weights=None, n=None):
     (dict(dtype=7), binding.DIT_ERR_INVALID_ARG),
     (dict(batch=0), binding.DIT_ERR_INVALID_ARG),
     (dict(freq_dim=255), binding.DIT_ERR_INVALID_ARG),
+    (dict(block_kind=4), binding.DIT_ERR_INVALID_ARG),
+    (dict(ffn_fp8=2), binding.DIT_ERR_INVALID_ARG),
+    (dict(ffn_fp8=1), binding.DIT_ERR_UNSUPPORTED),          # FP8 feed-forward needs the bf16 path
     (dict(heads=12), binding.DIT_ERR_UNSUPPORTED),           # head dim 32
     (dict(hidden=2048, heads=32, mlp_hidden=8192), binding.DIT_ERR_UNSUPPORTED),  # hidden > 1536
 ])

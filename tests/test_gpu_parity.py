@@ -62,11 +62,17 @@ def small_video_bf16():        # T = 48, QK-RMSNorm + 3D RoPE
                             batch=2, index=-1)
 
 
+def small_image_bf16_dh64_ragged():   # dh 64, T = 225 (two key tiles, ragged), 6 guided rows
+    return S.DIT_XL2_CFG256.with_(hidden=256, heads=4, mlp_hidden=1024, depth=2, height=30, width=30, batch=3,
+                                  index=-1)
+
+
 SMALL = {
     "s8_f32": lambda: S.DIT_S8_F32,
     "video_f32": small_video_f32,
     "img_bf16_dh72": small_image_bf16_dh72,
     "img_bf16_dh64": small_image_bf16_dh64,
+    "img_bf16_dh64_ragged": small_image_bf16_dh64_ragged,
     "video_bf16": small_video_bf16,
     "b4_bf16_full": lambda: S.DIT_B4_BF16,
 }
@@ -123,7 +129,7 @@ def test_forward_parity(name, gates):
     m.close()
 
 
-@pytest.mark.parametrize("name", ["s8_f32", "img_bf16_dh72", "video_bf16", "video_f32"])
+@pytest.mark.parametrize("name", ["s8_f32", "img_bf16_dh72", "img_bf16_dh64_ragged", "video_bf16", "video_f32"])
 def test_residual_stream_parity_per_block(name):
     cfg = SMALL[name]()
     W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
@@ -276,24 +282,80 @@ def test_host_side_errors_launch_nothing():
     m.close()
 
 
+def tie_keys_to_queries(cfg, W, f):
+    """Copy of W whose key projections equal the query projections scaled by f (and the
+    query projections scaled by f): every logit q_i . q_j then peaks on its own token, far
+    above the first key tile's best, so the attention's running maximum must move."""
+    W = [w.copy() for w in W]
+    names = [n for n, _, _ in S.weight_specs(cfg)]
+    d = cfg.hidden
+    for i in range(cfg.depth):
+        w, b = W[names.index(f"blocks.{i}.qkv.w")], W[names.index(f"blocks.{i}.qkv.b")]
+        w[:d] *= f
+        b[:d] *= f
+        w[d:2 * d] = w[:d]
+        b[d:2 * d] = b[:d]
+    return W
+
+
+def test_attention_rescale_path_in_the_forward():
+    """A model whose logits span far more than 2^8 across key tiles (T = 576, five key
+    tiles): the forward's attention takes its rescale path (read back through the handle's
+    counter) and still matches the oracle, per block and at the output."""
+    cfg = small_image_bf16_dh72().with_(height=48, width=48, batch=2)
+    W = tie_keys_to_queries(cfg, S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0), 8.0)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    assert m.attention_rescales() == 0
+    got = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    assert m.sync_status() == binding.DIT_OK
+    events = m.attention_rescales()
+    assert events > 0
+    assert_parity(cfg, got, O.forward(cfg, W, inp["x"], inp["t"], inp["y"]), "rescale forward")
+    h1 = m.debug_residual(d["x"], d["t"], d["y"], cfg.cfg_scale, 1).cpu().numpy()
+    assert_parity(cfg, h1, O.forward(cfg, W, inp["x"], inp["t"], inp["y"], stop_after_block=1), "after block 1")
+    # the standard weights never take that path
+    m.close()
+    m = DiT(cfg, S.make_weights(cfg))
+    m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale)
+    assert m.attention_rescales() == 0
+    m.close()
+
+
 # ----------------------------------------------------------------------------- full-size workloads
 # The benchmark's launch configuration (standard weights/inputs, full batch) on the GPU;
 # the oracle recomputes one sampled sample (rows of a batch are independent, so sample
 # b of the batched GPU output must equal the oracle run on sample b alone).
-@pytest.mark.parametrize("cfg", [S.DIT_XL2_CFG256, S.DIT_XL2_CFG512, S.VIDEO_RF], ids=["xl2_cfg256", "xl2_cfg512", "video_rf"])
-def test_full_size_sampled_parity(cfg):
+FULL = [S.DIT_XL2_CFG256, S.DIT_XL2_CFG512, S.VIDEO_RF]
+FULL_IDS = ["xl2_cfg256", "xl2_cfg512", "video_rf"]
+
+
+@pytest.mark.parametrize("cfg", FULL, ids=FULL_IDS)
+@pytest.mark.parametrize("gates", ["random", "strong"])
+def test_full_size_sampled_parity(cfg, gates):
+    """Standard weights: the last sample (its guided partner is the batch's last row).
+    Gate biases 1.0, so every block moves the residual stream strongly: the first and the
+    last sample.  Every other sample is checked against a single-sample GPU forward."""
     W = S.make_weights(cfg)
+    if gates == "strong":
+        W = S.set_adaln(cfg, W, gate_bias=1.0)
     inp = S.make_inputs(cfg)
     m = DiT(cfg, W)
     d = dev(inp)
     got = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
     assert m.sync_status() == binding.DIT_OK
-    m.close()
-    b = cfg.batch - 1   # the last sample: its guided partner is the last row of the batch
-    want = O.forward(cfg, S.weight_dict(cfg, W), inp["x"][b:b + 1], inp["t"][b:b + 1], inp["y"][b:b + 1])
-    assert_parity(cfg, got[b:b + 1], want, cfg.name)
-    # every sample: finite and of the expected shape
     assert got.shape == cfg.out_shape() and np.all(np.isfinite(got))
+    # rows are independent: each sample of the batched forward equals the same sample alone
+    for b in range(cfg.batch):
+        one = m.forward(d["x"][b:b + 1].contiguous(), d["t"][b:b + 1].contiguous(), d["y"][b:b + 1].contiguous(),
+                        cfg.cfg_scale).cpu().numpy()
+        assert metrics(one[0], got[b])[0] < 1e-5, b
+    m.close()
+    Wd = S.weight_dict(cfg, W)
+    for b in ([cfg.batch - 1] if gates == "random" else [0, cfg.batch - 1]):
+        want = O.forward(cfg, Wd, inp["x"][b:b + 1], inp["t"][b:b + 1], inp["y"][b:b + 1])
+        assert_parity(cfg, got[b:b + 1], want, f"{cfg.name} sample {b} {gates} gates")
 
 
 # ----------------------------------------------------------------------------- edge shapes
@@ -310,6 +372,8 @@ EDGE = {
                                                          width=16, batch=2),
     # a single sample
     "batch1_video": lambda: small_video_bf16().with_(batch=1),
+    # dh 64 over eight key tiles (T = 1024), guided
+    "dh64_T1024": lambda: small_image_bf16_dh64_ragged().with_(height=64, width=64, depth=1, batch=1),
 }
 
 
