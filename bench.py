@@ -51,10 +51,21 @@ def peaks():
     return FALLBACK, "fallback"
 
 
+WORKLOADS = {
+    "xl2_256": S.DIT_XL2_CFG256,           # the headline workload
+    "xl2_512": S.DIT_XL2_CFG512,
+    "video": S.VIDEO_RF,
+    "b4": S.DIT_B4_BF16,
+    "xl2_256_fp8": S.DIT_XL2_CFG256.with_(ffn_fp8=1),
+}
+
+
 def workload_desc(cfg):
-    return (f"DiT-XL/2 CFG 256px: {cfg.batch} latents {cfg.in_channels}x{cfg.height}x{cfg.width} -> "
-            f"{cfg.rows} rows x {cfg.tokens} tokens, d={cfg.hidden}, {cfg.depth} blocks, {cfg.heads} heads, "
-            f"s={cfg.cfg_scale}")
+    lat = (f"{cfg.in_channels}x{cfg.frames}x{cfg.height}x{cfg.width}" if cfg.frames > 1
+           else f"{cfg.in_channels}x{cfg.height}x{cfg.width}")
+    extra = ", FP8 E4M3 feed-forward" if getattr(cfg, "ffn_fp8", 0) else ""
+    return (f"{cfg.name}: {cfg.batch} latents {lat} -> {cfg.rows} rows x {cfg.tokens} tokens, d={cfg.hidden}, "
+            f"{cfg.depth} blocks, {cfg.heads} heads, s={cfg.cfg_scale}{extra}")
 
 
 def kernel_flops(cfg):
@@ -291,6 +302,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch every kernel directly instead of replaying a CUDA graph")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="xl2_256",
+                    help="the workload one step runs (default: the headline DiT-XL/2 CFG 256px; the others are "
+                         "for profiling and comparison)")
+    ap.add_argument("--lean", action="store_true",
+                    help="warm-up and timed steps only (no kernel table, end-to-end or sampler passes): the command "
+                         "profiler captures run under")
     ap.add_argument("--all-configs", action="store_true",
                     help="also time the other workloads (S/8 fp32, B/4, XL/2 512px CFG, video) and report them under "
                          "'all_configs' in the same JSON line")
@@ -309,7 +326,7 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
-    cfg = CFG
+    cfg = WORKLOADS[args.workload]
     weights = S.make_weights(cfg)
     model = DiT(cfg, weights)
     model.set_option(DIT_OPT_USE_GRAPH, 0 if args.no_graph else 1)
@@ -350,6 +367,19 @@ def main():
     total_ms = max_over_ranks(sum(step_ms), world, "cuda")
     status = model.sync_status()
     clocks = sampler.summary()
+
+    if args.lean:
+        line = {"metric": METRIC, "value": aggregate_rate(cfg.rows * cfg.tokens, world, args.steps, total_ms / 1e3),
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "config": {"workload": workload_desc(cfg)}, "lean": True, "device_status": status}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        model.close()
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
 
     # launches per step of each kernel kind (one profiled forward)
     model.profile(True)

@@ -197,6 +197,7 @@ struct dit_handle {
   int force_guidance = 0;
   int cfg_channels = 0;  // DIT_OPT_CFG_CHANNELS: guided output channels (0: all)
   int repeat_kind = -1;  // DIT_OPT_REPEAT_KIND: kernel kind launched twice per use (-1: none)
+  int ksplit_short = 2;  // DIT_OPT_SPLIT_K: K slices of the short-K residual GEMMs
   // CUDA-graph replay of the whole forward (DIT_OPT_USE_GRAPH): one cached executable graph,
   // valid for the exact pointers and parameters it was captured with
   struct GraphKey {
@@ -861,6 +862,9 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
       EpiArgs pt = pa;  // swapped: rows = d output features, columns = tokens
       pt.M = d;
       pt.N = p.M;
+      // short K (the d-wide projections): two K slices double the work units per SM, so
+      // the pipeline fill and the last epilogue are no longer exposed
+      pt.ksplit = K <= 2048 ? H->ksplit_short : 1;
       DIT_LAUNCH(H, kind, st, launch_gemm_tc(EPI_RESID_T, 256, ta, tb, K, pt, H->num_sms, st, &H->tm_h_red), where);
     } else {
       DIT_LAUNCH(H, kind, st,
@@ -1230,6 +1234,15 @@ dit_status dit_set_option(dit_handle* H, int option, int value) {
   if (option == DIT_OPT_CFG_CHANNELS) {
     if (value < 0) return fail(H, DIT_ERR_INVALID_ARG, "guided channel count must be >= 0");
     H->cfg_channels = value;
+    return DIT_OK;
+  }
+  if (option == DIT_OPT_SPLIT_K) {
+    if (value < 1 || value > 8) return fail(H, DIT_ERR_INVALID_ARG, "split-K must be 1..8");
+    H->ksplit_short = value;
+    H->has_gseen = H->has_sseen = false;  // a new kernel configuration: recapture
+    if (H->gexec != nullptr) cudaGraphExecDestroy(H->gexec);
+    if (H->sexec != nullptr) cudaGraphExecDestroy(H->sexec);
+    H->gexec = H->sexec = nullptr;
     return DIT_OK;
   }
   if (option == DIT_OPT_REPEAT_KIND) {

@@ -330,14 +330,15 @@ __device__ __forceinline__ void epilogue_cols_staged(const EpiArgs& ea, const CU
 // the stream back.
 // FP8 = true: E4M3 operands, the accumulator is first scaled by the weight row's scale sa[f]
 // and each token's scale sb[tok].
+// with_bias = false: a split-K slice other than the first adds its partial product only.
 template <int NC, bool FP8 = false>
 __device__ __forceinline__ void epilogue_resid_t(const EpiArgs& ea, const CUtensorMap* tmC, uint32_t tacc, int f_base,
-                                                 int lane, int n0, int c0, uint8_t* stg) {
+                                                 int lane, int n0, int c0, uint8_t* stg, bool with_bias = true) {
   static_assert(NC % 32 == 0, "32-token chunks");
   constexpr int NCH = NC / 32;
   const int f = f_base + lane;
   const bool fok = f < ea.M;
-  const float bf = fok ? __ldg(ea.bias + f) : 0.f;
+  const float bf = (fok && with_bias) ? __ldg(ea.bias + f) : 0.f;
   const float sf = (FP8 && fok) ? __ldg(ea.sa + f) : 1.f;
   uint32_t r[2][32];
   tmem_ld_chunk<32>(tacc + c0, r[0]);

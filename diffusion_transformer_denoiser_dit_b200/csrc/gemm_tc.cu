@@ -21,6 +21,12 @@
 
 namespace dit {
 
+// k-blocks per split-K slice for a requested split (1 when not split); the slice count is then
+// ceil(kblocks / result), so no slice is empty.
+__host__ __device__ inline int kblocks_per_slice(int kblocks, int split) {
+  return split > 1 && kblocks > 0 ? (kblocks + split - 1) / split : (kblocks > 0 ? kblocks : 1);
+}
+
 template <int BN, int EPI>
 struct TcCfg {
   static constexpr bool F8 = epi_fp8<EPI>();            // E4M3 operands (one byte per element)
@@ -64,7 +70,11 @@ __global__ void __launch_bounds__(320, 1)
   const int m_tiles = (ea.M + 127) / 128;
   const int n_tiles = (ea.N + BN - 1) / BN;
   const int num_tiles = m_tiles * n_tiles;
-  const int kblocks = (K + C::BK - 1) / C::BK;
+  const int kblocks_all = (K + C::BK - 1) / C::BK;
+  // split-K (the reduce-add residual epilogues only): work unit u is k-slice u / num_tiles of
+  // tile u % num_tiles, so the slices of one tile are far apart in time
+  const int kblocks = kblocks_per_slice(kblocks_all, (EPI == EPI_RESID_T || EPI == EPI_RESID_T8) ? ea.ksplit : 1);
+  const int num_units = num_tiles * ((kblocks_all + kblocks - 1) / kblocks);  // every slice has >= 1 k-block
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -100,9 +110,11 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t ph = 0;
       bool ok = true;
       uint32_t armed = 0;  // bit s: stage s has been filled at least once
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
+        const int tile = unit % num_tiles, kb0 = (unit / num_tiles) * kblocks;
         const int m0 = (tile % m_tiles) * 128, n0 = (tile / m_tiles) * BN;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        const int kb1 = min(kb0 + kblocks, kblocks_all);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(EMPTY_BAR(s), ph ^ 1u, ea.status)) {
             ok = false;
             break;
@@ -132,13 +144,14 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t ph = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x, ++it) {
+        const int kb0 = (unit / num_tiles) * kblocks, nkb = min(kblocks, kblocks_all - kb0);
         const int a = it & 1;
         const uint32_t uph = (it >> 1) & 1;
         if (!mbar_wait(TEMPTY_BAR(a), uph ^ 1u, ea.status)) break;
         tc_fence_after();
         const uint32_t dt = tmem_base + a * C::ACC_COLS;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(FULL_BAR(s), ph, ea.status)) {
             ok = false;
             break;
@@ -170,7 +183,9 @@ __global__ void __launch_bounds__(320, 1)
   } else {  // ------------------------ epilogue warps 2..9
     const int q = warp & 3;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int unit = blockIdx.x; unit < num_units; unit += gridDim.x, ++it) {
+      const int tile = unit % num_tiles;
+      const bool first_slice = unit < num_tiles;  // the bias is added once per tile
       const int a = it & 1;
       const uint32_t uph = (it >> 1) & 1;
       const bool ok = mbar_wait(TFULL_BAR(a), uph, ea.status);
@@ -182,7 +197,7 @@ __global__ void __launch_bounds__(320, 1)
       if constexpr (EPI == EPI_RESID_T || EPI == EPI_RESID_T8)
         epilogue_resid_t<BN / 2, EPI == EPI_RESID_T8>(ea, &tmC, tacc, m0 + q * 32, lane, n0,
                                                        ((warp - 2) >> 2) * (BN / 2),
-                                                       staging + (warp - 2) * kStageBytesPerWarp);
+                                                       staging + (warp - 2) * kStageBytesPerWarp, first_slice);
       else if constexpr (EPI == EPI_GELU8)
         epilogue_gelu8<BN / 2>(ea, tacc, m0 + q * 32 + lane, n0, ((warp - 2) >> 2) * (BN / 2));
       else if constexpr (EPI == EPI_QKV_T)
@@ -295,7 +310,9 @@ static cudaError_t launch_bn(const CUtensorMap* tA, const CUtensorMap* tB, const
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  const int tiles = ((ea.M + 127) / 128) * ((ea.N + BN - 1) / BN);
+  const int kb_all = (K + C::BK - 1) / C::BK;
+  const int kb = kblocks_per_slice(kb_all, (EPI == EPI_RESID_T || EPI == EPI_RESID_T8) ? ea.ksplit : 1);
+  const int tiles = ((ea.M + 127) / 128) * ((ea.N + BN - 1) / BN) * ((kb_all + kb - 1) / kb);
   if (tiles == 0) return cudaSuccess;
   const int grid = tiles < num_sms ? tiles : num_sms;
   return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(320), C::SMEM, st, *tA, *tB, tC ? *tC : *tB, K, ea);

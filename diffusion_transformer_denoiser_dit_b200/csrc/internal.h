@@ -63,6 +63,9 @@ struct EpiArgs {
   const float* sa;
   const float* sb;
   const float* sg;
+  // EPI_RESID_T / EPI_RESID_T8: split K into this many slices (each adds its partial product
+  // into the residual stream; 0 or 1 = no split)
+  int ksplit;
   int* status;
 };
 

@@ -248,9 +248,12 @@ void dit_destroy(dit_handle* h);
    launches every kernel of kind k twice where the forward launches it once, so that the step
    time grows by that kind's in-pipeline cost (the second launch repeats the same work on the
    same buffers; for the residual kinds DIT_KERNEL_PROJ and DIT_KERNEL_FC2 it adds the update
-   twice, so outputs are meaningless while it is on).  Part of the graph cache key. */
+   twice, so outputs are meaningless while it is on).  Part of the graph cache key.
+   DIT_OPT_SPLIT_K = s (1..8, default 2): the residual GEMMs with a short reduction (the
+   d-wide out-projections) split K into s slices, each adding its share into the residual
+   stream (the results differ from s = 1 only in float32 summation order). */
 enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2, DIT_OPT_OVERLAP_LAUNCH = 3, DIT_OPT_CFG_CHANNELS = 4,
-       DIT_OPT_REPEAT_KIND = 5 };
+       DIT_OPT_REPEAT_KIND = 5, DIT_OPT_SPLIT_K = 6 };
 dit_status dit_set_option(dit_handle* h, int option, int value);
 
 /*

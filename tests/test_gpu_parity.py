@@ -432,3 +432,24 @@ def test_guidance_on_the_first_channels_only():
         m.set_option(binding.DIT_OPT_CFG_CHANNELS, -1)
     assert m.sync_status() == binding.DIT_OK
     m.close()
+
+
+def test_split_k_residual_gemms_match_unsplit():
+    """DIT_OPT_SPLIT_K: the out-projection's K slices each add their share into the residual
+    stream; any split gives the unsplit result up to float32 summation order, and parity."""
+    cfg = small_image_bf16_dh72()
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    d = dev(inp)
+    outs = {}
+    for sk in (1, 2, 3, 8):
+        m.set_option(binding.DIT_OPT_SPLIT_K, sk)
+        outs[sk] = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    assert m.sync_status() == binding.DIT_OK
+    for sk in (2, 3, 8):
+        assert metrics(outs[sk], outs[1])[0] < 1e-4, sk
+    assert_parity(cfg, outs[2], O.forward(cfg, W, inp["x"], inp["t"], inp["y"]), "split-K 2")
+    with pytest.raises(binding.DitError):
+        m.set_option(binding.DIT_OPT_SPLIT_K, 0)
+    m.close()
