@@ -241,14 +241,16 @@ def cpu_baseline(cfg, weights):
                       f"float64 numpy oracle, {el:.1f} s"}
 
 
-def time_config(cfg, steps, warmup, graph, flush):
+def time_config(cfg, steps, warmup, graph, flush, options=None):
     """Device time of `steps` whole forwards of `cfg` (seeded weights and inputs, L2 flushed between
-    steps outside the events).  Returns per-step milliseconds."""
+    steps outside the events), with library options {option: value}.  Returns per-step milliseconds."""
     import torch
     from diffusion_transformer_denoiser_dit_b200 import DiT
     from diffusion_transformer_denoiser_dit_b200.binding import DIT_OPT_USE_GRAPH
     model = DiT(cfg, S.make_weights(cfg))
     model.set_option(DIT_OPT_USE_GRAPH, 1 if graph else 0)
+    for opt, val in (options or {}).items():
+        model.set_option(opt, val)
     inp = S.make_inputs(cfg)
     x, t, y = (torch.from_numpy(inp[k]).cuda() for k in ("x", "t", "y"))
     out = torch.empty(cfg.out_shape(), dtype=torch.float32, device="cuda")
@@ -271,7 +273,11 @@ def time_config(cfg, steps, warmup, graph, flush):
 
 
 def all_configs(steps, warmup, graph, flush, peak_tf):
+    from diffusion_transformer_denoiser_dit_b200.binding import DIT_OPT_PAIR_GEMM
     res = {}
+    runs = []
+    pair_after = {"c3 XL/2 CFG 256px": "c3 XL/2 CFG 256px, SM-pair GEMMs",
+                  "c4 XL/2 CFG 512px": "c4 XL/2 CFG 512px, SM-pair GEMMs"}
     for name, cfg in (("c1 S/8 fp32", S.DIT_S8_F32), ("c2 B/4 bf16", S.DIT_B4_BF16),
                       ("c3 XL/2 CFG 256px", S.DIT_XL2_CFG256), ("c4 XL/2 CFG 512px", S.DIT_XL2_CFG512),
                       ("c5 video RF 4096 tokens", S.VIDEO_RF),
@@ -280,7 +286,11 @@ def all_configs(steps, warmup, graph, flush, peak_tf):
                       ("c3 XL/2 CFG 256px, adaLN conditioning", S.DIT_XL2_CFG256.with_(block_kind=S.BLOCK_ADALN)),
                       ("c3 XL/2 CFG 256px, FP8 E4M3 feed-forward", S.DIT_XL2_CFG256.with_(ffn_fp8=1)),
                       ("c5 video RF 4096 tokens, FP8 E4M3 feed-forward", S.VIDEO_RF.with_(ffn_fp8=1))):
-        ms = time_config(cfg, steps, warmup, graph, flush)
+        runs.append((name, cfg, None))
+        if name in pair_after:   # the same workload on SM-pair GEMMs, timed right after it
+            runs.append((pair_after[name], cfg, {DIT_OPT_PAIR_GEMM: 1}))
+    for name, cfg, opts in runs:
+        ms = time_config(cfg, steps, warmup, graph, flush, opts)
         med = statistics.median(ms)
         _, fl = kernel_flops(cfg)
         tf = fl / (med / 1e3) / 1e12
@@ -305,6 +315,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="xl2_256",
                     help="the workload one step runs (default: the headline DiT-XL/2 CFG 256px; the others are "
                          "for profiling and comparison)")
+    ap.add_argument("--pair-gemm", action="store_true", help="run the block GEMMs on SM pairs (DIT_OPT_PAIR_GEMM)")
     ap.add_argument("--lean", action="store_true",
                     help="warm-up and timed steps only (no kernel table, end-to-end or sampler passes): the command "
                          "profiler captures run under")
@@ -318,7 +329,7 @@ def main():
     import torch
     import torch.distributed as dist
     from diffusion_transformer_denoiser_dit_b200 import DiT
-    from diffusion_transformer_denoiser_dit_b200.binding import DIT_OPT_REPEAT_KIND, DIT_OPT_USE_GRAPH
+    from diffusion_transformer_denoiser_dit_b200.binding import DIT_OPT_PAIR_GEMM, DIT_OPT_REPEAT_KIND, DIT_OPT_USE_GRAPH
 
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -330,6 +341,8 @@ def main():
     weights = S.make_weights(cfg)
     model = DiT(cfg, weights)
     model.set_option(DIT_OPT_USE_GRAPH, 0 if args.no_graph else 1)
+    if args.pair_gemm:
+        model.set_option(DIT_OPT_PAIR_GEMM, 1)
     inp = S.make_inputs(cfg, seed=replica_seed(cfg, rank))
     x = torch.from_numpy(inp["x"]).cuda()
     t = torch.from_numpy(inp["t"]).cuda()

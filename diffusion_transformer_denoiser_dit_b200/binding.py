@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdit_b200
 DIT_OK, DIT_ERR_INVALID_ARG, DIT_ERR_UNSUPPORTED, DIT_ERR_OOM, DIT_ERR_CUDA = 0, 1, 2, 3, 4
 DIT_ERR_DEVICE_TIMEOUT, DIT_ERR_BAD_LABEL, DIT_ERR_NO_DEVICE = 5, 6, 7
 DIT_OPT_FORCE_GUIDANCE, DIT_OPT_USE_GRAPH, DIT_OPT_OVERLAP_LAUNCH, DIT_OPT_CFG_CHANNELS = 1, 2, 3, 4
-DIT_OPT_REPEAT_KIND, DIT_OPT_SPLIT_K = 5, 6
+DIT_OPT_REPEAT_KIND, DIT_OPT_SPLIT_K, DIT_OPT_PAIR_GEMM = 5, 6, 7
 DIT_SAMPLER_DDIM, DIT_SAMPLER_EULER = 0, 1
 
 # every exported symbol declared in include/dit.h

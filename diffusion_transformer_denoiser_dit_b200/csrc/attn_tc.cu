@@ -266,8 +266,9 @@ __global__ void __launch_bounds__(384, 1)
         return true;
       };
       // Q K^T of the next key tile goes in before P V of the current one, so the tensor
-      // cores work while the softmax runs; across an item boundary P V goes first (the
-      // next item's Q is loaded only after the current item's last Q K^T).
+      // cores work while the softmax runs, across item boundaries too: the next item's Q sits
+      // in the other Q buffer, loaded after this item's K / V tiles, and its first K / V
+      // stage is freed by earlier MMAs only, so that Q K^T never waits on this P V.
       int n_qk = 0;
       bool ok = true;
       // Group 1 starts about half a key-tile period behind group 0 (once group 0 has written
@@ -275,7 +276,7 @@ __global__ void __launch_bounds__(384, 1)
       // of coinciding; group 0 needs nothing from group 1 to get there.
       if (g == 1 && !mbar_wait(BAR(B_GO), 0, status)) ok = false;
       for (int n = 0; n < ntiles && ok; ++n) {
-        while (ok && (n_qk <= n || (n_qk == n + 1 && n_qk < ntiles && cq.j != 0))) ok = issue_qk(n_qk++);
+        while (ok && (n_qk <= n || (n_qk == n + 1 && n_qk < ntiles))) ok = issue_qk(n_qk++);
         if (ok) ok = issue_pv(n);
       }
     }

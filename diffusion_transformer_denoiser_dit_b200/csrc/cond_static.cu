@@ -75,7 +75,7 @@ extern "C" dit_status dit_condition_static(const float* t, const void* y, int B,
                                            int cond_kind, int num_classes, int freq_dim, int hidden, float t_scale,
                                            float* c_out, int* status, dit_stream_t stream) {
   if (t == nullptr || y == nullptr || w1 == nullptr || b1 == nullptr || w2 == nullptr || b2 == nullptr ||
-      c_out == nullptr || B < 1 || hidden < 1 || freq_dim < 2 || (freq_dim & 1))
+      c_out == nullptr || B < 1 || hidden < 4 || (hidden & 3) || freq_dim < 4 || (freq_dim & 3))
     return DIT_ERR_INVALID_ARG;
   if (cond_kind != DIT_COND_CLASS && cond_kind != DIT_COND_VECTOR) return DIT_ERR_INVALID_ARG;
   if (cond_kind == DIT_COND_CLASS && (table == nullptr || num_classes < 1)) return DIT_ERR_INVALID_ARG;

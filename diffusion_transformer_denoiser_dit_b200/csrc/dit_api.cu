@@ -31,6 +31,7 @@ struct BlockW {
   float *fc1_s = nullptr, *fc2_s = nullptr;
   float g_w = 0.f, g_b = 0.f;
   CUtensorMap tm_qkv, tm_fc1, tm_xq, tm_fc1_8;  // weights as the B operand (box = tile width rows)
+  CUtensorMap tm_fc1_h;  // fc1 weights as the B operand of the SM-pair GEMM (each CTA loads half: 128 rows)
   CUtensorMap ta_qkv, ta_proj, ta_fc2, ta_xo, ta_fc2_8;  // weights as the A operand of the swapped GEMMs (box 128 rows)
 };
 
@@ -64,7 +65,7 @@ bool validate(const dit_config* c, std::string& err) {
   if (c->qk_norm != 0 && c->qk_norm != 1) return bad("qk_norm must be 0 or 1");
   if (c->cond_kind != DIT_COND_CLASS && c->cond_kind != DIT_COND_VECTOR) return bad("unknown cond_kind");
   if (c->cond_kind == DIT_COND_CLASS && c->num_classes <= 0) return bad("num_classes must be positive");
-  if (c->freq_dim <= 0 || (c->freq_dim & 1)) return bad("freq_dim must be positive and even");
+  if (c->freq_dim <= 0 || (c->freq_dim & 3)) return bad("freq_dim must be a positive multiple of 4");
   if (c->max_batch <= 0) return bad("max_batch must be positive");
   if (!isfinite(c->t_scale)) return bad("t_scale must be finite");
   if (c->block_kind < DIT_BLOCK_ADALN_ZERO || c->block_kind > DIT_BLOCK_ADALN) return bad("unknown block_kind");
@@ -81,6 +82,10 @@ bool supported(const dit_config* c, std::string& err) {
   }
   if (c->hidden % 4 || c->hidden > 1536) {
     err = "hidden must be a multiple of 4 and at most 1536";
+    return false;
+  }
+  if (c->freq_dim > 1536) {
+    err = "freq_dim must be at most 1536";
     return false;
   }
   if (c->pos_kind == DIT_POS_SINCOS2D && (c->frames / c->patch_t != 1 || c->hidden % 4)) {
@@ -197,7 +202,8 @@ struct dit_handle {
   int force_guidance = 0;
   int cfg_channels = 0;  // DIT_OPT_CFG_CHANNELS: guided output channels (0: all)
   int repeat_kind = -1;  // DIT_OPT_REPEAT_KIND: kernel kind launched twice per use (-1: none)
-  int ksplit_short = 2;  // DIT_OPT_SPLIT_K: K slices of the short-K residual GEMMs
+  int ksplit_short = 1;  // DIT_OPT_SPLIT_K: K slices of the short-K residual GEMMs (1: deterministic)
+  int pair_gemm = 0;     // DIT_OPT_PAIR_GEMM: block GEMMs on SM pairs (tcgen05 cta_group::2)
   // CUDA-graph replay of the whole forward (DIT_OPT_USE_GRAPH): one cached executable graph,
   // valid for the exact pointers and parameters it was captured with
   struct GraphKey {
@@ -637,6 +643,7 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
              make_tmap_e4m3_kmajor(&b.ta_fc2_8, b.fc2_w8, d, mlp, 128);
       else
         ok = ok && make_tmap_bf16_kmajor(&b.tm_fc1, b.fc1_w, mlp, d, g.bn_fc1) &&
+             make_tmap_bf16_kmajor(&b.tm_fc1_h, b.fc1_w, mlp, d, 128) &&
              make_tmap_bf16_kmajor(&b.ta_fc2, b.fc2_w, d, mlp, 128);
       if (cross)
         ok = ok && make_tmap_bf16_kmajor(&b.tm_xq, b.xq_w, d, d, 2 * g.dh) &&
@@ -846,8 +853,11 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
   };
   // gated residual update h += gate[row] * (A W^T + b) on the tensor cores (swapped operands)
   // or the SIMT GEMM
-  auto run_resid = [&](int kind, const CUtensorMap* ta, const CUtensorMap* tb, const void* A, const void* W, int K,
-                       const float* bias, const float* gate, int ld_gate, const char* where) -> dit_status {
+  // tb: the activations as the B operand (256-row box); tb_half: the same with a 128-row box
+  // for the SM-pair GEMM (nullptr: no pair variant)
+  auto run_resid = [&](int kind, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* tb_half,
+                       const void* A, const void* W, int K, const float* bias, const float* gate, int ld_gate,
+                       const char* where) -> dit_status {
     EpiArgs pa = {};
     pa.M = p.M;
     pa.N = d;
@@ -865,7 +875,11 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
       // short K (the d-wide projections): two K slices double the work units per SM, so
       // the pipeline fill and the last epilogue are no longer exposed
       pt.ksplit = K <= 2048 ? H->ksplit_short : 1;
-      DIT_LAUNCH(H, kind, st, launch_gemm_tc(EPI_RESID_T, 256, ta, tb, K, pt, H->num_sms, st, &H->tm_h_red), where);
+      if (H->pair_gemm && tb_half != nullptr)
+        DIT_LAUNCH(H, kind, st, launch_gemm_tc2(EPI_RESID_T, 256, ta, tb_half, K, pt, H->num_sms, st, &H->tm_h_red),
+                   where);
+      else
+        DIT_LAUNCH(H, kind, st, launch_gemm_tc(EPI_RESID_T, 256, ta, tb, K, pt, H->num_sms, st, &H->tm_h_red), where);
     } else {
       DIT_LAUNCH(H, kind, st,
                  launch_gemm_simt(EPI_RESID, static_cast<const float*>(A), static_cast<const float*>(W), p.M, d, K, pa, st),
@@ -941,8 +955,12 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
         EpiArgs qt = qa;  // swapped: rows = 3d output features, columns = tokens
         qt.M = 3 * d;
         qt.N = p.M;
-        DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_tc(EPI_QKV_T, 256, &b.ta_qkv, &H->tb_u, d, qt, H->num_sms, st),
-                   "qkv gemm");
+        if (H->pair_gemm)
+          DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_tc2(EPI_QKV_T, 256, &b.ta_qkv, &H->tm_u, d, qt, H->num_sms, st),
+                     "qkv gemm");
+        else
+          DIT_LAUNCH(H, DIT_KERNEL_QKV, st, launch_gemm_tc(EPI_QKV_T, 256, &b.ta_qkv, &H->tb_u, d, qt, H->num_sms, st),
+                     "qkv gemm");
       }
       DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_tc(aa, H->attn_maps, H->status, st), "attention");
     } else {
@@ -963,7 +981,8 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
       }
       DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_simt(aa, st), "attention");
     }
-    DIT_TRY(run_resid(DIT_KERNEL_PROJ, &b.ta_proj, &H->tb_o, H->o, b.proj_w, d, b.proj_b, gate1, ld_gate, "proj gemm"));
+    DIT_TRY(run_resid(DIT_KERNEL_PROJ, &b.ta_proj, &H->tb_o, &H->tm_o, H->o, b.proj_w, d, b.proj_b, gate1, ld_gate,
+                      "proj gemm"));
 
     if (g.kind == DIT_BLOCK_CROSS_ATTN) {  // h += CrossAttn(LNx(h), [e_t, e_y])
       DIT_TRY(run_ln(Norm{b.xln_b, b.xln_s, 0}, "cross-attention ln"));
@@ -1005,7 +1024,7 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
         xk.dh = g.dh;
         DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_xattn_f32(xk, st), "cross-attention");
       }
-      DIT_TRY(run_resid(DIT_KERNEL_PROJ, &b.ta_xo, &H->tb_o, H->o, b.xo_w, d, b.xo_b, H->ones, 0,
+      DIT_TRY(run_resid(DIT_KERNEL_PROJ, &b.ta_xo, &H->tb_o, &H->tm_o, H->o, b.xo_w, d, b.xo_b, H->ones, 0,
                         "cross-attention output gemm"));
     }
 
@@ -1064,15 +1083,21 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
     f1.ldo = mlp;
     f1.status = H->status;
     if (H->bf16) {
-      DIT_LAUNCH(H, DIT_KERNEL_FC1, st,
-                 launch_gemm_tc(EPI_GELU, g.bn_fc1, &H->tm_u, &b.tm_fc1, d, f1, H->num_sms, st, &H->tm_g_out),
-                 "fc1 gemm");
+      if (H->pair_gemm)
+        DIT_LAUNCH(H, DIT_KERNEL_FC1, st,
+                   launch_gemm_tc2(EPI_GELU, 256, &H->tm_u, &b.tm_fc1_h, d, f1, H->num_sms, st, &H->tm_g_out),
+                   "fc1 gemm");
+      else
+        DIT_LAUNCH(H, DIT_KERNEL_FC1, st,
+                   launch_gemm_tc(EPI_GELU, g.bn_fc1, &H->tm_u, &b.tm_fc1, d, f1, H->num_sms, st, &H->tm_g_out),
+                   "fc1 gemm");
     } else {
       DIT_LAUNCH(H, DIT_KERNEL_FC1, st, launch_gemm_simt(EPI_GELU, static_cast<const float*>(H->u), static_cast<const float*>(b.fc1_w), p.M,
                                  mlp, d, f1, st),
              "fc1 gemm");
     }
-    DIT_TRY(run_resid(DIT_KERNEL_FC2, &b.ta_fc2, &H->tb_g, H->gbuf, b.fc2_w, mlp, b.fc2_b, gate2, ld_gate, "fc2 gemm"));
+    DIT_TRY(run_resid(DIT_KERNEL_FC2, &b.ta_fc2, &H->tb_g, &H->tm_g, H->gbuf, b.fc2_w, mlp, b.fc2_b, gate2, ld_gate,
+                      "fc2 gemm"));
   }
   if (out == nullptr) return DIT_OK;
 
@@ -1239,6 +1264,14 @@ dit_status dit_set_option(dit_handle* H, int option, int value) {
   if (option == DIT_OPT_SPLIT_K) {
     if (value < 1 || value > 8) return fail(H, DIT_ERR_INVALID_ARG, "split-K must be 1..8");
     H->ksplit_short = value;
+    H->has_gseen = H->has_sseen = false;  // a new kernel configuration: recapture
+    if (H->gexec != nullptr) cudaGraphExecDestroy(H->gexec);
+    if (H->sexec != nullptr) cudaGraphExecDestroy(H->sexec);
+    H->gexec = H->sexec = nullptr;
+    return DIT_OK;
+  }
+  if (option == DIT_OPT_PAIR_GEMM) {
+    H->pair_gemm = value != 0;
     H->has_gseen = H->has_sseen = false;  // a new kernel configuration: recapture
     if (H->gexec != nullptr) cudaGraphExecDestroy(H->gexec);
     if (H->sexec != nullptr) cudaGraphExecDestroy(H->sexec);

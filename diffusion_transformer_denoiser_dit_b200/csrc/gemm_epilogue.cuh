@@ -424,6 +424,28 @@ __device__ __forceinline__ void epilogue_gelu8(const EpiArgs& ea, uint32_t tacc,
   }
 }
 
+// 32 consecutive tokens of one V^T row from registers, starting at a destination whose
+// offset from a 16-byte boundary is (8 - A) % 8 tokens: A scalar stores reach the boundary,
+// then 16-byte groups of 8 tokens, then the scalar tail.  A is a template argument so that the
+// register array is indexed with constants.
+template <int A>
+__device__ __forceinline__ void store_vt_row32(uint16_t* dst, const uint32_t* v, float bf) {
+#pragma unroll
+  for (int t = 0; t < A; ++t) dst[t] = f32_to_bf16(__uint_as_float(v[t]) + bf);
+#pragma unroll
+  for (int g = 0; A + 8 * g + 8 <= 32; ++g) {
+    const int t = A + 8 * g;
+    *reinterpret_cast<uint4*>(dst + t) =
+        make_uint4(pack_bf16x2(__uint_as_float(v[t + 0]) + bf, __uint_as_float(v[t + 1]) + bf),
+                   pack_bf16x2(__uint_as_float(v[t + 2]) + bf, __uint_as_float(v[t + 3]) + bf),
+                   pack_bf16x2(__uint_as_float(v[t + 4]) + bf, __uint_as_float(v[t + 5]) + bf),
+                   pack_bf16x2(__uint_as_float(v[t + 6]) + bf, __uint_as_float(v[t + 7]) + bf));
+  }
+  constexpr int tail = A + (32 - A) / 8 * 8;
+#pragma unroll
+  for (int t = tail; t < 32; ++t) dst[t] = f32_to_bf16(__uint_as_float(v[t]) + bf);
+}
+
 // Swapped-operand Q / K / V^T scatter: lane = output feature f of [q | k | v],
 // columns = tokens.  V^T rows are contiguous in tokens, so a lane writes 8 tokens per
 // 16-byte store; q and k are written one token per instruction (32 consecutive
@@ -452,20 +474,36 @@ __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc,
       const int r0 = tok0 / ea.T, t0 = tok0 - r0 * ea.T;
       const bool one_row = (last / ea.T) == r0 && last - tok0 == 31;
       if (which == 2) {
-        if (one_row && (t0 & 7) == 0) {
+        if (one_row) {  // V^T row segment of 32 tokens: 16-byte groups from the first aligned token on
           uint16_t* dst = static_cast<uint16_t*>(ea.v) + (static_cast<size_t>(r0 * ea.H + head) * ea.DP + j) * ea.Tpad + t0;
-#pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8)
-            reinterpret_cast<uint4*>(dst)[g8] =
-                make_uint4(pack_bf16x2(__uint_as_float(v[8 * g8 + 0]) + bf, __uint_as_float(v[8 * g8 + 1]) + bf),
-                           pack_bf16x2(__uint_as_float(v[8 * g8 + 2]) + bf, __uint_as_float(v[8 * g8 + 3]) + bf),
-                           pack_bf16x2(__uint_as_float(v[8 * g8 + 4]) + bf, __uint_as_float(v[8 * g8 + 5]) + bf),
-                           pack_bf16x2(__uint_as_float(v[8 * g8 + 6]) + bf, __uint_as_float(v[8 * g8 + 7]) + bf));
-        } else {
+          switch ((8 - (t0 & 7)) & 7) {
+            case 0: store_vt_row32<0>(dst, v, bf); break;
+            case 1: store_vt_row32<1>(dst, v, bf); break;
+            case 2: store_vt_row32<2>(dst, v, bf); break;
+            case 3: store_vt_row32<3>(dst, v, bf); break;
+            case 4: store_vt_row32<4>(dst, v, bf); break;
+            case 5: store_vt_row32<5>(dst, v, bf); break;
+            case 6: store_vt_row32<6>(dst, v, bf); break;
+            default: store_vt_row32<7>(dst, v, bf); break;
+          }
+        } else if (ea.T < 32) {  // short rows: a chunk spans several sample rows
           for (int t = 0; t < 32 && tok0 + t < ea.N; ++t) {
             const int rt = (tok0 + t) / ea.T, tt = tok0 + t - rt * ea.T;
             static_cast<uint16_t*>(ea.v)[(static_cast<size_t>(rt * ea.H + head) * ea.DP + j) * ea.Tpad + tt] =
                 f32_to_bf16(__uint_as_float(v[t]) + bf);
+          }
+        } else {  // the chunk crosses into the next sample row (or the end): split once, no divides
+          const int b = ea.T - t0;  // tokens of row r0 in the chunk
+          uint16_t* d0 = static_cast<uint16_t*>(ea.v) + (static_cast<size_t>(r0 * ea.H + head) * ea.DP + j) * ea.Tpad + t0;
+          uint16_t* d1 = static_cast<uint16_t*>(ea.v) + (static_cast<size_t>((r0 + 1) * ea.H + head) * ea.DP + j) * ea.Tpad;
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            if (tok0 + t >= ea.N) break;
+            const uint16_t val = f32_to_bf16(__uint_as_float(v[t]) + bf);
+            if (t < b)
+              d0[t] = val;
+            else
+              d1[t - b] = val;
           }
         }
       } else {
@@ -473,10 +511,23 @@ __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc,
           uint16_t* dst = qk + (static_cast<size_t>(r0 * ea.H + head) * ea.Tpad + t0) * ea.DP + j;
 #pragma unroll
           for (int t = 0; t < 32; ++t) dst[static_cast<size_t>(t) * ea.DP] = f32_to_bf16(__uint_as_float(v[t]) + bf);
-        } else {
+        } else if (ea.T < 32) {  // short rows: a chunk spans several sample rows
           for (int t = 0; t < 32 && tok0 + t < ea.N; ++t) {
             const int rt = (tok0 + t) / ea.T, tt = tok0 + t - rt * ea.T;
             qk[(static_cast<size_t>(rt * ea.H + head) * ea.Tpad + tt) * ea.DP + j] = f32_to_bf16(__uint_as_float(v[t]) + bf);
+          }
+        } else {  // the chunk crosses into the next sample row (or the end): split once, no divides
+          const int b = ea.T - t0;
+          uint16_t* d0 = qk + (static_cast<size_t>(r0 * ea.H + head) * ea.Tpad + t0) * ea.DP + j;
+          uint16_t* d1 = qk + static_cast<size_t>((r0 + 1) * ea.H + head) * ea.Tpad * ea.DP + j;
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            if (tok0 + t >= ea.N) break;
+            const uint16_t val = f32_to_bf16(__uint_as_float(v[t]) + bf);
+            if (t < b)
+              d0[static_cast<size_t>(t) * ea.DP] = val;
+            else
+              d1[static_cast<size_t>(t - b) * ea.DP] = val;
           }
         }
       }

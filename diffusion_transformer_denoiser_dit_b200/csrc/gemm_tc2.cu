@@ -279,6 +279,10 @@ cudaError_t launch_gemm_tc2(int epi, int bn, const CUtensorMap* tA, const CUtens
       break;
     case EPI_QKV_HEAD:
       DIT_BN2_CASE(128, EPI_QKV_HEAD) DIT_BN2_CASE(144, EPI_QKV_HEAD) break;
+    case EPI_RESID_T:
+      DIT_BN2_CASE(256, EPI_RESID_T) break;
+    case EPI_QKV_T:
+      DIT_BN2_CASE(256, EPI_QKV_T) break;
     default:
       break;
   }

@@ -30,36 +30,50 @@ __global__ void cond_sinusoid_kernel(const float* __restrict__ t, int B, int R, 
 
 // The condition MLP's two layers, out[r, j] = W[j] . in[r] + b[j] for all sample rows r:
 // a block of 8 warps owns 8 output features (one per warp) and a group of up to 32 rows
-// (lane = row).  The rows' inputs are staged in shared memory in K-chunks of 128, read once
-// per block; each lane loads 32 consecutive weights of its warp's feature at a time and hands
-// them round with shuffles, so a multiply-add costs a shuffle, a shared load and an FMA.
-constexpr int kCondK = 128;  // K-chunk staged per pass
+// (lane = row).  The group's whole input rows [32, K] are staged in shared memory at once
+// (every load in flight together; rows padded to K + 1 floats so the lanes' reads fall in
+// different banks); each lane loads 32 consecutive weights of its warp's feature at a time and
+// hands them round with shuffles, into four independent accumulators.
 constexpr int kCondRows = 32;
+
+// Stage rows are Kpad + 1 floats, Kpad = K rounded up to 32, zero past K (K % 4 == 0).
+__host__ __device__ inline int cond_stage_ld(int K) { return (K + 31) / 32 * 32 + 1; }
 
 __device__ __forceinline__ float cond_dot(const float* __restrict__ w, const float* __restrict__ in, int K, int r0,
                                           int nr, float* stage, int lane) {
-  float acc = 0.f;
-  for (int k0 = 0; k0 < K; k0 += kCondK) {
-    const int kn = min(kCondK, K - k0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < nr * kn; i += blockDim.x) {
-      const int rr = i / kn, kk = i - rr * kn;
-      stage[rr * (kCondK + 1) + kk] = in[static_cast<size_t>(r0 + rr) * K + k0 + kk];
-    }
-    __syncthreads();
-    for (int kb = 0; kb < kn; kb += 32) {
-      const float wl = kb + lane < kn ? __ldg(w + k0 + kb + lane) : 0.f;
-      const float* srow = stage + lane * (kCondK + 1) + kb;
-      const int kc = min(32, kn - kb);
-      if (kc == 32) {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) acc = fmaf(__shfl_sync(0xffffffffu, wl, q), srow[q], acc);
-      } else {
-        for (int q = 0; q < kc; ++q) acc = fmaf(__shfl_sync(0xffffffffu, wl, q), srow[q], acc);
-      }
-    }
+  __syncthreads();  // the previous row group's reads of the stage are done
+  const int ld = cond_stage_ld(K), K4 = K >> 2, Kpad = ld - 1;
+  for (int i = threadIdx.x; i < nr * K4; i += blockDim.x) {
+    const int rr = i / K4, k4 = i - rr * K4;
+    const float4 v = reinterpret_cast<const float4*>(in + static_cast<size_t>(r0 + rr) * K)[k4];
+    float* dst = stage + rr * ld + 4 * k4;
+    dst[0] = v.x;
+    dst[1] = v.y;
+    dst[2] = v.z;
+    dst[3] = v.w;
   }
-  return acc;
+  for (int i = threadIdx.x; i < kCondRows * (Kpad - K); i += blockDim.x) {  // zero tail of every row
+    const int rr = i / (Kpad - K);
+    stage[rr * ld + K + (i - rr * (Kpad - K))] = 0.f;
+  }
+  for (int i = threadIdx.x; i < (kCondRows - nr) * K; i += blockDim.x)  // rows past the group: zero
+    stage[(nr + i / K) * ld + i % K] = 0.f;
+  __syncthreads();
+  // the warp's whole weight row, lane l holding elements l, l + 32, ...: all loads in flight
+  // at once instead of one round trip per 32-wide step
+  constexpr int kMaxW = 1536 / 32;
+  float wreg[kMaxW];
+#pragma unroll
+  for (int i = 0; i < kMaxW; ++i) wreg[i] = (32 * i < Kpad && 32 * i + lane < K) ? __ldg(w + 32 * i + lane) : 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const float* srow = stage + lane * ld;
+#pragma unroll
+  for (int i = 0; i < kMaxW; ++i) {
+    if (32 * i >= Kpad) break;
+#pragma unroll
+    for (int q = 0; q < 32; ++q) acc[q & 3] = fmaf(__shfl_sync(0xffffffffu, wreg[i], q), srow[32 * i + q], acc[q & 3]);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
 // hid[r, j] = SiLU(W1[j] . E[r] + b1[j])
@@ -68,7 +82,7 @@ __global__ void __launch_bounds__(256) cond_hidden_kernel(const float* __restric
                                                           int K, int N) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float stage[kCondRows * (kCondK + 1)];
+  extern __shared__ float stage[];  // [32][K + 1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * 8 + warp;
   const int jc = j < N ? j : N - 1;  // every warp takes part in the block's staging barriers
@@ -85,7 +99,7 @@ __global__ void __launch_bounds__(256) cond_hidden_kernel(const float* __restric
 __global__ void __launch_bounds__(256) cond_out_kernel(CondArgs a) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float stage[kCondRows * (kCondK + 1)];
+  extern __shared__ float stage[];  // [32][d + 1]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * 8 + warp;
   const int jc = j < a.d ? j : a.d - 1;
@@ -138,15 +152,29 @@ __global__ void __launch_bounds__(256) cond_out_kernel(CondArgs a) {
 }
 
 cudaError_t launch_condition(const CondArgs& a, cudaStream_t st) {
+  if ((a.freq % 4) != 0 || (a.d % 4) != 0) return cudaErrorInvalidValue;
+  const size_t smem_h = static_cast<size_t>(kCondRows) * cond_stage_ld(a.freq) * sizeof(float);
+  const size_t smem_o = static_cast<size_t>(kCondRows) * cond_stage_ld(a.d) * sizeof(float);
+  static bool attr_done[kMaxDevices] = {};
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {  // the largest stage the library's limits allow (d, freq_dim <= 1536)
+    const int mx = static_cast<int>(static_cast<size_t>(kCondRows) * cond_stage_ld(1536) * sizeof(float));
+    cudaError_t e = cudaFuncSetAttribute(cond_hidden_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(cond_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  if (a.freq > 1536 || a.d > 1536) return cudaErrorInvalidValue;
   const int n = a.R * a.freq;
   cudaError_t e = launch_kernel(cond_sinusoid_kernel, dim3((n + 255) / 256), dim3(256), 0, st, a.t, a.B, a.R, a.freq,
                                  a.t_scale, a.E);
   if (e != cudaSuccess) return e;
   const int rg = (a.R + kCondRows - 1) / kCondRows;
-  e = launch_kernel(cond_hidden_kernel, dim3((a.d + 7) / 8, rg), dim3(256), 0, st, (const float*)a.E, a.w1, a.b1,
+  e = launch_kernel(cond_hidden_kernel, dim3((a.d + 7) / 8, rg), dim3(256), smem_h, st, (const float*)a.E, a.w1, a.b1,
                     a.hid, a.R, a.freq, a.d);
   if (e != cudaSuccess) return e;
-  return launch_kernel(cond_out_kernel, dim3((a.d + 7) / 8, rg), dim3(256), 0, st, a);
+  return launch_kernel(cond_out_kernel, dim3((a.d + 7) / 8, rg), dim3(256), smem_o, st, a);
 }
 
 // ============================================================================ patch embed
@@ -193,118 +221,106 @@ __global__ void patch_embed_kernel(PatchArgs a) {
   }
 }
 
-// Fast path (Kp <= 256, d <= 1536, d % 4 == 0): one warp per pair of tokens of the B unique
-// samples.  Lane l holds patch elements l, l+32, ... of both tokens and broadcasts them with
-// shuffles; it accumulates output features 4(l + 32i) .. +3 from the transposed weights
-// [Kp, d] (coalesced 16-byte loads, shared by the two tokens), then adds bias and position
-// and stores whole 16-byte groups to row b and, when guided, to row B + b as well.
-constexpr int kPeMaxVec = 12;   // float4 groups per lane: d <= 32 * 4 * 12 = 1536
-constexpr int kPeMaxKv = 8;     // patch elements per lane: Kp <= 256
-__global__ void __launch_bounds__(256) patch_embed_pairs_kernel(PatchArgs a) {
+// Tiled path: a block computes 32 tokens (of the B unique samples) x 128 output features.
+// The tokens' patch vectors and the block's slice of the transposed weights [Kp, d] are
+// staged in shared memory in K-chunks of 32; each thread accumulates 4 features x 4 tokens
+// (one 16-byte weight load and four broadcast patch loads per 16 multiply-adds), then adds
+// bias and position and stores 16-byte groups to row b and, when guided, to row B + b.
+constexpr int kPeTok = 32, kPeFeat = 128, kPeK = 32;
+__global__ void __launch_bounds__(256) patch_embed_tiled_kernel(PatchArgs a) {
   pdl_trigger();
   pdl_wait();
+  __shared__ float sx[kPeK][kPeTok + 1];        // patch element k of token t
+  __shared__ __align__(16) float sw[kPeK][kPeFeat];  // weight (k, feature)
   const int gh = a.H / a.ph, gw = a.W / a.pw, gf = a.F / a.pt;
   const int T = gf * gh * gw;
   const int Kp = a.C * a.pt * a.ph * a.pw;
-  const int lane = threadIdx.x & 31;
-  const int nvec = (a.d + 127) / 128;
-  const long long units = static_cast<long long>(a.B) * T;  // unique tokens
-  const long long pairs = (units + 1) / 2;
-  const long long gwarp = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long pr = gwarp; pr < pairs; pr += nwarps) {
-    float xv[2][kPeMaxKv];
-    int tb[2], ttau[2];
-    bool live[2];
+  __shared__ int tok_off[kPeTok];   // offset in x of each token's patch corner (-1: past the end)
+  __shared__ int k_off[kPeK];       // offset of each patch element from the corner
+  const int units = a.B * T;        // the launcher checks that x and the unit count fit 31 bits
+  const int u0 = blockIdx.x * kPeTok;
+  const int f0 = blockIdx.y * kPeFeat;
+  const int fq = threadIdx.x & 31;   // feature quad: features f0 + 4 fq .. + 3
+  const int tq = threadIdx.x >> 5;   // token quad: tokens u0 + 4 tq .. + 3
+  if (threadIdx.x < kPeTok) {
+    const int u = u0 + threadIdx.x;
+    int off = -1;
+    if (u < units) {
+      const int b = u / T, tau = u - b * T;
+      const int f = tau / (gh * gw), ii = (tau / gw) % gh, jj = tau % gw;
+      off = ((b * a.C * a.F + f * a.pt) * a.H + ii * a.ph) * a.W + jj * a.pw;
+    }
+    tok_off[threadIdx.x] = off;
+  }
+  float4 acc[4];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const long long id = 2 * pr + u;
-      live[u] = id < units;
-      const long long idc = live[u] ? id : units - 1;
-      tb[u] = static_cast<int>(idc / T);
-      ttau[u] = static_cast<int>(idc - static_cast<long long>(tb[u]) * T);
-      const int f = ttau[u] / (gh * gw), i = (ttau[u] / gw) % gh, jj = ttau[u] % gw;
+  for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < Kp; k0 += kPeK) {
+    const int kn = min(kPeK, Kp - k0);
+    __syncthreads();
+    if (threadIdx.x < kPeK) {
+      const int k = k0 + threadIdx.x;
+      const int iw = k % a.pw, ih = (k / a.pw) % a.ph, it = (k / (a.pw * a.ph)) % a.pt, c = k / (a.pw * a.ph * a.pt);
+      k_off[threadIdx.x] = ((c * a.F + it) * a.H + ih) * a.W + iw;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kPeK * kPeTok; i += blockDim.x) {  // gather patch elements
+      const int t = i >> 5, kk = i & 31;  // kPeK == 32
+      const int to = tok_off[t];
+      sx[kk][t] = (kk < kn && to >= 0) ? __ldg(a.x + to + k_off[kk]) : 0.f;
+    }
+    for (int i = threadIdx.x; i < kPeK * (kPeFeat / 4); i += blockDim.x) {  // weight slice
+      const int kk = i / (kPeFeat / 4), q = i - kk * (kPeFeat / 4);
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (kk < kn && f0 + 4 * q < a.d)
+        w = __ldg(reinterpret_cast<const float4*>(a.wt + static_cast<size_t>(k0 + kk) * a.d + f0) + q);
+      reinterpret_cast<float4*>(&sw[kk][0])[q] = w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kn; ++kk) {
+      const float4 w = reinterpret_cast<const float4*>(&sw[kk][0])[fq];
 #pragma unroll
-      for (int kk = 0; kk < kPeMaxKv; ++kk) {
-        const int k = kk * 32 + lane;
-        float v = 0.f;
-        if (k < Kp) {
-          const int iw = k % a.pw, ih = (k / a.pw) % a.ph, it = (k / (a.pw * a.ph)) % a.pt, c = k / (a.pw * a.ph * a.pt);
-          const size_t xi = ((((static_cast<size_t>(tb[u]) * a.C + c) * a.F + f * a.pt + it) * a.H + i * a.ph + ih) *
-                             a.W) + jj * a.pw + iw;
-          v = __ldg(a.x + xi);
-        }
-        xv[u][kk] = v;
+      for (int i = 0; i < 4; ++i) {
+        const float xv = sx[kk][4 * tq + i];
+        acc[i].x = fmaf(xv, w.x, acc[i].x);
+        acc[i].y = fmaf(xv, w.y, acc[i].y);
+        acc[i].z = fmaf(xv, w.z, acc[i].z);
+        acc[i].w = fmaf(xv, w.w, acc[i].w);
       }
     }
-    float4 acc[2][kPeMaxVec];
+  }
+  const int f = f0 + 4 * fq;
+  if (f >= a.d) return;
+  const int Tr = a.Trow ? a.Trow : T;
+  const float4 bb = __ldg(reinterpret_cast<const float4*>(a.b + f));
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
-#pragma unroll
-      for (int i = 0; i < kPeMaxVec; ++i) acc[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int kk = 0; kk < kPeMaxKv; ++kk) {
-      if (kk * 32 >= Kp) break;
-      const int kn = min(32, Kp - kk * 32);
-      for (int kl = 0; kl < kn; ++kl) {
-        const float x0 = __shfl_sync(0xffffffffu, xv[0][kk], kl);
-        const float x1 = __shfl_sync(0xffffffffu, xv[1][kk], kl);
-        const float4* wr = reinterpret_cast<const float4*>(a.wt + static_cast<size_t>(kk * 32 + kl) * a.d);
-#pragma unroll
-        for (int i = 0; i < kPeMaxVec; ++i) {
-          const int c4 = lane + 32 * i;
-          if (i < nvec && 4 * c4 < a.d) {
-            const float4 w = __ldg(wr + c4);
-            acc[0][i].x = fmaf(x0, w.x, acc[0][i].x);
-            acc[0][i].y = fmaf(x0, w.y, acc[0][i].y);
-            acc[0][i].z = fmaf(x0, w.z, acc[0][i].z);
-            acc[0][i].w = fmaf(x0, w.w, acc[0][i].w);
-            acc[1][i].x = fmaf(x1, w.x, acc[1][i].x);
-            acc[1][i].y = fmaf(x1, w.y, acc[1][i].y);
-            acc[1][i].z = fmaf(x1, w.z, acc[1][i].z);
-            acc[1][i].w = fmaf(x1, w.w, acc[1][i].w);
-          }
-        }
-      }
+  for (int i = 0; i < 4; ++i) {
+    const int u = u0 + 4 * tq + i;
+    if (u >= units) break;
+    const int b = u / T, tau = u - b * T;
+    float4 v = make_float4(acc[i].x + bb.x, acc[i].y + bb.y, acc[i].z + bb.z, acc[i].w + bb.w);
+    if (a.pos) {
+      const float4 pp = __ldg(reinterpret_cast<const float4*>(a.pos + static_cast<size_t>(tau) * a.d + f));
+      v.x += pp.x;
+      v.y += pp.y;
+      v.z += pp.z;
+      v.w += pp.w;
     }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      if (!live[u]) continue;
-      const float4* pos = a.pos ? reinterpret_cast<const float4*>(a.pos + static_cast<size_t>(ttau[u]) * a.d) : nullptr;
-      const int Tr = a.Trow ? a.Trow : T;
-      float4* h0 = reinterpret_cast<float4*>(a.h + (static_cast<size_t>(tb[u]) * Tr + a.tok0 + ttau[u]) * a.d);
-      float4* h1 = reinterpret_cast<float4*>(a.h + (static_cast<size_t>(tb[u] + a.B) * Tr + a.tok0 + ttau[u]) * a.d);
-      const bool dup = a.R > a.B;
-#pragma unroll
-      for (int i = 0; i < kPeMaxVec; ++i) {
-        const int c4 = lane + 32 * i;
-        if (i < nvec && 4 * c4 < a.d) {
-          const float4 bb = __ldg(reinterpret_cast<const float4*>(a.b) + c4);
-          float4 v = make_float4(acc[u][i].x + bb.x, acc[u][i].y + bb.y, acc[u][i].z + bb.z, acc[u][i].w + bb.w);
-          if (pos) {
-            const float4 pp = __ldg(pos + c4);
-            v.x += pp.x;
-            v.y += pp.y;
-            v.z += pp.z;
-            v.w += pp.w;
-          }
-          h0[c4] = v;
-          if (dup) h1[c4] = v;
-        }
-      }
-    }
+    *reinterpret_cast<float4*>(a.h + (static_cast<size_t>(b) * Tr + a.tok0 + tau) * a.d + f) = v;
+    if (a.R > a.B) *reinterpret_cast<float4*>(a.h + (static_cast<size_t>(b + a.B) * Tr + a.tok0 + tau) * a.d + f) = v;
   }
 }
 
 cudaError_t launch_patch_embed(const PatchArgs& a, cudaStream_t st) {
   const int T = (a.F / a.pt) * (a.H / a.ph) * (a.W / a.pw);
   const int Kp = a.C * a.pt * a.ph * a.pw;
-  if (a.wt != nullptr && Kp <= 32 * kPeMaxKv && a.d <= 128 * kPeMaxVec && (a.d & 3) == 0 && (a.R == a.B || a.R == 2 * a.B)) {
-    const long long pairs = (static_cast<long long>(a.B) * T + 1) / 2;
-    const long long blocks = (pairs + 7) / 8;
-    const int grid = static_cast<int>(blocks < 148LL * 8 ? blocks : 148LL * 8);
-    if (grid == 0) return cudaSuccess;
-    return launch_kernel(patch_embed_pairs_kernel, dim3(grid), dim3(256), 0, st, a);
+  const long long xsize = static_cast<long long>(a.B) * a.C * a.F * a.H * a.W;
+  if (a.wt != nullptr && (a.d & 3) == 0 && (a.R == a.B || a.R == 2 * a.B) && xsize < (1LL << 31)) {
+    const long long units = static_cast<long long>(a.B) * T;
+    const dim3 grid(static_cast<unsigned>((units + kPeTok - 1) / kPeTok), (a.d + kPeFeat - 1) / kPeFeat);
+    if (units == 0) return cudaSuccess;
+    return launch_kernel(patch_embed_tiled_kernel, grid, dim3(256), 0, st, a);
   }
   const size_t smem = static_cast<size_t>(kPatchTok) * Kp * sizeof(float);
   if (smem > 48 * 1024) {

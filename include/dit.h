@@ -93,7 +93,7 @@ typedef struct dit_config {
   int cond_kind;      /* DIT_COND_CLASS: label table of num_classes+1 rows (last = null);
                          DIT_COND_VECTOR: caller passes a float32 vector of width d per sample */
   int num_classes;    /* 1000 for ImageNet; the null label is num_classes */
-  int freq_dim;       /* width of the timestep sinusoid (256) */
+  int freq_dim;       /* width of the timestep sinusoid (256; a multiple of 4, at most 1536) */
   int max_batch;      /* largest user batch B; device workspace is sized for 2*max_batch rows */
   float t_scale;      /* the sinusoid sees t * t_scale (1 for integer steps, 1000 for t in [0,1)) */
   int block_kind;     /* DIT_BLOCK_* (0 = adaLN-Zero, the design of the standard DiT models) */
@@ -249,11 +249,16 @@ void dit_destroy(dit_handle* h);
    time grows by that kind's in-pipeline cost (the second launch repeats the same work on the
    same buffers; for the residual kinds DIT_KERNEL_PROJ and DIT_KERNEL_FC2 it adds the update
    twice, so outputs are meaningless while it is on).  Part of the graph cache key.
-   DIT_OPT_SPLIT_K = s (1..8, default 2): the residual GEMMs with a short reduction (the
+   DIT_OPT_SPLIT_K = s (1..8, default 1): the residual GEMMs with a short reduction (the
    d-wide out-projections) split K into s slices, each adding its share into the residual
-   stream (the results differ from s = 1 only in float32 summation order). */
+   stream.  The slices' additions reach memory in no fixed order, so with s > 1 repeated
+   forwards may differ in float32 rounding (not bit-identical); s = 1 is deterministic.
+   DIT_OPT_PAIR_GEMM = 0/1 (default 0): run the bf16 block GEMMs (QKV without QK norm / RoPE,
+   out-projection, FFN) on SM pairs, tcgen05.mma.cta_group::2 with 256 x 256 tiles: each SM
+   loads its 128 rows of A and half of B per stage (32 KB instead of 48 KB), so six stages fit
+   instead of four.  The split-K option does not apply to the pair kernels. */
 enum { DIT_OPT_FORCE_GUIDANCE = 1, DIT_OPT_USE_GRAPH = 2, DIT_OPT_OVERLAP_LAUNCH = 3, DIT_OPT_CFG_CHANNELS = 4,
-       DIT_OPT_REPEAT_KIND = 5, DIT_OPT_SPLIT_K = 6 };
+       DIT_OPT_REPEAT_KIND = 5, DIT_OPT_SPLIT_K = 6, DIT_OPT_PAIR_GEMM = 7 };
 dit_status dit_set_option(dit_handle* h, int option, int value);
 
 /*
@@ -321,8 +326,8 @@ dit_status dit_profile_read(dit_handle* h, float* total_ms, int* launches);
  *   guided = 1 appends B rows with the null label (class models only);
  *   c_out dev f32 [rows, hidden]; status dev int32 (or NULL) receives DIT_ERR_BAD_LABEL
  *   when a label lies outside [0, num_classes] (the label is clamped).
- * Limits of the fixed scratch: rows <= 128, freq_dim <= 512, hidden <= 1536; larger
- * requests return DIT_ERR_INVALID_ARG before anything is launched.  The array
+ * Limits of the fixed scratch: rows <= 128, freq_dim <= 512, hidden <= 1536 (both multiples
+ * of 4); other requests return DIT_ERR_INVALID_ARG before anything is launched.  The array
  * (1.75 MiB) stays resident on every GPU that loaded the library until the process
  * exits.  The first call on a device looks up the array's device address (once per
  * device, with that device current; again after a device reset gives the device a new

@@ -436,7 +436,9 @@ def test_guidance_on_the_first_channels_only():
 
 def test_split_k_residual_gemms_match_unsplit():
     """DIT_OPT_SPLIT_K: the out-projection's K slices each add their share into the residual
-    stream; any split gives the unsplit result up to float32 summation order, and parity."""
+    stream; any split gives the unsplit result up to float32 summation order, and parity.
+    A reordered float32 sum can flip the bf16 rounding of a later activation (2^-9 relative),
+    so two splits agree to about 1e-3, not to float32 precision."""
     cfg = small_image_bf16_dh72()
     W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
     inp = S.make_inputs(cfg)
@@ -448,8 +450,29 @@ def test_split_k_residual_gemms_match_unsplit():
         outs[sk] = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
     assert m.sync_status() == binding.DIT_OK
     for sk in (2, 3, 8):
-        assert metrics(outs[sk], outs[1])[0] < 1e-4, sk
+        assert metrics(outs[sk], outs[1])[0] < 5e-3, sk
     assert_parity(cfg, outs[2], O.forward(cfg, W, inp["x"], inp["t"], inp["y"]), "split-K 2")
     with pytest.raises(binding.DitError):
         m.set_option(binding.DIT_OPT_SPLIT_K, 0)
+    m.close()
+
+
+@pytest.mark.parametrize("name", ["img_bf16_dh72", "b4_bf16_full", "video_bf16", "img_bf16_dh64_ragged"])
+def test_pair_gemm_forward_parity(name):
+    """DIT_OPT_PAIR_GEMM: the block GEMMs on SM pairs (cta_group::2, 256-row tiles, ragged
+    token counts included) match the oracle, and graph replay of that forward is bit-identical."""
+    cfg = SMALL[name]()
+    W = S.set_adaln(cfg, S.make_weights(cfg), gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    m = DiT(cfg, W)
+    m.set_option(binding.DIT_OPT_PAIR_GEMM, 1)
+    d = dev(inp)
+    got = m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale).cpu().numpy()
+    assert m.sync_status() == binding.DIT_OK
+    assert_parity(cfg, got, O.forward(cfg, W, inp["x"], inp["t"], inp["y"]), f"pair {name}")
+    m.set_option(binding.DIT_OPT_USE_GRAPH, 1)
+    out = torch.empty(cfg.out_shape(), device="cuda")
+    for _ in range(3):
+        m.forward(d["x"], d["t"], d["y"], cfg.cfg_scale, out=out)
+    assert np.array_equal(out.cpu().numpy(), got)
     m.close()
