@@ -259,29 +259,31 @@ __device__ __forceinline__ void epilogue_cols(const EpiArgs& ea, uint32_t tacc, 
 }
 
 // Epilogues that write through shared memory, each warp in its own 4 KB staging
-// buffer: GELU stages a 32-row x 32-column bf16 chunk and writes it back out with plain
-// coalesced 16-byte stores (whole 64-byte row segments instead of 32 scattered pieces
-// per instruction); RESID_T stages [token][feature] boxes that one lane hands to the
-// TMA unit as a float32 reduce-add into the residual stream, so the SM never reads the
-// stream back.
+// buffer: GELU and the swapped Q / K / V^T scatter stage 32 x 32 bf16 chunks and write
+// them back out with plain coalesced 16-byte stores, whole 64-byte row segments instead
+// of 32 scattered pieces per instruction; RESID_T stages [token][feature] boxes that one
+// lane hands to the TMA unit as a float32 reduce-add into the residual stream, so the SM
+// never reads the stream back (plain loads and stores of the stream, or red.global.add,
+// slow the concurrent main loop more).
 template <int EPI>
 __host__ __device__ constexpr bool epi_staged() {
-  return EPI == EPI_GELU || EPI == EPI_RESID_T || EPI == EPI_RESID_T8;
+  return EPI == EPI_GELU || EPI == EPI_RESID_T || EPI == EPI_RESID_T8 || EPI == EPI_QKV_T;
 }
 constexpr int kStageBytesPerWarp = 4096;
 constexpr int kEpilogueWarps = 8;
 
-// GELU epilogue through shared memory: each 32-row x 32-column chunk is written to
-// the warp's staging buffer as rows of 64 bytes (bf16), with the 16-byte groups of row
-// r rotated by ((r >> 1) & 3) so the 32 lanes' row writes do not collide on banks,
-// then read back so that 4 consecutive lanes cover one 64-byte output row: each store
-// instruction writes 8 whole row segments instead of 32 scattered pieces.
+// GELU epilogue through shared memory: two 32-column chunks (64 columns, 128 bytes of
+// bf16 per row) are written to the warp's 4 KB staging buffer as 32 rows of 128 bytes, the
+// 16-byte group g of row r stored at g ^ (r & 7) so that the lanes' row writes and the
+// read-back both spread over all banks, then read back so that 8 consecutive lanes cover
+// one whole 128-byte output line: each store instruction writes 4 full lines.  Whole
+// lines keep the store requests the epilogue sends to L2 few, which matters because they
+// share the SM's path to L2 with the main loop's TMA loads of the next tile.
 template <int NC, int EPI>
-__device__ __forceinline__ void epilogue_cols_staged(const EpiArgs& ea, const CUtensorMap* tmC, uint32_t tacc,
-                                                     int m_base, int lane, int n0, int c0, uint8_t* stg) {
+__device__ __forceinline__ void epilogue_cols_staged(const EpiArgs& ea, uint32_t tacc, int m_base, int lane, int n0,
+                                                     int c0, uint8_t* stg) {
   static_assert(EPI == EPI_GELU, "staged row-major epilogue is the GELU output");
-  static_assert(NC % 32 == 0, "staged epilogues work on 32-column chunks");
-  (void)tmC;
+  static_assert(NC % 64 == 0, "staged epilogues work on 64-column pieces");
   constexpr int NCH = NC / 32;
   uint32_t r[2][32];
   tmem_ld_chunk<32>(tacc + c0, r[0]);
@@ -290,7 +292,9 @@ __device__ __forceinline__ void epilogue_cols_staged(const EpiArgs& ea, const CU
   for (int c = 0; c < NCH; ++c) {
     if (c + 1 < NCH) tmem_ld_chunk<32>(tacc + c0 + (c + 1) * 32, r[(c + 1) & 1]);
     const int n = n0 + c0 + c * 32;
+    const int h = c & 1;  // which half of the 64-column piece
     const uint32_t* v = r[c & 1];
+    if (h == 0) __syncwarp();  // every lane is done reading the previous piece
     if (n < ea.N) {
 #pragma unroll
       for (int c16 = 0; c16 < 4; ++c16) {
@@ -305,18 +309,20 @@ __device__ __forceinline__ void epilogue_cols_staged(const EpiArgs& ea, const CU
                            gelu_tanh_fast(__uint_as_float(v[8 * c16 + 5]) + b1.y));
         pk.w = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 6]) + b1.z),
                            gelu_tanh_fast(__uint_as_float(v[8 * c16 + 7]) + b1.w));
-        *reinterpret_cast<uint4*>(stg + lane * 64 + ((c16 ^ ((lane >> 1) & 3)) << 4)) = pk;
+        *reinterpret_cast<uint4*>(stg + lane * 128 + (((h * 4 + c16) ^ (lane & 7)) << 4)) = pk;
       }
+    }
+    if (h == 1) {
       __syncwarp();
+      const int np = n - 32;  // first column of the piece
 #pragma unroll
-      for (int it = 0; it < 4; ++it) {  // 8 rows x 64 bytes per instruction
-        const int rr = it * 8 + (lane >> 2), c16 = lane & 3;
-        const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((c16 ^ ((rr >> 1) & 3)) << 4));
-        const int m = m_base + rr;
-        if (m < ea.M)
-          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n + c16 * 8) = val;
+      for (int it = 0; it < 8; ++it) {  // 4 rows x 128 bytes per instruction
+        const int rr = it * 4 + (lane >> 3), g = lane & 7;
+        const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((g ^ (rr & 7)) << 4));
+        const int m = m_base + rr, col = np + g * 8;
+        if (m < ea.M && col < ea.N)
+          *reinterpret_cast<uint4*>(static_cast<uint16_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + col) = val;
       }
-      __syncwarp();
     }
     if (c + 1 < NCH) tmem_ld_wait<32>(r[(c + 1) & 1]);
   }
@@ -447,11 +453,18 @@ __device__ __forceinline__ void store_vt_row32(uint16_t* dst, const uint32_t* v,
 }
 
 // Swapped-operand Q / K / V^T scatter: lane = output feature f of [q | k | v],
-// columns = tokens.  V^T rows are contiguous in tokens, so a lane writes 8 tokens per
-// 16-byte store; q and k are written one token per instruction (32 consecutive
-// head-dim entries across the lanes).
+// columns = tokens.  A chunk of 32 features x 32 tokens normally goes through the warp's
+// staging buffer so that each global store instruction writes eight whole 64-byte
+// segments: q and k are staged [token][feature] (one token's 32 features, contiguous in
+// the head-major layout except at a head boundary, which falls between 16-byte groups
+// because the head dim is a multiple of 8), V^T is staged [feature][token] (32
+// consecutive tokens of one V^T row, 16-byte groups of row r rotated by (r >> 1) & 3).
+// Chunks that straddle two sample rows, V^T chunks that start off a 16-byte boundary and
+// widths d that are not a multiple of 32 are written lane by lane instead: V^T as 16-byte
+// groups of 8 tokens, q and k one token per instruction.
 template <int NC>
-__device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc, int f_base, int lane, int n0, int c0) {
+__device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc, int f_base, int lane, int n0, int c0,
+                                               uint8_t* stg) {
   static_assert(NC % 32 == 0, "32-token chunks");
   constexpr int NCH = NC / 32;
   const int f = f_base + lane;
@@ -461,6 +474,22 @@ __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc,
   const int head = within / ea.dh, j = within - head * ea.dh;
   const float bf = fok ? __ldg(ea.bias + f) : 0.f;
   uint16_t* qk = static_cast<uint16_t*>(which == 0 ? ea.q : ea.k);
+  // staging: all 32 features of the warp are q, all k or all v
+  const bool warp_one_kind = (ea.d & 31) == 0 && f_base + 31 < ea.M;
+  int gh = 0, gj = 0;  // q / k read-back: head and offset of this lane's 8-feature group (lane & 3)
+  int vh[4] = {0, 0, 0, 0}, vj[4] = {0, 0, 0, 0};  // V^T read-back: feature row it * 8 + (lane >> 2)
+  if (warp_one_kind) {
+    const int wbase = f_base - (f_base / ea.d) * ea.d;
+    const int wg = wbase + 8 * (lane & 3);
+    gh = wg / ea.dh;
+    gj = wg - gh * ea.dh;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int wf = wbase + it * 8 + (lane >> 2);
+      vh[it] = wf / ea.dh;
+      vj[it] = wf - vh[it] * ea.dh;
+    }
+  }
   uint32_t r[2][32];
   tmem_ld_chunk<32>(tacc + c0, r[0]);
   tmem_ld_wait<32>(r[0]);
@@ -473,7 +502,42 @@ __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc,
       const int last = min(tok0 + 31, ea.N - 1);
       const int r0 = tok0 / ea.T, t0 = tok0 - r0 * ea.T;
       const bool one_row = (last / ea.T) == r0 && last - tok0 == 31;
-      if (which == 2) {
+      if (warp_one_kind && one_row && (which < 2 || (t0 & 7) == 0)) {
+        uint8_t* buf = stg + (c & 1) * 2048;
+        __syncwarp();  // every lane is done reading this buffer's previous chunk
+        if (which == 2) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t* w = v + 8 * g;
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(w[0]) + bf, __uint_as_float(w[1]) + bf),
+                           pack_bf16x2(__uint_as_float(w[2]) + bf, __uint_as_float(w[3]) + bf),
+                           pack_bf16x2(__uint_as_float(w[4]) + bf, __uint_as_float(w[5]) + bf),
+                           pack_bf16x2(__uint_as_float(w[6]) + bf, __uint_as_float(w[7]) + bf));
+          }
+          __syncwarp();
+          uint16_t* vb = static_cast<uint16_t*>(ea.v) + static_cast<size_t>(r0 * ea.H) * ea.DP * ea.Tpad + t0 +
+                         8 * (lane & 3);
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int rr = it * 8 + (lane >> 2), g = lane & 3;
+            const uint4 val = *reinterpret_cast<const uint4*>(buf + rr * 64 + ((g ^ ((rr >> 1) & 3)) << 4));
+            *reinterpret_cast<uint4*>(vb + (static_cast<size_t>(vh[it]) * ea.DP + vj[it]) * ea.Tpad) = val;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            *reinterpret_cast<uint16_t*>(buf + t * 64 + lane * 2) = f32_to_bf16(__uint_as_float(v[t]) + bf);
+          __syncwarp();
+          uint16_t* qb = qk + (static_cast<size_t>(r0 * ea.H + gh) * ea.Tpad + t0) * ea.DP + gj;
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int tt = it * 8 + (lane >> 2);
+            *reinterpret_cast<uint4*>(qb + static_cast<size_t>(tt) * ea.DP) =
+                *reinterpret_cast<const uint4*>(buf + tt * 64 + (lane & 3) * 16);
+          }
+        }
+      } else if (which == 2) {
         if (one_row) {  // V^T row segment of 32 tokens: 16-byte groups from the first aligned token on
           uint16_t* dst = static_cast<uint16_t*>(ea.v) + (static_cast<size_t>(r0 * ea.H + head) * ea.DP + j) * ea.Tpad + t0;
           switch ((8 - (t0 & 7)) & 7) {

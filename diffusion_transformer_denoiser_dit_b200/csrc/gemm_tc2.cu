@@ -185,9 +185,10 @@ __global__ void __launch_bounds__(320, 1)
         epilogue_resid_t<BN / 2>(ea, &tmC, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
                                  staging + (warp - 2) * kStageBytesPerWarp);
       else if constexpr (EPI == EPI_QKV_T)
-        epilogue_qkv_t<BN / 2>(ea, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2));
+        epilogue_qkv_t<BN / 2>(ea, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
+                               staging + (warp - 2) * kStageBytesPerWarp);
       else if constexpr (epi_staged<EPI>())
-        epilogue_cols_staged<BN / 2, EPI>(ea, &tmC, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
+        epilogue_cols_staged<BN / 2, EPI>(ea, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
                                           staging + (warp - 2) * kStageBytesPerWarp);
       else
         epilogue_cols<BN / 2, (EPI == EPI_QKV_HEAD ? EPI_QKV : EPI), EPI == EPI_QKV_HEAD || EPI == EPI_XATTN>(
@@ -269,7 +270,7 @@ cudaError_t launch_gemm_tc2(int epi, int bn, const CUtensorMap* tA, const CUtens
       DIT_BN2_CASE(64, EPI_F32) DIT_BN2_CASE(128, EPI_F32) DIT_BN2_CASE(144, EPI_F32) DIT_BN2_CASE(192, EPI_F32)
       DIT_BN2_CASE(256, EPI_F32) break;
     case EPI_GELU:
-      DIT_BN2_CASE(128, EPI_GELU) DIT_BN2_CASE(192, EPI_GELU) DIT_BN2_CASE(256, EPI_GELU)
+      DIT_BN2_CASE(128, EPI_GELU) DIT_BN2_CASE(256, EPI_GELU)
       break;
     case EPI_RESID:
       DIT_BN2_CASE(128, EPI_RESID) DIT_BN2_CASE(192, EPI_RESID)

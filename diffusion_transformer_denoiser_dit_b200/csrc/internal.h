@@ -19,7 +19,7 @@ enum Epi : int {
   // Swapped operands (A = weights, B = activations: GEMM rows are output features,
   // GEMM columns are tokens; ea.M = features, ea.N = tokens):
   EPI_RESID_T = 6,   // h[tok, f] += gate[row(tok), f] * (acc + bias[f])   (TMA reduce-add)
-  EPI_QKV_T = 7,     // q, k, v^T scatter, column by column
+  EPI_QKV_T = 7,     // q, k, v^T scatter, 32 x 32 chunks staged through shared memory
   // Cross-attention onto a two-token condition sequence, fused into the query projection:
   // tile = 2 heads; each thread holds one token's query for one head, scores it against the
   // two keys, and writes the softmax mix of the two values to o [M, d] (bf16).
