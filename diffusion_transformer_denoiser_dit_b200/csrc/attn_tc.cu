@@ -34,6 +34,14 @@
 
 namespace dit {
 
+// One pair of probabilities in every kEx2PolyEvery is exponentiated with a polynomial on
+// the FMA pipe (ex2_poly_f2) instead of the MUFU unit, which the exponentials and the bf16
+// conversions otherwise saturate; 0 turns it off.
+#ifndef DIT_EX2_POLY_EVERY
+#define DIT_EX2_POLY_EVERY 4
+#endif
+constexpr int kEx2PolyEvery = DIT_EX2_POLY_EVERY > 0 ? DIT_EX2_POLY_EVERY : 1 << 30;
+
 template <int DH>
 struct AttnCfg {
   static constexpr int DP = (DH + 15) / 16 * 16;
@@ -349,10 +357,18 @@ __global__ void __launch_bounds__(384, 1)
         uint64_t rs2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          rs2[i & 1] = f2_add(rs2[i & 1], f2_pack(p0, p1));
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2);
+          uint64_t p2;
+          if (i % kEx2PolyEvery == kEx2PolyEvery - 1) {  // this pair on the FMA pipe (MUFU relief)
+            p2 = ex2_poly_f2(x2);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          rs2[i & 1] = f2_add(rs2[i & 1], p2);
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
           pk[i] = pack_bf16x2(p0, p1);
         }
         // the previous P V must be complete before O is rescaled and the P buffer rewritten;

@@ -381,6 +381,35 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x for a pair of floats on the FMA and integer pipes instead of the MUFU unit.  x is
+// clamped to >= -126 and split as x = n + f: adding and then subtracting 1.5 * 2^23 rounds x
+// to the nearest integer n (round-to-nearest-even addition), so f = x - n lies in [-1/2, 1/2].
+// 2^f comes from a cubic fitted on [-1/2, 1/2] by iteratively reweighted least squares on the
+// relative error (largest relative error 7.5e-5, far below the bf16 rounding, 2^-9, of the
+// probabilities it produces), and n is added to the exponent field: after the addition the
+// low mantissa bits of x + 1.5 * 2^23 hold n, and shifting them up by 23 places n there.
+__device__ __forceinline__ uint64_t ex2_poly_f2(uint64_t x2) {
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f, c2 = 0.2426111400127411f,
+                  c3 = 0.055171653628349304f;
+  float a, b;
+  f2_unpack(x2, a, b);
+  x2 = f2_pack(fmaxf(a, -126.0f), fmaxf(b, -126.0f));
+  const uint64_t t2 = f2_add(x2, f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t n2 = f2_add(t2, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t fr = f2_fma(n2, f2_pack(-1.0f, -1.0f), x2);
+  uint64_t p = f2_fma(f2_pack(c3, c3), fr, f2_pack(c2, c2));
+  p = f2_fma(p, fr, f2_pack(c1, c1));
+  p = f2_fma(p, fr, f2_pack(c0, c0));
+  uint32_t plo, phi, tlo, thi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(plo), "=r"(phi) : "l"(p));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(tlo), "=r"(thi) : "l"(t2));
+  plo += tlo << 23;
+  phi += thi << 23;
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(plo), "r"(phi));
+  return r;
+}
+
 // ---------------------------------------------------------------- CTA pairs (cta_group::2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -345,13 +345,13 @@ constexpr int kLnRows = 32;     // token rows per block
 constexpr int kLnThreads = 256;
 
 // Writes the modulated row; the normalised values replace x (the E4M3 output needs them twice).
-template <int OUT>
-__device__ __forceinline__ void ln_store_row(const LnArgs& a, int m, int lane, int nv, float4 (&x)[kLnMaxVec],
-                                             float mean, float rstd, const float* sh, const float* sc) {
+template <int OUT, int VEC>
+__device__ __forceinline__ void ln_store_row(const LnArgs& a, int m, int lane, int nv, float4 (&x)[VEC], float mean,
+                                             float rstd, const float* sh, const float* sc) {
   float amax = 0.f, ss = 0.f;
-  float4(&o)[kLnMaxVec] = x;
+  float4(&o)[VEC] = x;
 #pragma unroll
-  for (int k = 0; k < kLnMaxVec; ++k) {
+  for (int k = 0; k < VEC; ++k) {
     const int c = lane + 32 * k;
     if (c < nv) {
       const float4 s4 = reinterpret_cast<const float4*>(sc)[c], b4 = reinterpret_cast<const float4*>(sh)[c];
@@ -384,31 +384,32 @@ __device__ __forceinline__ void ln_store_row(const LnArgs& a, int m, int lane, i
     }
     uint32_t* u8 = reinterpret_cast<uint32_t*>(a.u8 + static_cast<size_t>(m) * a.d);
 #pragma unroll
-    for (int k = 0; k < kLnMaxVec; ++k) {
+    for (int k = 0; k < VEC; ++k) {
       const int c = lane + 32 * k;
       if (c < nv) u8[c] = pack_e4m3x4(o[k].x * inv, o[k].y * inv, o[k].z * inv, o[k].w * inv);
     }
   }
 }
 
-__device__ __forceinline__ void ln_load_row(const float* h, int d, int lane, int nv, float4 (&x)[kLnMaxVec]) {
+template <int VEC>
+__device__ __forceinline__ void ln_load_row(const float* h, int lane, int nv, float4 (&x)[VEC]) {
   const float4* hp = reinterpret_cast<const float4*>(h);
 #pragma unroll
-  for (int k = 0; k < kLnMaxVec; ++k) {
+  for (int k = 0; k < VEC; ++k) {
     const int c = lane + 32 * k;
     x[k] = c < nv ? hp[c] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
-__device__ __forceinline__ void ln_stats(const float4 (&x)[kLnMaxVec], int lane, int nv, int d, float& mean,
-                                         float& rstd) {
+template <int VEC>
+__device__ __forceinline__ void ln_stats(const float4 (&x)[VEC], int lane, int nv, int d, float& mean, float& rstd) {
   float sum = 0.f;
 #pragma unroll
-  for (int k = 0; k < kLnMaxVec; ++k) sum += (x[k].x + x[k].y) + (x[k].z + x[k].w);
+  for (int k = 0; k < VEC; ++k) sum += (x[k].x + x[k].y) + (x[k].z + x[k].w);
   mean = warp_sum(sum) / d;
   float q = 0.f;
 #pragma unroll
-  for (int k = 0; k < kLnMaxVec; ++k) {
+  for (int k = 0; k < VEC; ++k) {
     const int c = lane + 32 * k;
     if (c < nv) {
       const float dx = x[k].x - mean, dy = x[k].y - mean, dz = x[k].z - mean, dw = x[k].w - mean;
@@ -418,8 +419,11 @@ __device__ __forceinline__ void ln_stats(const float4 (&x)[kLnMaxVec], int lane,
   rstd = rsqrtf(warp_sum(q) / d + 1e-6f);
 }
 
-// OUT: 0 float32, 1 bf16, 2 FP8 E4M3 with the row's scales (see LnArgs).
-template <int OUT>
+// OUT: 0 float32, 1 bf16, 2 FP8 E4M3 with the row's scales (see LnArgs).  VEC: float4 per lane
+// per row (the smallest of 3, 6, 9, 12 that covers d / 4), so a row takes no more registers
+// than it needs.  Each warp's first two rows are requested before the block stages its
+// modulation vectors, so the two loads' latencies overlap.
+template <int OUT, int VEC>
 __global__ void __launch_bounds__(kLnThreads) ln_modulate_kernel(LnArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -427,6 +431,12 @@ __global__ void __launch_bounds__(kLnThreads) ln_modulate_kernel(LnArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nv = a.d >> 2;
   const int m0 = blockIdx.x * kLnRows;
+  float4 xa[VEC], xb[VEC];
+  {
+    const int ma = m0 + warp * (kLnRows / 8), mb = ma + 1;
+    if (ma < a.M) ln_load_row<VEC>(a.h + static_cast<size_t>(ma) * a.d, lane, nv, xa);
+    if (mb < a.M) ln_load_row<VEC>(a.h + static_cast<size_t>(mb) * a.d, lane, nv, xb);
+  }
   // sample rows of this block's first and last token rows; staged when at most two
   const int rfirst = a.ld_mod ? m0 / a.T : 0;
   const int rlast = a.ld_mod ? min(m0 + kLnRows - 1, a.M - 1) / a.T : 0;
@@ -443,39 +453,47 @@ __global__ void __launch_bounds__(kLnThreads) ln_modulate_kernel(LnArgs a) {
   for (int pr = 0; pr < kLnRows / 8; pr += 2) {  // each warp: rows m0 + 4 warp + {0, 1}, then {2, 3}
     const int ma = m0 + warp * (kLnRows / 8) + pr, mb = ma + 1;
     if (ma >= a.M) break;
-    float4 xa[kLnMaxVec], xb[kLnMaxVec];
-    ln_load_row(a.h + static_cast<size_t>(ma) * a.d, a.d, lane, nv, xa);
     const bool hb = mb < a.M;
-    if (hb) ln_load_row(a.h + static_cast<size_t>(mb) * a.d, a.d, lane, nv, xb);
+    if (pr > 0) {
+      ln_load_row<VEC>(a.h + static_cast<size_t>(ma) * a.d, lane, nv, xa);
+      if (hb) ln_load_row<VEC>(a.h + static_cast<size_t>(mb) * a.d, lane, nv, xb);
+    }
     float mean, rstd;
-    ln_stats(xa, lane, nv, a.d, mean, rstd);
+    ln_stats<VEC>(xa, lane, nv, a.d, mean, rstd);
     {
       const int r = a.ld_mod ? ma / a.T : 0;
       const float* sh = staged ? ln_mod + 2 * (r - rfirst) * a.d : a.shift + static_cast<size_t>(r) * a.ld_mod;
       const float* sc = staged ? ln_mod + (2 * (r - rfirst) + 1) * a.d : a.scale + static_cast<size_t>(r) * a.ld_mod;
-      ln_store_row<OUT>(a, ma, lane, nv, xa, mean, rstd, sh, sc);
+      ln_store_row<OUT, VEC>(a, ma, lane, nv, xa, mean, rstd, sh, sc);
     }
     if (hb) {
-      ln_stats(xb, lane, nv, a.d, mean, rstd);
+      ln_stats<VEC>(xb, lane, nv, a.d, mean, rstd);
       const int r = a.ld_mod ? mb / a.T : 0;
       const float* sh = staged ? ln_mod + 2 * (r - rfirst) * a.d : a.shift + static_cast<size_t>(r) * a.ld_mod;
       const float* sc = staged ? ln_mod + (2 * (r - rfirst) + 1) * a.d : a.scale + static_cast<size_t>(r) * a.ld_mod;
-      ln_store_row<OUT>(a, mb, lane, nv, xb, mean, rstd, sh, sc);
+      ln_store_row<OUT, VEC>(a, mb, lane, nv, xb, mean, rstd, sh, sc);
     }
   }
+}
+
+template <int VEC>
+static cudaError_t launch_ln_vec(const LnArgs& a, int grid, size_t smem, cudaStream_t st) {
+  if (a.u8 != nullptr) return launch_kernel(ln_modulate_kernel<2, VEC>, dim3(grid), dim3(kLnThreads), smem, st, a);
+  if (a.u_bf16) return launch_kernel(ln_modulate_kernel<1, VEC>, dim3(grid), dim3(kLnThreads), smem, st, a);
+  return launch_kernel(ln_modulate_kernel<0, VEC>, dim3(grid), dim3(kLnThreads), smem, st, a);
 }
 
 cudaError_t launch_ln_modulate(const LnArgs& a, cudaStream_t st) {
   if ((a.d & 3) != 0 || a.d > 4 * 32 * kLnMaxVec) return cudaErrorInvalidValue;
   const int grid = (a.M + kLnRows - 1) / kLnRows;
   if (grid == 0) return cudaSuccess;
+  if (a.u8 != nullptr && (a.su == nullptr || a.sg == nullptr)) return cudaErrorInvalidValue;
   const size_t smem = 4 * static_cast<size_t>(a.d) * sizeof(float);
-  if (a.u8 != nullptr) {
-    if (a.su == nullptr || a.sg == nullptr) return cudaErrorInvalidValue;
-    return launch_kernel(ln_modulate_kernel<2>, dim3(grid), dim3(kLnThreads), smem, st, a);
-  }
-  if (a.u_bf16) return launch_kernel(ln_modulate_kernel<1>, dim3(grid), dim3(kLnThreads), smem, st, a);
-  return launch_kernel(ln_modulate_kernel<0>, dim3(grid), dim3(kLnThreads), smem, st, a);
+  const int nv = a.d >> 2;
+  if (nv <= 32 * 3) return launch_ln_vec<3>(a, grid, smem, st);
+  if (nv <= 32 * 6) return launch_ln_vec<6>(a, grid, smem, st);
+  if (nv <= 32 * 9) return launch_ln_vec<9>(a, grid, smem, st);
+  return launch_ln_vec<12>(a, grid, smem, st);
 }
 
 // ============================================================================ f32 GEMM
