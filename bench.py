@@ -273,6 +273,41 @@ def time_config(cfg, steps, warmup, graph, flush, options=None):
     return [a.elapsed_time(b) for a, b in evs]
 
 
+def gemm_reference(cfg, kernels, flush, reps=10):
+    """cuBLAS (torch.matmul, bf16 in and out, no fused epilogue) on the four block GEMM shapes of
+    this workload, timed like the kernel table: CUDA events around each launch, L2 flushed between
+    launches.  For context beside the fused kernels; it is not part of the forward."""
+    import torch
+    M, d = cfg.rows * cfg.tokens, cfg.hidden
+    mlp = cfg.mlp_hidden if getattr(cfg, "mlp_hidden", 0) else 4 * d
+    shapes = {"qkv": (M, 3 * d, d), "proj": (M, d, d), "fc1": (M, mlp, d), "fc2": (M, d, mlp)}
+    out = {}
+    g = torch.Generator(device="cuda").manual_seed(0)
+    for kind, (m, n, k) in shapes.items():
+        a = torch.randn(m, k, device="cuda", generator=g).to(torch.bfloat16)
+        w = (torch.randn(n, k, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        y = torch.empty(m, n, device="cuda", dtype=torch.bfloat16)
+        for _ in range(3):
+            torch.matmul(a, w.t(), out=y)
+        ts = []
+        for i in range(reps):
+            flush.fill_(float(i))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, w.t(), out=y)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        us = statistics.median(ts)
+        row = {"shape_mnk": [m, n, k], "cublas_us": us, "cublas_tflops": 2.0 * m * n * k / (us * 1e-6) / 1e12}
+        if kind in kernels:
+            row["fused_us"] = kernels[kind]["us_per_launch"]
+            row["fused_over_cublas"] = kernels[kind]["us_per_launch"] / us
+        out[kind] = row
+        del a, w, y
+    return out
+
+
 def all_configs(steps, warmup, graph, flush, peak_tf):
     from diffusion_transformer_denoiser_dit_b200.binding import DIT_OPT_PAIR_GEMM
     res = {}
@@ -568,6 +603,10 @@ def main():
         "clocks": clocks,
         "device_status": status,
     }
+    if rank == 0 and world == 1:
+        line["gemm_vs_cublas"] = gemm_reference(cfg, kernels, flush)
+        line["gemm_vs_cublas_note"] = ("cuBLAS writes plain bf16; the library's kernels fuse bias + GELU, the gated "
+                                       "residual reduce-add into the float32 stream and the head-major Q/K/V^T scatter")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, weights)
     del weights
