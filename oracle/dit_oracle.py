@@ -271,7 +271,8 @@ def self_attention(u, wqkv, bqkv, wo, bo, heads: int, qn=None, kn=None, coords=N
     QK-RMSNorm (gains qn, kn) and 3D RoPE (coords) for the video model."""
     r, t, d = u.shape
     dh = d // heads
-    qkv = linear(u, wqkv, bqkv)
+    fp8 = _STATE.get("attn_fp8")
+    qkv = linear_e4m3(u, wqkv, bqkv) if fp8 else linear(u, wqkv, bqkv)
     q, k, v = qkv[..., :d], qkv[..., d:2 * d], qkv[..., 2 * d:]
     o = np.zeros((r, t, d), dtype=F64)
     for i in range(r):
@@ -283,7 +284,7 @@ def self_attention(u, wqkv, bqkv, wo, bo, heads: int, qn=None, kn=None, coords=N
             if coords is not None:
                 qh, kh = rope_3d(qh, coords), rope_3d(kh, coords)
             o[i, :, sl] = attention(qh, kh, vh)
-    return linear(o, wo, bo)
+    return linear_e4m3(o, wo, bo) if fp8 else linear(o, wo, bo)
 
 
 def ffn(u, w1, b1, w2, b2):
@@ -294,9 +295,11 @@ def ffn(u, w1, b1, w2, b2):
 
 
 # --------------------------------------------------------------------------- #
-# FP8 (E4M3) feed-forward: a reading, not the pages' ([DiT-wiki] "U-Net과 비교" names
-# mixed precision among the techniques that carry over from language models; the pages fix
-# no format, so this is the quantised computation the FP8 path is held to)
+# FP8 (E4M3) linears: a reading, not the pages' ([DiT-wiki] "U-Net과 비교" names mixed
+# precision among the techniques that carry over from language models; the pages fix no
+# format, so this is the quantised computation the FP8 path is held to).  With attn_fp8 the
+# self-attention's in-projection and out-projection are linear_e4m3 (per-token amax scales of
+# the LN output and of the concatenated heads); with ffn_fp8 the feed-forward is ffn_e4m3.
 # --------------------------------------------------------------------------- #
 E4M3_MAX = 448.0
 
@@ -448,14 +451,16 @@ def embed(cfg, W, x5):
 def forward(cfg, weights: Sequence[np.ndarray] | Dict[str, np.ndarray], x, t, y,
             cfg_scale: Optional[float] = None, force_guidance: bool = False,
             stop_after_block: Optional[int] = None, cfg_channels: Optional[int] = None,
-            ffn_fp8: bool = False):
-    """ffn_fp8: every block's feed-forward in E4M3 (ffn_e4m3) instead of exact arithmetic."""
-    prev = _STATE.get("ffn_fp8", False)
+            ffn_fp8: bool = False, attn_fp8: bool = False):
+    """ffn_fp8: every block's feed-forward in E4M3 (ffn_e4m3) instead of exact arithmetic.
+    attn_fp8: every self-attention's in- and out-projection in E4M3 (linear_e4m3)."""
+    prev = (_STATE.get("ffn_fp8", False), _STATE.get("attn_fp8", False))
     _STATE["ffn_fp8"] = bool(ffn_fp8)
+    _STATE["attn_fp8"] = bool(attn_fp8)
     try:
         return _forward(cfg, weights, x, t, y, cfg_scale, force_guidance, stop_after_block, cfg_channels)
     finally:
-        _STATE["ffn_fp8"] = prev
+        _STATE["ffn_fp8"], _STATE["attn_fp8"] = prev
 
 
 def _forward(cfg, weights, x, t, y, cfg_scale, force_guidance, stop_after_block, cfg_channels):

@@ -1,4 +1,4 @@
-"""Pins of the oracle's FP8 (E4M3) feed-forward (CPU only).
+"""Pins of the oracle's FP8 (E4M3) linears: the feed-forward and the attention projections (CPU only).
 
 The quantiser is checked against torch's float8_e4m3fn cast (a library routine) on every
 representable value, every midpoint between neighbours (ties to even) and random values; the
@@ -90,3 +90,60 @@ def test_fp8_forward_stays_near_the_exact_forward(gates):
     rel = np.linalg.norm(a - b) / np.linalg.norm(a)
     assert 0 < rel < 5e-2, rel
     assert np.array_equal(O.forward(cfg, W, inp["x"], inp["t"], inp["y"]), a)   # the switch is scoped
+
+
+def _torch_linear_e4m3(x, w, b):
+    """linear_e4m3 written with torch's float8_e4m3fn cast (per-row amax / 448 scales)."""
+    def q(a):
+        s = a.abs().amax(dim=-1, keepdim=True) / 448.0
+        s = torch.where(s > 0, s, torch.ones_like(s))
+        return (a / s).to(torch.float8_e4m3fn).to(torch.float64) * s
+    return q(x) @ q(w).T + b
+
+
+def test_attn_fp8_self_attention_matches_a_torch_float8_composition():
+    """Both projections of the E4M3 self-attention, written independently with torch's float8
+    cast and torch's softmax: in-projection on the LN output's rows, out-projection on the
+    concatenated heads' rows (a slip such as leaving the out-projection exact fails here)."""
+    rng = np.random.default_rng(34)
+    r, t, d, heads = 2, 20, 48, 3
+    u = rng.standard_normal((r, t, d)) * 2.0
+    wqkv, bqkv = rng.standard_normal((3 * d, d)) * 0.2, rng.standard_normal(3 * d) * 0.1
+    wo, bo = rng.standard_normal((d, d)) * 0.2, rng.standard_normal(d) * 0.1
+    O._STATE["attn_fp8"] = True
+    try:
+        got = O.self_attention(u, wqkv, bqkv, wo, bo, heads)
+    finally:
+        O._STATE["attn_fp8"] = False
+    U = torch.from_numpy(u)
+    qkv = _torch_linear_e4m3(U.reshape(r * t, d), torch.from_numpy(wqkv), torch.from_numpy(bqkv)).reshape(r, t, 3 * d)
+    dh = d // heads
+    q = qkv[..., :d].reshape(r, t, heads, dh).transpose(1, 2)
+    k = qkv[..., d:2 * d].reshape(r, t, heads, dh).transpose(1, 2)
+    v = qkv[..., 2 * d:].reshape(r, t, heads, dh).transpose(1, 2)
+    o = torch.softmax(q @ k.transpose(-1, -2) / dh ** 0.5, dim=-1) @ v
+    o = o.transpose(1, 2).reshape(r * t, d)
+    want = _torch_linear_e4m3(o, torch.from_numpy(wo), torch.from_numpy(bo)).reshape(r, t, d).numpy()
+    assert np.allclose(got, want, rtol=1e-10, atol=1e-10)
+    exact = O.self_attention(u, wqkv, bqkv, wo, bo, heads)
+    assert not np.allclose(got, exact, rtol=1e-4, atol=1e-4)     # the switch does something
+
+
+@pytest.mark.parametrize("gates", ["random", "strong"])
+def test_attn_fp8_forward_stays_near_the_exact_forward(gates):
+    """E4M3 attention projections (and with them the E4M3 feed-forward) perturb the forward
+    by a few percent at most; the switches are scoped to the call."""
+    cfg = S.DIT_XL2_CFG256.with_(hidden=288, heads=4, mlp_hidden=1152, depth=2, height=16, width=16, batch=2,
+                                 index=-1)
+    W = S.make_weights(cfg)
+    if gates == "strong":
+        W = S.set_adaln(cfg, W, gate_bias=1.0)
+    inp = S.make_inputs(cfg)
+    a = O.forward(cfg, W, inp["x"], inp["t"], inp["y"])
+    b = O.forward(cfg, W, inp["x"], inp["t"], inp["y"], attn_fp8=True)
+    c = O.forward(cfg, W, inp["x"], inp["t"], inp["y"], attn_fp8=True, ffn_fp8=True)
+    for z in (b, c):
+        rel = np.linalg.norm(a - z) / np.linalg.norm(a)
+        assert 0 < rel < 5e-2, rel
+    assert not np.array_equal(b, c)
+    assert np.array_equal(O.forward(cfg, W, inp["x"], inp["t"], inp["y"]), a)
