@@ -58,13 +58,20 @@ WORKLOADS = {
     "video": S.VIDEO_RF,
     "b4": S.DIT_B4_BF16,
     "xl2_256_fp8": S.DIT_XL2_CFG256.with_(ffn_fp8=1),
+    "xl2_256_fp8all": S.DIT_XL2_CFG256.with_(ffn_fp8=1, attn_fp8=1),
 }
+
+
+def fp8_desc(cfg):
+    parts = [n for n, on in (("attention projections", getattr(cfg, "attn_fp8", 0)),
+                              ("feed-forward", getattr(cfg, "ffn_fp8", 0))) if on]
+    return " + ".join(parts)
 
 
 def workload_desc(cfg):
     lat = (f"{cfg.in_channels}x{cfg.frames}x{cfg.height}x{cfg.width}" if cfg.frames > 1
            else f"{cfg.in_channels}x{cfg.height}x{cfg.width}")
-    extra = ", FP8 E4M3 feed-forward" if getattr(cfg, "ffn_fp8", 0) else ""
+    extra = f", FP8 E4M3 {fp8_desc(cfg)}" if fp8_desc(cfg) else ""
     return (f"{cfg.name}: {cfg.batch} latents {lat} -> {cfg.rows} rows x {cfg.tokens} tokens, d={cfg.hidden}, "
             f"{cfg.depth} blocks, {cfg.heads} heads, s={cfg.cfg_scale}{extra}")
 
@@ -321,7 +328,9 @@ def all_configs(steps, warmup, graph, flush, peak_tf):
                       ("c3 XL/2 CFG 256px, cross-attention conditioning", S.DIT_XL2_CFG256.with_(block_kind=S.BLOCK_CROSS_ATTN)),
                       ("c3 XL/2 CFG 256px, adaLN conditioning", S.DIT_XL2_CFG256.with_(block_kind=S.BLOCK_ADALN)),
                       ("c3 XL/2 CFG 256px, FP8 E4M3 feed-forward", S.DIT_XL2_CFG256.with_(ffn_fp8=1)),
-                      ("c5 video RF 4096 tokens, FP8 E4M3 feed-forward", S.VIDEO_RF.with_(ffn_fp8=1))):
+                      ("c5 video RF 4096 tokens, FP8 E4M3 feed-forward", S.VIDEO_RF.with_(ffn_fp8=1)),
+                      ("c3 XL/2 CFG 256px, FP8 E4M3 attention projections + feed-forward",
+                       S.DIT_XL2_CFG256.with_(ffn_fp8=1, attn_fp8=1))):
         runs.append((name, cfg, None))
         if name in pair_after:   # the same workload on SM-pair GEMMs, timed right after it
             runs.append((pair_after[name], cfg, {DIT_OPT_PAIR_GEMM: 1}))
@@ -334,7 +343,7 @@ def all_configs(steps, warmup, graph, flush, peak_tf):
                      "tokens_per_s": cfg.rows * cfg.tokens / (med / 1e3),
                      "samples_per_s": cfg.batch / (med / 1e3), "tflops": tf,
                      "frac_of_burst_bf16": tf / peak_tf if cfg.dtype == S.DTYPE_BF16 else None,
-                     "dtype": ("bf16 + e4m3 feed-forward" if getattr(cfg, "ffn_fp8", 0) else "bf16")
+                     "dtype": (f"bf16 + e4m3 {fp8_desc(cfg)}" if fp8_desc(cfg) else "bf16")
                               if cfg.dtype == S.DTYPE_BF16 else "f32",
                      "rows": cfg.rows, "tokens_per_row": cfg.tokens, "flops_per_step": fl}
     return res

@@ -38,7 +38,8 @@ class DitConfig(ctypes.Structure):
                 ("patch_t", c_int), ("patch_h", c_int), ("patch_w", c_int), ("hidden", c_int), ("depth", c_int),
                 ("heads", c_int), ("mlp_hidden", c_int), ("learn_sigma", c_int), ("pos_kind", c_int),
                 ("qk_norm", c_int), ("cond_kind", c_int), ("num_classes", c_int), ("freq_dim", c_int),
-                ("max_batch", c_int), ("t_scale", c_float), ("block_kind", c_int), ("ffn_fp8", c_int)]
+                ("max_batch", c_int), ("t_scale", c_float), ("block_kind", c_int), ("ffn_fp8", c_int),
+                ("attn_fp8", c_int)]
 
 
 class DitError(RuntimeError):
@@ -99,7 +100,8 @@ def make_config(cfg, max_batch: Optional[int] = None) -> DitConfig:
     return DitConfig(cfg.dtype, cfg.in_channels, cfg.frames, cfg.height, cfg.width, cfg.patch_t, cfg.patch_h,
                      cfg.patch_w, cfg.hidden, cfg.depth, cfg.heads, cfg.mlp_hidden, cfg.learn_sigma, cfg.pos_kind,
                      cfg.qk_norm, cfg.cond_kind, cfg.num_classes, cfg.freq_dim, mb, float(cfg.t_scale),
-                     int(getattr(cfg, "block_kind", 0)), int(getattr(cfg, "ffn_fp8", 0)))
+                     int(getattr(cfg, "block_kind", 0)), int(getattr(cfg, "ffn_fp8", 0)),
+                     int(getattr(cfg, "attn_fp8", 0)))
 
 
 def status_string(code: int) -> str:

@@ -30,6 +30,10 @@ struct BlockW {
   uint8_t *fc1_w8 = nullptr, *fc2_w8 = nullptr;
   float *fc1_s = nullptr, *fc2_s = nullptr;
   float g_w = 0.f, g_b = 0.f;
+  // FP8 attention projections: E4M3 in- and out-projection weights, per-output-channel scales
+  uint8_t *qkv_w8 = nullptr, *proj_w8 = nullptr;
+  float *qkv_s = nullptr, *proj_s = nullptr;
+  CUtensorMap tm_qkv8, ta_qkv8, ta_proj8;  // as the B operand (two-head tiles) / the swapped A operand
   CUtensorMap tm_qkv, tm_fc1, tm_xq, tm_fc1_8;  // weights as the B operand (box = tile width rows)
   CUtensorMap tm_fc1_h;  // fc1 weights as the B operand of the SM-pair GEMM (each CTA loads half: 128 rows)
   CUtensorMap ta_qkv, ta_proj, ta_fc2, ta_xo, ta_fc2_8;  // weights as the A operand of the swapped GEMMs (box 128 rows)
@@ -70,6 +74,7 @@ bool validate(const dit_config* c, std::string& err) {
   if (!isfinite(c->t_scale)) return bad("t_scale must be finite");
   if (c->block_kind < DIT_BLOCK_ADALN_ZERO || c->block_kind > DIT_BLOCK_ADALN) return bad("unknown block_kind");
   if (c->ffn_fp8 != 0 && c->ffn_fp8 != 1) return bad("ffn_fp8 must be 0 or 1");
+  if (c->attn_fp8 != 0 && c->attn_fp8 != 1) return bad("attn_fp8 must be 0 or 1");
   return true;
 }
 
@@ -104,6 +109,10 @@ bool supported(const dit_config* c, std::string& err) {
   }
   if (c->ffn_fp8 && c->dtype != DIT_DTYPE_BF16) {
     err = "the FP8 feed-forward runs on the bf16 tensor-core path only";
+    return false;
+  }
+  if (c->attn_fp8 && c->dtype != DIT_DTYPE_BF16) {
+    err = "the FP8 attention projections run on the bf16 tensor-core path only";
     return false;
   }
   const long long kp = 1LL * c->in_channels * c->patch_t * c->patch_h * c->patch_w;
@@ -184,6 +193,8 @@ struct dit_handle {
   float* ones = nullptr;                     // [d] of 1.0: the gate of the ungated designs
   uint8_t *u8 = nullptr, *g8 = nullptr;      // FP8 feed-forward operands [Mmax, d], [Mmax, mlp]
   float *su = nullptr, *sg = nullptr;        // their per-token scales [Mmax]
+  uint8_t* o8 = nullptr;                     // FP8 attention output [Mmax, d] (the out-projection's operand)
+  float* so = nullptr;                       // its per-token scales [Mmax]
   void* xkv_w = nullptr;                     // cross-attention key / value weights of all blocks [nkv, d]
   float *xkv_b = nullptr, *xkv = nullptr;    // their biases [nkv]; keys / values [2 Rmax, nkv] (f32)
   void* ctx = nullptr;                       // condition sequence [CTXalloc, d]: rows 2r, 2r+1 = e_t, e_y
@@ -196,6 +207,7 @@ struct dit_handle {
   void* y_stage = nullptr;
   CUtensorMap tm_ada, tm_sc[5], tm_u, tm_o, tm_g, tm_dec, tm_xkv, tm_ctx[5];
   CUtensorMap tm_u8, tb_g8;  // FP8: LN output as fc1's A operand; fc1 output as fc2's B operand
+  CUtensorMap tb_u8, tb_o8;  // FP8: LN output / attention output as the swapped GEMMs' B operand
   CUtensorMap tm_g_out, tm_h_red;  // TMA-store targets: GELU output, residual stream
   CUtensorMap tb_u, tb_o, tb_g;     // activations as the B operand of the swapped GEMMs (box 256 rows)
   AttnMaps attn_maps;
@@ -396,9 +408,16 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
       ALLOC(b.xo_w, void, (size_t)d * d * es);
       ALLOC(b.xo_b, float, (size_t)d * 4);
     }
-    ALLOC(b.qkv_w, void, (size_t)3 * d * d * es);
+    if (cfg->attn_fp8) {
+      ALLOC(b.qkv_w8, uint8_t, (size_t)3 * d * d);
+      ALLOC(b.qkv_s, float, (size_t)3 * d * 4);
+      ALLOC(b.proj_w8, uint8_t, (size_t)d * d);
+      ALLOC(b.proj_s, float, (size_t)d * 4);
+    } else {
+      ALLOC(b.qkv_w, void, (size_t)3 * d * d * es);
+      ALLOC(b.proj_w, void, (size_t)d * d * es);
+    }
     ALLOC(b.qkv_b, float, (size_t)3 * d * 4);
-    ALLOC(b.proj_w, void, (size_t)d * d * es);
     ALLOC(b.proj_b, float, (size_t)d * 4);
     if (cfg->ffn_fp8) {
       ALLOC(b.fc1_w8, uint8_t, (size_t)mlp * d);
@@ -447,11 +466,17 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
   }
   ALLOC(H->o, void, M * d * es);
   ALLOC(H->z, float, M * g.P * 4);
-  if (cfg->ffn_fp8) {
+  if (cfg->ffn_fp8 || cfg->attn_fp8) {
     ALLOC(H->u8, uint8_t, M * d);
-    ALLOC(H->g8, uint8_t, M * mlp);
     ALLOC(H->su, float, M * 4);
     ALLOC(H->sg, float, M * 4);
+  }
+  if (cfg->attn_fp8) {
+    ALLOC(H->o8, uint8_t, M * d);
+    ALLOC(H->so, float, M * 4);
+  }
+  if (cfg->ffn_fp8) {
+    ALLOC(H->g8, uint8_t, M * mlp);
     ALLOC(H->gbuf, void, 16);
   } else {
     ALLOC(H->gbuf, void, M * mlp * es);
@@ -473,7 +498,7 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
   }
   float* staging = nullptr;
   if (H->bf16) ALLOC(staging, float, maxn * 4);
-  if (cfg->ffn_fp8 && staging == nullptr) {
+  if ((cfg->ffn_fp8 || cfg->attn_fp8) && staging == nullptr) {
     dit_destroy(H);
     return DIT_ERR_INVALID_ARG;
   }
@@ -525,14 +550,31 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
       UP_GAIN(b.ln1_s);
       UP(b.ln1_b, (size_t)d, false);
     }
-    UP(b.qkv_w, (size_t)3 * d * d, H->bf16);
+    // E4M3 weights of the FP8 attention projections, quantised per output channel on the device
+#define UP_E4M3(dst8, scale, rows)                                                                      \
+  do {                                                                                                 \
+    if (cudaMemcpy(staging, weights[wi++], (size_t)(rows) * d * 4, cudaMemcpyHostToDevice) != cudaSuccess || \
+        launch_quantize_rows_e4m3(staging, (dst8), (scale), (rows), d, 0) != cudaSuccess ||              \
+        cudaDeviceSynchronize() != cudaSuccess) {                                                      \
+      dit_destroy(H);                                                                                  \
+      return DIT_ERR_CUDA;                                                                             \
+    }                                                                                                  \
+  } while (0)
+    if (cfg->attn_fp8)
+      UP_E4M3(b.qkv_w8, b.qkv_s, 3 * d);
+    else
+      UP(b.qkv_w, (size_t)3 * d * d, H->bf16);
     UP(b.qkv_b, (size_t)3 * d, false);
     if (cfg->qk_norm) {
       UP(b.qn, (size_t)g.dh, false);
       UP(b.kn, (size_t)g.dh, false);
     }
-    UP(b.proj_w, (size_t)d * d, H->bf16);
+    if (cfg->attn_fp8)
+      UP_E4M3(b.proj_w8, b.proj_s, d);
+    else
+      UP(b.proj_w, (size_t)d * d, H->bf16);
     UP(b.proj_b, (size_t)d, false);
+#undef UP_E4M3
     if (cross) {
       UP_GAIN(b.xln_s);
       UP(b.xln_b, (size_t)d, false);
@@ -620,9 +662,12 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
     }
     ok = ok && make_tmap_bf16_kmajor(&H->tm_u, H->u, g.Mmax, d, 128);
     ok = ok && make_tmap_bf16_kmajor(&H->tm_o, H->o, g.Mmax, d, 128);
-    if (cfg->ffn_fp8) {
+    if (cfg->ffn_fp8 || cfg->attn_fp8)
       ok = ok && make_tmap_e4m3_kmajor(&H->tm_u8, H->u8, g.Mmax, d, 128) &&
-           make_tmap_e4m3_kmajor(&H->tb_g8, H->g8, g.Mmax, mlp, 256);
+           make_tmap_e4m3_kmajor(&H->tb_u8, H->u8, g.Mmax, d, 256);
+    if (cfg->attn_fp8) ok = ok && make_tmap_e4m3_kmajor(&H->tb_o8, H->o8, g.Mmax, d, 256);
+    if (cfg->ffn_fp8) {
+      ok = ok && make_tmap_e4m3_kmajor(&H->tb_g8, H->g8, g.Mmax, mlp, 256);
     } else {
       ok = ok && make_tmap_bf16_kmajor(&H->tm_g, H->gbuf, g.Mmax, mlp, 128) &&
            make_tmap_bf16(&H->tm_g_out, H->gbuf, g.Mmax, mlp, 32, 32, 64) &&
@@ -635,9 +680,14 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
     ok = ok && make_attention_maps(&H->attn_maps, H->q, H->k, H->v, H->o, g.Rmax, cfg->heads, g.Ts, g.Tpad, g.dh, g.DP, d);
     for (int i = 0; i < N && ok; ++i) {
       BlockW& b = H->blk[i];
-      ok = make_tmap_bf16_kmajor(&b.tm_qkv, b.qkv_w, 3 * d, d, g.headwise ? g.bn_qkv : 128) &&
-           make_tmap_bf16_kmajor(&b.ta_qkv, b.qkv_w, 3 * d, d, 128) &&
-           make_tmap_bf16_kmajor(&b.ta_proj, b.proj_w, d, d, 128);
+      if (cfg->attn_fp8)
+        ok = make_tmap_e4m3_kmajor(&b.tm_qkv8, b.qkv_w8, 3 * d, d, g.headwise ? g.bn_qkv : 128) &&
+             make_tmap_e4m3_kmajor(&b.ta_qkv8, b.qkv_w8, 3 * d, d, 128) &&
+             make_tmap_e4m3_kmajor(&b.ta_proj8, b.proj_w8, d, d, 128);
+      else
+        ok = make_tmap_bf16_kmajor(&b.tm_qkv, b.qkv_w, 3 * d, d, g.headwise ? g.bn_qkv : 128) &&
+             make_tmap_bf16_kmajor(&b.ta_qkv, b.qkv_w, 3 * d, d, 128) &&
+             make_tmap_bf16_kmajor(&b.ta_proj, b.proj_w, d, d, 128);
       if (cfg->ffn_fp8)
         ok = ok && make_tmap_e4m3_kmajor(&b.tm_fc1_8, b.fc1_w8, mlp, d, g.bn_fc1) &&
              make_tmap_e4m3_kmajor(&b.ta_fc2_8, b.fc2_w8, d, mlp, 128);
@@ -663,7 +713,8 @@ int dit_forward_launch_count(const dit_handle* H, int B, float cfg_scale) {
   (void)B;
   (void)cfg_scale;
   const Geometry& g = H->g;
-  int per_block = 7 + ((!H->bf16 && (H->cfg.qk_norm || H->cfg.pos_kind == DIT_POS_ROPE3D)) ? 1 : 0);
+  int per_block = 7 + ((!H->bf16 && (H->cfg.qk_norm || H->cfg.pos_kind == DIT_POS_ROPE3D)) ? 1 : 0) +
+                  (H->cfg.attn_fp8 ? 1 : 0);  // the attention output's E4M3 quantisation
   if (g.kind == DIT_BLOCK_CROSS_ATTN) per_block += H->bf16 ? 3 : 4;
   const int front = 3 + (g.nmod > 0 ? 1 : 0) + (g.nkv > 0 ? 1 : 0) + 1;  // condition, projections, embedding
   return front + H->cfg.depth * per_block + 1 + 2;
@@ -914,7 +965,26 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
       n1 = {b.ln1_b, b.ln1_s, 0};
       n2 = {b.ln2_b, b.ln2_s, 0};
     }
-    DIT_TRY(run_ln(n1, "ln1"));
+    if (c.attn_fp8) {  // LN1 straight to E4M3 with per-token scales (the in-projection's operand)
+      LnArgs ln;
+      ln.h = H->h;
+      ln.u = H->u;
+      ln.u_bf16 = 1;
+      ln.u8 = H->u8;
+      ln.su = H->su;
+      ln.sg = H->sg;  // written, unused: no GELU follows
+      ln.g_w = 0.f;
+      ln.g_b = 0.f;
+      ln.ld_mod = n1.ld;
+      ln.M = p.M;
+      ln.T = Ts;
+      ln.d = d;
+      ln.shift = n1.shift;
+      ln.scale = n1.scale;
+      DIT_LAUNCH(H, DIT_KERNEL_LN, st, launch_ln_modulate(ln, st), "ln1 (fp8)");
+    } else {
+      DIT_TRY(run_ln(n1, "ln1"));
+    }
 
     EpiArgs qa = {};
     qa.M = p.M;
@@ -947,7 +1017,25 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
     aa.d = d;
     aa.bf16 = H->bf16;
 
-    if (H->bf16) {
+    if (H->bf16 && c.attn_fp8) {  // E4M3 in-projection (kind::f8f6f4), scales applied in the epilogue
+      if (g.headwise) {
+        EpiArgs q8 = qa;
+        q8.sa = H->su;
+        q8.sb = b.qkv_s;
+        DIT_LAUNCH(H, DIT_KERNEL_QKV, st,
+                   launch_gemm_tc(EPI_QKV_HEAD8, g.bn_qkv, &H->tm_u8, &b.tm_qkv8, d, q8, H->num_sms, st),
+                   "qkv gemm (fp8)");
+      } else {
+        EpiArgs q8 = qa;  // swapped: rows = 3d output features, columns = tokens
+        q8.M = 3 * d;
+        q8.N = p.M;
+        q8.sa = b.qkv_s;
+        q8.sb = H->su;
+        DIT_LAUNCH(H, DIT_KERNEL_QKV, st,
+                   launch_gemm_tc(EPI_QKV_T8, 256, &b.ta_qkv8, &H->tb_u8, d, q8, H->num_sms, st), "qkv gemm (fp8)");
+      }
+      DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_tc(aa, H->attn_maps, H->status, st), "attention");
+    } else if (H->bf16) {
       if (g.headwise) {
         DIT_LAUNCH(H, DIT_KERNEL_QKV, st,
                    launch_gemm_tc(EPI_QKV_HEAD, g.bn_qkv, &H->tm_u, &b.tm_qkv, d, qa, H->num_sms, st), "qkv gemm");
@@ -981,8 +1069,29 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
       }
       DIT_LAUNCH(H, DIT_KERNEL_ATTN, st, launch_attention_simt(aa, st), "attention");
     }
-    DIT_TRY(run_resid(DIT_KERNEL_PROJ, &b.ta_proj, &H->tb_o, &H->tm_o, H->o, b.proj_w, d, b.proj_b, gate1, ld_gate,
-                      "proj gemm"));
+    if (c.attn_fp8) {  // the heads' output to E4M3 per token, then the E4M3 out-projection
+      DIT_LAUNCH(H, DIT_KERNEL_PROJ, st,
+                 launch_quantize_rows_bf16_e4m3(static_cast<const uint16_t*>(H->o), H->o8, H->so, p.M, d, st),
+                 "attention output to e4m3");
+      EpiArgs pt = {};
+      pt.M = d;
+      pt.N = p.M;
+      pt.bias = b.proj_b;
+      pt.h = H->h;
+      pt.ldh = d;
+      pt.gate = gate1;
+      pt.ld_gate = ld_gate;
+      pt.T = Ts;
+      pt.sa = b.proj_s;
+      pt.sb = H->so;
+      pt.status = H->status;
+      DIT_LAUNCH(H, DIT_KERNEL_PROJ, st,
+                 launch_gemm_tc(EPI_RESID_T8, 256, &b.ta_proj8, &H->tb_o8, d, pt, H->num_sms, st, &H->tm_h_red),
+                 "proj gemm (fp8)");
+    } else {
+      DIT_TRY(run_resid(DIT_KERNEL_PROJ, &b.ta_proj, &H->tb_o, &H->tm_o, H->o, b.proj_w, d, b.proj_b, gate1, ld_gate,
+                        "proj gemm"));
+    }
 
     if (g.kind == DIT_BLOCK_CROSS_ATTN) {  // h += CrossAttn(LNx(h), [e_t, e_y])
       DIT_TRY(run_ln(Norm{b.xln_b, b.xln_s, 0}, "cross-attention ln"));

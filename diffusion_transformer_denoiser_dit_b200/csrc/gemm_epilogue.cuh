@@ -140,16 +140,21 @@ __device__ __forceinline__ void epilogue_chunk(const EpiArgs& ea, const uint32_t
 }
 
 // One whole head (DH columns) of q, k or v for output row m: bias, optional
-// QK-RMSNorm and 3D RoPE, head-major store.
-template <int DH>
+// QK-RMSNorm and 3D RoPE, head-major store.  FP8: E4M3 operands, the accumulator is first
+// scaled by the token's scale sa[m] and each weight row's scale sb[n + j].
+template <int DH, bool FP8 = false>
 __device__ __forceinline__ void epilogue_head(const EpiArgs& ea, const uint32_t* r, int m, int n) {
   if (n >= ea.N) return;
   const int which = n / ea.d;
   const int head = (n - which * ea.d) / DH;
   const int row = m / ea.T, tok = m - row * ea.T;
+  const float sm = FP8 && m < ea.M ? __ldg(ea.sa + m) : 1.f;
   float v[DH];
 #pragma unroll
-  for (int j = 0; j < DH; ++j) v[j] = __uint_as_float(r[j]) + __ldg(ea.bias + n + j);
+  for (int j = 0; j < DH; ++j) {
+    const float acc = FP8 ? __uint_as_float(r[j]) * sm * __ldg(ea.sb + n + j) : __uint_as_float(r[j]);
+    v[j] = acc + __ldg(ea.bias + n + j);
+  }
   if (which < 2) {
     const float* gn = which == 0 ? ea.qn : ea.kn;
     if (gn != nullptr) {
@@ -242,7 +247,7 @@ __device__ __forceinline__ void epilogue_cols(const EpiArgs& ea, uint32_t tacc, 
     if constexpr (EPI == EPI_XATTN)
       epilogue_xattn<NC>(ea, r, m, n0 + c0);
     else
-      epilogue_head<NC>(ea, r, m, n0 + c0);
+      epilogue_head<NC, EPI == EPI_QKV_HEAD8>(ea, r, m, n0 + c0);
   } else {
     constexpr int W = NC % 32 == 0 ? 32 : (NC % 16 == 0 ? 16 : 8);
     constexpr int NCH = NC / W;
@@ -267,7 +272,7 @@ __device__ __forceinline__ void epilogue_cols(const EpiArgs& ea, uint32_t tacc, 
 // slow the concurrent main loop more).
 template <int EPI>
 __host__ __device__ constexpr bool epi_staged() {
-  return EPI == EPI_GELU || EPI == EPI_RESID_T || EPI == EPI_RESID_T8 || EPI == EPI_QKV_T;
+  return EPI == EPI_GELU || EPI == EPI_RESID_T || EPI == EPI_RESID_T8 || EPI == EPI_QKV_T || EPI == EPI_QKV_T8;
 }
 constexpr int kStageBytesPerWarp = 4096;
 constexpr int kEpilogueWarps = 8;
@@ -462,7 +467,9 @@ __device__ __forceinline__ void store_vt_row32(uint16_t* dst, const uint32_t* v,
 // Chunks that straddle two sample rows, V^T chunks that start off a 16-byte boundary and
 // widths d that are not a multiple of 32 are written lane by lane instead: V^T as 16-byte
 // groups of 8 tokens, q and k one token per instruction.
-template <int NC>
+// FP8 = true: E4M3 operands, the accumulator is first scaled by the weight row's scale sa[f]
+// and each token's scale sb[tok].
+template <int NC, bool FP8 = false>
 __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc, int f_base, int lane, int n0, int c0,
                                                uint8_t* stg) {
   static_assert(NC % 32 == 0, "32-token chunks");
@@ -473,6 +480,7 @@ __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc,
   const int within = f - which * ea.d;
   const int head = within / ea.dh, j = within - head * ea.dh;
   const float bf = fok ? __ldg(ea.bias + f) : 0.f;
+  const float sf = (FP8 && fok) ? __ldg(ea.sa + f) : 1.f;
   uint16_t* qk = static_cast<uint16_t*>(which == 0 ? ea.q : ea.k);
   // staging: all 32 features of the warp are q, all k or all v
   const bool warp_one_kind = (ea.d & 31) == 0 && f_base + 31 < ea.M;
@@ -497,7 +505,14 @@ __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc,
   for (int c = 0; c < NCH; ++c) {
     if (c + 1 < NCH) tmem_ld_chunk<32>(tacc + c0 + (c + 1) * 32, r[(c + 1) & 1]);
     const int tok0 = n0 + c0 + c * 32;
-    const uint32_t* v = r[c & 1];
+    uint32_t* v = r[c & 1];
+    if constexpr (FP8) {
+      if (tok0 < ea.N) {  // lane l holds token tok0 + l's scale, handed to every lane
+        const float st_l = tok0 + lane < ea.N ? __ldg(ea.sb + tok0 + lane) : 0.f;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] = __float_as_uint(__uint_as_float(v[t]) * sf * __shfl_sync(0xffffffffu, st_l, t));
+      }
+    }
     if (fok && tok0 < ea.N) {
       const int last = min(tok0 + 31, ea.N - 1);
       const int r0 = tok0 / ea.T, t0 = tok0 - r0 * ea.T;

@@ -200,14 +200,15 @@ __global__ void __launch_bounds__(320, 1)
                                                        staging + (warp - 2) * kStageBytesPerWarp, first_slice);
       else if constexpr (EPI == EPI_GELU8)
         epilogue_gelu8<BN / 2>(ea, tacc, m0 + q * 32 + lane, n0, ((warp - 2) >> 2) * (BN / 2));
-      else if constexpr (EPI == EPI_QKV_T)
-        epilogue_qkv_t<BN / 2>(ea, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
+      else if constexpr (EPI == EPI_QKV_T || EPI == EPI_QKV_T8)
+        epilogue_qkv_t<BN / 2, EPI == EPI_QKV_T8>(ea, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
                                staging + (warp - 2) * kStageBytesPerWarp);
       else if constexpr (epi_staged<EPI>())
         epilogue_cols_staged<BN / 2, EPI>(ea, tacc, m0 + q * 32, lane, n0, ((warp - 2) >> 2) * (BN / 2),
                                           staging + (warp - 2) * kStageBytesPerWarp);
       else
-        epilogue_cols<BN / 2, (EPI == EPI_QKV_HEAD ? EPI_QKV : EPI), EPI == EPI_QKV_HEAD || EPI == EPI_XATTN>(
+        epilogue_cols<BN / 2, (EPI == EPI_QKV_HEAD ? EPI_QKV : EPI),
+                      EPI == EPI_QKV_HEAD || EPI == EPI_QKV_HEAD8 || EPI == EPI_XATTN>(
             ea, tacc, m0 + q * 32 + lane, n0, ((warp - 2) >> 2) * (BN / 2));
       tc_fence_before();
       mbar_arrive(TEMPTY_BAR(a));
@@ -356,6 +357,10 @@ cudaError_t launch_gemm_tc(int epi, int bn, const CUtensorMap* tA, const CUtenso
       DIT_BN_CASE(256, EPI_GELU8) break;
     case EPI_RESID_T8:
       DIT_BN_CASE(256, EPI_RESID_T8) break;
+    case EPI_QKV_T8:
+      DIT_BN_CASE(256, EPI_QKV_T8) break;
+    case EPI_QKV_HEAD8:
+      DIT_BN_CASE(128, EPI_QKV_HEAD8) DIT_BN_CASE(144, EPI_QKV_HEAD8) break;
     default:
       break;
   }

@@ -29,10 +29,12 @@ enum Epi : int {
   EPI_F32_8 = 9,     // out[m, n] = sa[m] sb[n] acc + bias[n]                  (float32)
   EPI_GELU8 = 10,    // g = gelu(sa[m] sb[n] acc + bias[n]) stored as E4M3 g / sg[m] (bytes [M, ldo])
   EPI_RESID_T8 = 11, // swapped: h[tok, f] += gate * (sa[f] sb[tok] acc + bias[f]) (TMA reduce-add)
+  EPI_QKV_T8 = 12,   // swapped q, k, v^T scatter of sa[f] sb[tok] acc + bias[f]
+  EPI_QKV_HEAD8 = 13,  // whole-head scatter (+ QK-RMSNorm, 3D RoPE) of sa[m] sb[n] acc + bias[n]
 };
 template <int EPI>
 __host__ __device__ constexpr bool epi_fp8() {
-  return EPI == EPI_F32_8 || EPI == EPI_GELU8 || EPI == EPI_RESID_T8;
+  return EPI == EPI_F32_8 || EPI == EPI_GELU8 || EPI == EPI_RESID_T8 || EPI == EPI_QKV_T8 || EPI == EPI_QKV_HEAD8;
 }
 
 struct EpiArgs {
@@ -236,6 +238,9 @@ cudaError_t launch_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaSt
 // zero row), dst[r, c] = E4M3(src[r, c] / scale[r]).
 cudaError_t launch_quantize_rows_e4m3(const float* src, uint8_t* dst, float* scale, int rows, int cols,
                                       cudaStream_t st);
+// bf16 rows [rows, cols] -> E4M3 bytes with per-row scales amax / 448; cols % 4 == 0, <= 1536.
+cudaError_t launch_quantize_rows_bf16_e4m3(const uint16_t* src, uint8_t* dst, float* scale, int rows, int cols,
+                                           cudaStream_t st);
 cudaError_t launch_wait_probe(int* flag, int* status, long long limit_ns, cudaStream_t st);
 
 }  // namespace dit

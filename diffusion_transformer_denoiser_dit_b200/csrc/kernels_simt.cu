@@ -922,6 +922,51 @@ cudaError_t launch_quantize_rows_e4m3(const float* src, uint8_t* dst, float* sca
   return cudaGetLastError();
 }
 
+// bf16 rows -> E4M3 with a per-row scale amax / 448 (1 for an all-zero row), one warp per row:
+// the forward's attention output before the FP8 out-projection.  Each lane keeps its share of
+// the row (groups of 4) in registers between the amax and the conversion.
+constexpr int kQ8MaxVec = 12;  // d <= 1536
+__global__ void __launch_bounds__(256) quantize_rows_bf16_e4m3_kernel(const uint16_t* __restrict__ src,
+                                                                      uint8_t* __restrict__ dst,
+                                                                      float* __restrict__ scale, int rows, int cols) {
+  pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int n4 = cols >> 2;
+  const uint2* in = reinterpret_cast<const uint2*>(src + static_cast<size_t>(row) * cols);
+  float4 v[kQ8MaxVec];
+  float m = 0.f;
+#pragma unroll
+  for (int k = 0; k < kQ8MaxVec; ++k) {
+    const int c = lane + 32 * k;
+    if (c < n4) {
+      const uint2 p = in[c];
+      v[k] = make_float4(bf16_to_f32(static_cast<uint16_t>(p.x & 0xffffu)), bf16_to_f32(static_cast<uint16_t>(p.x >> 16)),
+                         bf16_to_f32(static_cast<uint16_t>(p.y & 0xffffu)), bf16_to_f32(static_cast<uint16_t>(p.y >> 16)));
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w))));
+    }
+  }
+  m = warp_max(m);
+  const float s = m > 0.f ? m * (1.0f / 448.0f) : 1.0f;
+  if (lane == 0) scale[row] = s;
+  const float inv = 1.0f / s;
+  uint32_t* out = reinterpret_cast<uint32_t*>(dst + static_cast<size_t>(row) * cols);
+#pragma unroll
+  for (int k = 0; k < kQ8MaxVec; ++k) {
+    const int c = lane + 32 * k;
+    if (c < n4) out[c] = pack_e4m3x4(v[k].x * inv, v[k].y * inv, v[k].z * inv, v[k].w * inv);
+  }
+}
+
+cudaError_t launch_quantize_rows_bf16_e4m3(const uint16_t* src, uint8_t* dst, float* scale, int rows, int cols,
+                                           cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (cols % 4 || cols > 4 * 32 * kQ8MaxVec) return cudaErrorInvalidValue;
+  return launch_kernel(quantize_rows_bf16_e4m3_kernel, dim3((rows + 7) / 8), dim3(256), 0, st, src, dst, scale, rows,
+                       cols);
+}
+
 // Waits on *flag (never set by anyone) with a bounded spin; records a timeout.
 __global__ void wait_probe_kernel(int* flag, int* status, long long limit_ns) {
   if (threadIdx.x != 0) return;

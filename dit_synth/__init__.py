@@ -59,6 +59,7 @@ class DiTConfig:
     index: int = -1  # position in the standard workload list (seeds); -1 = ad hoc
     block_kind: int = BLOCK_ADALN_ZERO
     ffn_fp8: int = 0   # 1: the feed-forward matmuls on FP8 E4M3 operands
+    attn_fp8: int = 0  # 1: the self-attention's in- and out-projection on FP8 E4M3 operands
 
     # ---- derived shapes (no arithmetic of the method) ----
     @property

@@ -102,6 +102,11 @@ typedef struct dit_config {
                          the LN output per token (amax / 448), the hidden activation per token with
                          the scale (||u||_2 max_n ||fc1.w_n||_2 + max |fc1.b|) / 448, a bound on
                          |GELU(z)| known before z is formed; accumulation stays float32 */
+  int attn_fp8;       /* 1: the self-attention's in- and out-projection run on FP8 E4M3 operands
+                         (bf16 path only): qkv.w / proj.w quantised per output channel (scale
+                         amax / 448) at create, the LN output and the concatenated heads' output
+                         per token (amax / 448); q, k, v, the attention itself and the residual
+                         stream stay bf16 / float32 */
 } dit_config;
 
 typedef struct dit_handle dit_handle;

@@ -56,6 +56,8 @@ def _create(cfg, weights=None, n=None):
     (dict(block_kind=4), binding.DIT_ERR_INVALID_ARG),
     (dict(ffn_fp8=2), binding.DIT_ERR_INVALID_ARG),
     (dict(ffn_fp8=1), binding.DIT_ERR_UNSUPPORTED),          # FP8 feed-forward needs the bf16 path
+    (dict(attn_fp8=3), binding.DIT_ERR_INVALID_ARG),
+    (dict(attn_fp8=1), binding.DIT_ERR_UNSUPPORTED),         # FP8 attention projections need the bf16 path
     (dict(heads=12), binding.DIT_ERR_UNSUPPORTED),           # head dim 32
     (dict(hidden=2048, heads=32, mlp_hidden=8192), binding.DIT_ERR_UNSUPPORTED),  # hidden > 1536
 ])
