@@ -34,8 +34,8 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of each kernel kind,
 # from one cold-cache ncu capture of this workload; a kind whose kernel has changed since its
 # capture has no entry (the roofline then reports traffic null).
-TRAFFIC_BYTES = {"fc1": 58.61e6, "fc2": 129.97e6, "qkv": 45.68e6, "proj": 59.53e6, "attn": 65.25e6,
-                 "ln": 38.10e6, "adaln": 473.41e6, "decode": 18.97e6}
+TRAFFIC_BYTES = {"fc1": 55.06e6, "fc2": 128.64e6, "qkv": 44.19e6, "proj": 59.52e6, "attn": 65.21e6,
+                 "ln": 38.14e6, "adaln": 473.41e6, "decode": 18.97e6}
 TRAFFIC_SOURCE = "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none, one launch, cold cache"
 # fallback peaks (used only when MEASURED_PEAKS.json is absent)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
