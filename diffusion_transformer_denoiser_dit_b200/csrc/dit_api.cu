@@ -208,7 +208,7 @@ struct dit_handle {
   CUtensorMap tm_ada, tm_sc[5], tm_u, tm_o, tm_g, tm_dec, tm_xkv, tm_ctx[5];
   CUtensorMap tm_u8, tb_g8;  // FP8: LN output as fc1's A operand; fc1 output as fc2's B operand
   CUtensorMap tb_u8, tb_o8;  // FP8: LN output / attention output as the swapped GEMMs' B operand
-  CUtensorMap tm_g_out, tm_h_red;  // TMA-store targets: GELU output, residual stream
+  CUtensorMap tm_h_red;  // the residual stream as the TMA reduce-add target
   CUtensorMap tb_u, tb_o, tb_g;     // activations as the B operand of the swapped GEMMs (box 256 rows)
   AttnMaps attn_maps;
   int force_guidance = 0;
@@ -670,7 +670,6 @@ dit_status dit_create(const dit_config* cfg, const float* const* weights, int n_
       ok = ok && make_tmap_e4m3_kmajor(&H->tb_g8, H->g8, g.Mmax, mlp, 256);
     } else {
       ok = ok && make_tmap_bf16_kmajor(&H->tm_g, H->gbuf, g.Mmax, mlp, 128) &&
-           make_tmap_bf16(&H->tm_g_out, H->gbuf, g.Mmax, mlp, 32, 32, 64) &&
            make_tmap_bf16_kmajor(&H->tb_g, H->gbuf, g.Mmax, mlp, 256);
     }
     ok = ok && make_tmap_bf16_kmajor(&H->tm_dec, H->dec_w, g.dec_rows, d, g.bn_dec);
@@ -1194,11 +1193,11 @@ dit_status run_forward(dit_handle* H, const float* x, const float* t, const void
     if (H->bf16) {
       if (H->pair_gemm)
         DIT_LAUNCH(H, DIT_KERNEL_FC1, st,
-                   launch_gemm_tc2(EPI_GELU, 256, &H->tm_u, &b.tm_fc1_h, d, f1, H->num_sms, st, &H->tm_g_out),
+                   launch_gemm_tc2(EPI_GELU, 256, &H->tm_u, &b.tm_fc1_h, d, f1, H->num_sms, st),
                    "fc1 gemm");
       else
         DIT_LAUNCH(H, DIT_KERNEL_FC1, st,
-                   launch_gemm_tc(EPI_GELU, g.bn_fc1, &H->tm_u, &b.tm_fc1, d, f1, H->num_sms, st, &H->tm_g_out),
+                   launch_gemm_tc(EPI_GELU, g.bn_fc1, &H->tm_u, &b.tm_fc1, d, f1, H->num_sms, st),
                    "fc1 gemm");
     } else {
       DIT_LAUNCH(H, DIT_KERNEL_FC1, st, launch_gemm_simt(EPI_GELU, static_cast<const float*>(H->u), static_cast<const float*>(b.fc1_w), p.M,

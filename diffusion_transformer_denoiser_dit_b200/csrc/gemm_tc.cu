@@ -326,7 +326,7 @@ int gemm_tc_supported_bn(int bn) {
 
 cudaError_t launch_gemm_tc(int epi, int bn, const CUtensorMap* tA, const CUtensorMap* tB, int K, const EpiArgs& ea,
                            int num_sms, cudaStream_t st, const CUtensorMap* tC) {
-  if ((epi == EPI_GELU || epi == EPI_RESID_T || epi == EPI_RESID_T8) && tC == nullptr) return cudaErrorInvalidValue;
+  if ((epi == EPI_RESID_T || epi == EPI_RESID_T8) && tC == nullptr) return cudaErrorInvalidValue;
 #define DIT_BN_CASE(BNV, EPIV) \
   if (bn == BNV) return launch_bn<BNV, EPIV>(tA, tB, tC, K, ea, num_sms, st);
   switch (epi) {

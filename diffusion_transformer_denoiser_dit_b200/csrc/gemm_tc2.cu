@@ -262,7 +262,7 @@ int gemm_tc2_supported_bn(int bn) { return bn == 64 || bn == 128 || bn == 144 ||
 
 cudaError_t launch_gemm_tc2(int epi, int bn, const CUtensorMap* tA, const CUtensorMap* tB, int K, const EpiArgs& ea,
                             int num_sms, cudaStream_t st, const CUtensorMap* tC) {
-  if ((epi == EPI_GELU || epi == EPI_RESID_T) && tC == nullptr) return cudaErrorInvalidValue;
+  if (epi == EPI_RESID_T && tC == nullptr) return cudaErrorInvalidValue;
 #define DIT_BN2_CASE(BNV, EPIV) \
   if (bn == BNV) return launch_pair_bn<BNV, EPIV>(tA, tB, tC, K, ea, num_sms, st);
   switch (epi) {

@@ -73,10 +73,9 @@ struct EpiArgs {
 
 // tensor-core GEMM D[M, N] = A[M, K] B[N, K]^T with A, B bf16 K-major.
 // Returns cudaSuccess or the launch error.
-// EPI_GELU and EPI_RESID_T write through shared memory with TMA: tmC maps the output
-// (GELU: bf16 [M, N], box 32 rows x 32 columns, 64B swizzle; RESID_T: the float32
-// residual stream [tokens, features], box 16 tokens x 32 features, 128B swizzle,
-// updated with a TMA reduce-add).  Other epilogues ignore tmC.
+// EPI_RESID_T / EPI_RESID_T8 update the residual stream through shared memory with a TMA
+// reduce-add: tmC maps the float32 stream [tokens, features], box 16 tokens x 32 features,
+// 128B swizzle.  Other epilogues ignore tmC.
 cudaError_t launch_gemm_tc(int epi, int block_n, const CUtensorMap* tmA, const CUtensorMap* tmB, int K,
                            const EpiArgs& ea, int num_sms, cudaStream_t st, const CUtensorMap* tmC = nullptr);
 int gemm_tc_supported_bn(int block_n);
