@@ -6,8 +6,8 @@
 // processed (tcgen05.wait::ld only after the processing), so TMEM latency overlaps
 // the arithmetic and the global-memory traffic of the previous chunk.
 // Epilogues: bias (+ tanh-GELU) to bf16, gated residual update of the float32
-// stream, modulation-vector scatter, head-major Q / K / V^T scatter (per column, or
-// per whole head with QK-RMSNorm and 3D RoPE), plain float32 output.
+// stream, modulation-vector scatter, head-major Q / K / V^T scatter (swapped, or per
+// whole head with QK-RMSNorm and 3D RoPE), plain float32 output.
 #pragma once
 
 #include "common.cuh"
@@ -58,84 +58,6 @@ __device__ __forceinline__ void epilogue_chunk(const EpiArgs& ea, const uint32_t
     float* o = static_cast<float*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n;
     for (int i = 0; i < W && n + i < ea.N; ++i)
       o[i] = __uint_as_float(r[i]) * sm * __ldg(ea.sb + n + i) + (ea.bias ? __ldg(ea.bias + n + i) : 0.f);
-  } else if constexpr (EPI == EPI_GELU) {
-    uint16_t* o = static_cast<uint16_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n;
-    if (full) {
-#pragma unroll
-      for (int i = 0; i < W / 8; ++i) {
-        const float4 b0 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + 2 * i);
-        const float4 b1 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + 2 * i + 1);
-        uint4 pk;
-        pk.x = pack_bf16x2(gelu_tanh_fast(__uint_as_float(r[8 * i + 0]) + b0.x),
-                           gelu_tanh_fast(__uint_as_float(r[8 * i + 1]) + b0.y));
-        pk.y = pack_bf16x2(gelu_tanh_fast(__uint_as_float(r[8 * i + 2]) + b0.z),
-                           gelu_tanh_fast(__uint_as_float(r[8 * i + 3]) + b0.w));
-        pk.z = pack_bf16x2(gelu_tanh_fast(__uint_as_float(r[8 * i + 4]) + b1.x),
-                           gelu_tanh_fast(__uint_as_float(r[8 * i + 5]) + b1.y));
-        pk.w = pack_bf16x2(gelu_tanh_fast(__uint_as_float(r[8 * i + 6]) + b1.z),
-                           gelu_tanh_fast(__uint_as_float(r[8 * i + 7]) + b1.w));
-        reinterpret_cast<uint4*>(o)[i] = pk;
-      }
-    } else {
-      for (int i = 0; i < W && n + i < ea.N; ++i)
-        o[i] = f32_to_bf16(gelu_tanh_fast(__uint_as_float(r[i]) + __ldg(ea.bias + n + i)));
-    }
-  } else if constexpr (EPI == EPI_RESID) {
-    const int row = m / ea.T;
-    const float* gt = ea.gate + static_cast<size_t>(row) * ea.ld_gate + n;
-    float* hp = ea.h + static_cast<size_t>(m) * ea.ldh + n;
-    if (full) {
-      float4 h4[W / 4];
-#pragma unroll
-      for (int i = 0; i < W / 4; ++i) h4[i] = reinterpret_cast<const float4*>(hp)[i];  // all loads in flight first
-#pragma unroll
-      for (int i = 0; i < W / 4; ++i) {
-        const float4 g4 = __ldg(reinterpret_cast<const float4*>(gt) + i);
-        const float4 b4 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + i);
-        h4[i].x = fmaf(g4.x, __uint_as_float(r[4 * i + 0]) + b4.x, h4[i].x);
-        h4[i].y = fmaf(g4.y, __uint_as_float(r[4 * i + 1]) + b4.y, h4[i].y);
-        h4[i].z = fmaf(g4.z, __uint_as_float(r[4 * i + 2]) + b4.z, h4[i].z);
-        h4[i].w = fmaf(g4.w, __uint_as_float(r[4 * i + 3]) + b4.w, h4[i].w);
-        reinterpret_cast<float4*>(hp)[i] = h4[i];
-      }
-    } else {
-      for (int i = 0; i < W && n + i < ea.N; ++i) hp[i] = fmaf(gt[i], __uint_as_float(r[i]) + ea.bias[n + i], hp[i]);
-    }
-  } else if constexpr (EPI == EPI_QKV) {
-    // per column: groups of 8 never straddle a head (head dim % 8 == 0, d % 8 == 0)
-    const int row = m / ea.T, tok = m - row * ea.T;
-#pragma unroll
-    for (int g8 = 0; g8 < W / 8; ++g8) {
-      const int nn = n + 8 * g8;
-      if (nn >= ea.N) break;
-      const int which = nn / ea.d;
-      const int within = nn - which * ea.d;
-      const int head = within / ea.dh, j = within - head * ea.dh;
-      const float4 b0 = __ldg(reinterpret_cast<const float4*>(ea.bias + nn));
-      const float4 b1 = __ldg(reinterpret_cast<const float4*>(ea.bias + nn) + 1);
-      const float v0 = __uint_as_float(r[8 * g8 + 0]) + b0.x, v1 = __uint_as_float(r[8 * g8 + 1]) + b0.y;
-      const float v2 = __uint_as_float(r[8 * g8 + 2]) + b0.z, v3 = __uint_as_float(r[8 * g8 + 3]) + b0.w;
-      const float v4 = __uint_as_float(r[8 * g8 + 4]) + b1.x, v5 = __uint_as_float(r[8 * g8 + 5]) + b1.y;
-      const float v6 = __uint_as_float(r[8 * g8 + 6]) + b1.z, v7 = __uint_as_float(r[8 * g8 + 7]) + b1.w;
-      if (which < 2) {
-        uint16_t* dst = static_cast<uint16_t*>(which == 0 ? ea.q : ea.k) +
-                        (static_cast<size_t>(row * ea.H + head) * ea.Tpad + tok) * ea.DP + j;
-        *reinterpret_cast<uint4*>(dst) =
-            make_uint4(pack_bf16x2(v0, v1), pack_bf16x2(v2, v3), pack_bf16x2(v4, v5), pack_bf16x2(v6, v7));
-      } else {
-        uint16_t* dst =
-            static_cast<uint16_t*>(ea.v) + (static_cast<size_t>(row * ea.H + head) * ea.DP + j) * ea.Tpad + tok;
-        const size_t s = ea.Tpad;
-        dst[0] = f32_to_bf16(v0);
-        dst[s] = f32_to_bf16(v1);
-        dst[2 * s] = f32_to_bf16(v2);
-        dst[3 * s] = f32_to_bf16(v3);
-        dst[4 * s] = f32_to_bf16(v4);
-        dst[5 * s] = f32_to_bf16(v5);
-        dst[6 * s] = f32_to_bf16(v6);
-        dst[7 * s] = f32_to_bf16(v7);
-      }
-    }
   }
 }
 

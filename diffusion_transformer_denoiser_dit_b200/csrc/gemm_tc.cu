@@ -338,11 +338,6 @@ cudaError_t launch_gemm_tc(int epi, int bn, const CUtensorMap* tA, const CUtenso
       DIT_BN_CASE(128, EPI_ADALN) DIT_BN_CASE(256, EPI_ADALN) break;
     case EPI_GELU:
       DIT_BN_CASE(128, EPI_GELU) DIT_BN_CASE(256, EPI_GELU) break;
-    case EPI_RESID:
-      DIT_BN_CASE(128, EPI_RESID) DIT_BN_CASE(192, EPI_RESID)
-      DIT_BN_CASE(256, EPI_RESID) break;
-    case EPI_QKV:
-      DIT_BN_CASE(128, EPI_QKV) DIT_BN_CASE(144, EPI_QKV) DIT_BN_CASE(192, EPI_QKV) DIT_BN_CASE(256, EPI_QKV) break;
     case EPI_QKV_HEAD:
       DIT_BN_CASE(128, EPI_QKV_HEAD) DIT_BN_CASE(144, EPI_QKV_HEAD) break;
     case EPI_RESID_T:

@@ -272,14 +272,6 @@ cudaError_t launch_gemm_tc2(int epi, int bn, const CUtensorMap* tA, const CUtens
     case EPI_GELU:
       DIT_BN2_CASE(128, EPI_GELU) DIT_BN2_CASE(256, EPI_GELU)
       break;
-    case EPI_RESID:
-      DIT_BN2_CASE(128, EPI_RESID) DIT_BN2_CASE(192, EPI_RESID)
-      DIT_BN2_CASE(256, EPI_RESID) break;
-    case EPI_QKV:
-      DIT_BN2_CASE(128, EPI_QKV) DIT_BN2_CASE(144, EPI_QKV) DIT_BN2_CASE(192, EPI_QKV) DIT_BN2_CASE(256, EPI_QKV)
-      break;
-    case EPI_QKV_HEAD:
-      DIT_BN2_CASE(128, EPI_QKV_HEAD) DIT_BN2_CASE(144, EPI_QKV_HEAD) break;
     case EPI_RESID_T:
       DIT_BN2_CASE(256, EPI_RESID_T) break;
     case EPI_QKV_T:
