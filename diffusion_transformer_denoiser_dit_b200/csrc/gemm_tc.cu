@@ -2,10 +2,11 @@
 // float32 accumulation in tensor memory, with the DiT epilogues fused in.
 //
 // Design (one persistent CTA per SM, 320 threads = 10 warps):
-//   warp 0      TMA producer: 128x64 A tile + BNx64 B tile per stage, 128-byte
-//               swizzle, STAGES-deep ring guarded by full/empty mbarriers.
+//   warp 0      TMA producer: 128 rows of A and BN rows of B per stage, 128 bytes of K
+//               each (64 bf16 or 128 E4M3 elements), 128-byte swizzle, STAGES-deep ring
+//               guarded by full/empty mbarriers.
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
-//               (M=128, N=BN, K=16, four per 64-wide stage) into one of two TMEM
+//               (M=128, N=BN, K=16 bf16 or 32 E4M3, four per stage) into one of two TMEM
 //               accumulators and commits stage releases / accumulator hand-off.
 //   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4)..+31 (one output row per
 //               thread) and one half of the tile's columns (warps 2-5 the first half,
