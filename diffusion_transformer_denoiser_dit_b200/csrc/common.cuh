@@ -112,10 +112,6 @@ __device__ __forceinline__ float tanh_fast(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ float gelu_tanh_fast(float x) {
-  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-  return 0.5f * x * (1.0f + tanh_fast(k0 * (x + k1 * x * x * x)));
-}
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -379,6 +375,25 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// tanh-GELU of a pair of floats, 0.5 x (1 + tanh(k0 (x + k1 x^3))), with the polynomial written
+// as x (k0 + k0 k1 x^2) and 0.5 x (1 + t) as 0.5 x + 0.5 x t, so that everything but the two
+// tanh evaluations runs as paired float32 instructions (half the instructions of two scalar
+// evaluations; the epilogue that applies it runs beside the GEMM's main loop).
+__device__ __forceinline__ uint64_t gelu_tanh_fast_f2(uint64_t x2) {
+  constexpr float k0 = 0.7978845608028654f, k01 = 0.7978845608028654f * 0.044715f;
+  const uint64_t sq = f2_mul(x2, x2);
+  float u0, u1;
+  f2_unpack(f2_mul(x2, f2_fma(sq, f2_pack(k01, k01), f2_pack(k0, k0))), u0, u1);
+  const uint64_t hx = f2_mul(x2, f2_pack(0.5f, 0.5f));
+  return f2_fma(hx, f2_pack(tanh_fast(u0), tanh_fast(u1)), hx);
+}
+// pack_bf16x2 of a float pair
+__device__ __forceinline__ uint32_t pack_bf16x2_f2(uint64_t v) {
+  float lo, hi;
+  f2_unpack(v, lo, hi);
+  return pack_bf16x2(lo, hi);
 }
 
 // 2^x for a pair of floats on the FMA and integer pipes instead of the MUFU unit.  x is

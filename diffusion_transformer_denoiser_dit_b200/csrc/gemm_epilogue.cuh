@@ -227,15 +227,16 @@ __device__ __forceinline__ void epilogue_cols_staged(const EpiArgs& ea, uint32_t
       for (int c16 = 0; c16 < 4; ++c16) {
         const float4 b0 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + 2 * c16);
         const float4 b1 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + 2 * c16 + 1);
-        uint4 pk;
-        pk.x = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 0]) + b0.x),
-                           gelu_tanh_fast(__uint_as_float(v[8 * c16 + 1]) + b0.y));
-        pk.y = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 2]) + b0.z),
-                           gelu_tanh_fast(__uint_as_float(v[8 * c16 + 3]) + b0.w));
-        pk.z = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 4]) + b1.x),
-                           gelu_tanh_fast(__uint_as_float(v[8 * c16 + 5]) + b1.y));
-        pk.w = pack_bf16x2(gelu_tanh_fast(__uint_as_float(v[8 * c16 + 6]) + b1.z),
-                           gelu_tanh_fast(__uint_as_float(v[8 * c16 + 7]) + b1.w));
+        const uint32_t* w = v + 8 * c16;
+        uint4 pk;  // bias and GELU on column pairs (paired float32 instructions)
+        pk.x = pack_bf16x2_f2(gelu_tanh_fast_f2(
+            f2_add(f2_pack(__uint_as_float(w[0]), __uint_as_float(w[1])), f2_pack(b0.x, b0.y))));
+        pk.y = pack_bf16x2_f2(gelu_tanh_fast_f2(
+            f2_add(f2_pack(__uint_as_float(w[2]), __uint_as_float(w[3])), f2_pack(b0.z, b0.w))));
+        pk.z = pack_bf16x2_f2(gelu_tanh_fast_f2(
+            f2_add(f2_pack(__uint_as_float(w[4]), __uint_as_float(w[5])), f2_pack(b1.x, b1.y))));
+        pk.w = pack_bf16x2_f2(gelu_tanh_fast_f2(
+            f2_add(f2_pack(__uint_as_float(w[6]), __uint_as_float(w[7])), f2_pack(b1.z, b1.w))));
         *reinterpret_cast<uint4*>(stg + lane * 128 + (((h * 4 + c16) ^ (lane & 7)) << 4)) = pk;
       }
     }
@@ -293,18 +294,23 @@ __device__ __forceinline__ void epilogue_resid_t(const EpiArgs& ea, const CUtens
         if (lane == 0) bulk_wait_read_but1();
         __syncwarp();
 #pragma unroll
-        for (int tt = 0; tt < 16; ++tt) {
+        for (int tt = 0; tt < 16; tt += 2) {  // token pairs: paired float32 arithmetic
           const int t = half * 16 + tt;
-          float g = g0;
+          float ga = g0, gb = g0;
           if (r1 != r0) {
-            const int rt = min(tok0 + t, ea.N - 1) / ea.T;
-            g = fok ? __ldg(ea.gate + static_cast<size_t>(rt) * ea.ld_gate + f) : 0.f;
+            const int ra = min(tok0 + t, ea.N - 1) / ea.T, rb = min(tok0 + t + 1, ea.N - 1) / ea.T;
+            ga = fok ? __ldg(ea.gate + static_cast<size_t>(ra) * ea.ld_gate + f) : 0.f;
+            gb = fok ? __ldg(ea.gate + static_cast<size_t>(rb) * ea.ld_gate + f) : 0.f;
           }
-          float acc = __uint_as_float(v[t]);
-          if constexpr (FP8) acc *= sf * __shfl_sync(0xffffffffu, st_l, t);
+          uint64_t acc = f2_pack(__uint_as_float(v[t]), __uint_as_float(v[t + 1]));
+          if constexpr (FP8)
+            acc = f2_mul(acc, f2_pack(sf * __shfl_sync(0xffffffffu, st_l, t), sf * __shfl_sync(0xffffffffu, st_l, t + 1)));
+          float ya, yb;
+          f2_unpack(f2_mul(f2_add(acc, f2_pack(bf, bf)), f2_pack(ga, gb)), ya, yb);
           // [token][feature] float32 rows of 128 bytes, 128B swizzle
-          *reinterpret_cast<float*>(buf + tt * 128 + ((((lane >> 2) ^ (tt & 7)) << 4) | ((lane & 3) << 2))) =
-              g * (acc + bf);
+          *reinterpret_cast<float*>(buf + tt * 128 + ((((lane >> 2) ^ (tt & 7)) << 4) | ((lane & 3) << 2))) = ya;
+          *reinterpret_cast<float*>(buf + (tt + 1) * 128 + ((((lane >> 2) ^ ((tt + 1) & 7)) << 4) | ((lane & 3) << 2))) =
+              yb;
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -342,12 +348,16 @@ __device__ __forceinline__ void epilogue_gelu8(const EpiArgs& ea, uint32_t tacc,
       for (int i4 = 0; i4 < 8; ++i4) {
         const float4 s4 = __ldg(reinterpret_cast<const float4*>(ea.sb + n) + i4);
         const float4 b4 = __ldg(reinterpret_cast<const float4*>(ea.bias + n) + i4);
-        const float z0 = fmaf(__uint_as_float(v[4 * i4 + 0]) * sm, s4.x, b4.x);
-        const float z1 = fmaf(__uint_as_float(v[4 * i4 + 1]) * sm, s4.y, b4.y);
-        const float z2 = fmaf(__uint_as_float(v[4 * i4 + 2]) * sm, s4.z, b4.z);
-        const float z3 = fmaf(__uint_as_float(v[4 * i4 + 3]) * sm, s4.w, b4.w);
-        pk[i4] = pack_e4m3x4(gelu_tanh_fast(z0) * inv, gelu_tanh_fast(z1) * inv, gelu_tanh_fast(z2) * inv,
-                             gelu_tanh_fast(z3) * inv);
+        // z = sm s acc + bias and GELU on column pairs (paired float32 instructions)
+        const uint64_t sm2 = f2_pack(sm, sm), inv2 = f2_pack(inv, inv);
+        const uint64_t za = f2_fma(f2_mul(f2_pack(__uint_as_float(v[4 * i4 + 0]), __uint_as_float(v[4 * i4 + 1])), sm2),
+                                   f2_pack(s4.x, s4.y), f2_pack(b4.x, b4.y));
+        const uint64_t zb = f2_fma(f2_mul(f2_pack(__uint_as_float(v[4 * i4 + 2]), __uint_as_float(v[4 * i4 + 3])), sm2),
+                                   f2_pack(s4.z, s4.w), f2_pack(b4.z, b4.w));
+        float g0, g1, g2, g3;
+        f2_unpack(f2_mul(gelu_tanh_fast_f2(za), inv2), g0, g1);
+        f2_unpack(f2_mul(gelu_tanh_fast_f2(zb), inv2), g2, g3);
+        pk[i4] = pack_e4m3x4(g0, g1, g2, g3);
       }
       uint4* o = reinterpret_cast<uint4*>(static_cast<uint8_t*>(ea.out) + static_cast<size_t>(m) * ea.ldo + n);
       o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -441,16 +451,17 @@ __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc,
       const bool one_row = (last / ea.T) == r0 && last - tok0 == 31;
       if (warp_one_kind && one_row && (which < 2 || (t0 & 7) == 0)) {
         uint8_t* buf = stg + (c & 1) * 2048;
+        const uint64_t bf2 = f2_pack(bf, bf);
         __syncwarp();  // every lane is done reading this buffer's previous chunk
         if (which == 2) {
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const uint32_t* w = v + 8 * g;
             *reinterpret_cast<uint4*>(buf + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) =
-                make_uint4(pack_bf16x2(__uint_as_float(w[0]) + bf, __uint_as_float(w[1]) + bf),
-                           pack_bf16x2(__uint_as_float(w[2]) + bf, __uint_as_float(w[3]) + bf),
-                           pack_bf16x2(__uint_as_float(w[4]) + bf, __uint_as_float(w[5]) + bf),
-                           pack_bf16x2(__uint_as_float(w[6]) + bf, __uint_as_float(w[7]) + bf));
+                make_uint4(pack_bf16x2_f2(f2_add(f2_pack(__uint_as_float(w[0]), __uint_as_float(w[1])), bf2)),
+                           pack_bf16x2_f2(f2_add(f2_pack(__uint_as_float(w[2]), __uint_as_float(w[3])), bf2)),
+                           pack_bf16x2_f2(f2_add(f2_pack(__uint_as_float(w[4]), __uint_as_float(w[5])), bf2)),
+                           pack_bf16x2_f2(f2_add(f2_pack(__uint_as_float(w[6]), __uint_as_float(w[7])), bf2)));
           }
           __syncwarp();
           uint16_t* vb = static_cast<uint16_t*>(ea.v) + static_cast<size_t>(r0 * ea.H) * ea.DP * ea.Tpad + t0 +
@@ -463,8 +474,11 @@ __device__ __forceinline__ void epilogue_qkv_t(const EpiArgs& ea, uint32_t tacc,
           }
         } else {
 #pragma unroll
-          for (int t = 0; t < 32; ++t)
-            *reinterpret_cast<uint16_t*>(buf + t * 64 + lane * 2) = f32_to_bf16(__uint_as_float(v[t]) + bf);
+          for (int t = 0; t < 32; t += 2) {  // bias and conversion on token pairs, one row each
+            const uint32_t p = pack_bf16x2_f2(f2_add(f2_pack(__uint_as_float(v[t]), __uint_as_float(v[t + 1])), bf2));
+            *reinterpret_cast<uint16_t*>(buf + t * 64 + lane * 2) = static_cast<uint16_t>(p & 0xffffu);
+            *reinterpret_cast<uint16_t*>(buf + (t + 1) * 64 + lane * 2) = static_cast<uint16_t>(p >> 16);
+          }
           __syncwarp();
           uint16_t* qb = qk + (static_cast<size_t>(r0 * ea.H + gh) * ea.Tpad + t0) * ea.DP + gj;
 #pragma unroll
