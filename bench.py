@@ -34,7 +34,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of each kernel kind,
 # from one cold-cache ncu capture of this workload; a kind whose kernel has changed since its
 # capture has no entry (the roofline then reports traffic null).
-TRAFFIC_BYTES = {"fc1": 55.06e6, "fc2": 128.64e6, "qkv": 44.19e6, "proj": 59.52e6, "attn": 65.21e6,
+TRAFFIC_BYTES = {"fc1": 55.16e6, "fc2": 130.17e6, "qkv": 44.23e6, "proj": 59.56e6, "attn": 65.21e6,
                  "ln": 38.14e6, "adaln": 473.41e6, "decode": 18.97e6}
 TRAFFIC_SOURCE = "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none, one launch, cold cache"
 # fallback peaks (used only when MEASURED_PEAKS.json is absent)
