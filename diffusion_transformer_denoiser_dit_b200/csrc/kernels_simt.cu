@@ -28,52 +28,65 @@ __global__ void cond_sinusoid_kernel(const float* __restrict__ t, int B, int R, 
   }
 }
 
-// The condition MLP's two layers, out[r, j] = W[j] . in[r] + b[j] for all sample rows r:
-// a block of 8 warps owns 8 output features (one per warp) and a group of up to 32 rows
-// (lane = row).  The group's whole input rows [32, K] are staged in shared memory at once
-// (every load in flight together; rows padded to K + 1 floats so the lanes' reads fall in
-// different banks); each lane loads 32 consecutive weights of its warp's feature at a time and
-// hands them round with shuffles, into four independent accumulators.
-constexpr int kCondRows = 32;
+// The condition MLP's two layers, out[r, j] = W[j] . in[r] + b[j] for all sample rows r.  A
+// block of 8 warps owns 8 output features and a group of up to 32 rows.  The 8 weight rows are
+// staged in shared memory once (coalesced float4 loads) and read back as broadcasts; warp w takes
+// the w-th eighth of K for every row of the group (lane = row, its input row read as float4), so
+// each 16-byte input load feeds 32 multiply-adds into 8 independent accumulators; the 8 partial
+// sums of every (row, feature) are added through shared memory.  Thread t then owns row t / 8 and
+// feature t % 8, so a warp's outputs are 4 rows of 8 consecutive features.
+constexpr int kCondRows = 32, kCondFeat = 8, kCondWarps = 8;
+constexpr int kCondRedLd = kCondFeat + 1;  // padded so the lanes' partial-sum writes hit distinct banks
 
-// Stage rows are Kpad + 1 floats, Kpad = K rounded up to 32, zero past K (K % 4 == 0).
-__host__ __device__ inline int cond_stage_ld(int K) { return (K + 31) / 32 * 32 + 1; }
+// Dynamic shared memory of one block: the weight slab [kCondFeat][K] and the partial sums
+// [kCondWarps][kCondRows][kCondRedLd].
+__host__ __device__ inline size_t cond_smem_bytes(int K) {
+  return (static_cast<size_t>(kCondFeat) * K + static_cast<size_t>(kCondWarps) * kCondRows * kCondRedLd) *
+         sizeof(float);
+}
 
-__device__ __forceinline__ float cond_dot(const float* __restrict__ w, const float* __restrict__ in, int K, int r0,
-                                          int nr, float* stage, int lane) {
-  __syncthreads();  // the previous row group's reads of the stage are done
-  const int ld = cond_stage_ld(K), K4 = K >> 2, Kpad = ld - 1;
-  for (int i = threadIdx.x; i < nr * K4; i += blockDim.x) {
-    const int rr = i / K4, k4 = i - rr * K4;
-    const float4 v = reinterpret_cast<const float4*>(in + static_cast<size_t>(r0 + rr) * K)[k4];
-    float* dst = stage + rr * ld + 4 * k4;
-    dst[0] = v.x;
-    dst[1] = v.y;
-    dst[2] = v.z;
-    dst[3] = v.w;
+// ws[f * K + k] = W[min(j0 + f, N - 1), k]  (K % 4 == 0; rows past N repeat the last one and are
+// never stored)
+__device__ __forceinline__ void cond_stage_w(const float* __restrict__ W, int N, int K, int j0, float* ws) {
+  const int K4 = K >> 2;
+  for (int i = threadIdx.x; i < kCondFeat * K4; i += blockDim.x) {
+    const int f = i / K4, k4 = i - f * K4;
+    const int j = min(j0 + f, N - 1);
+    reinterpret_cast<float4*>(ws + f * K)[k4] = __ldg(reinterpret_cast<const float4*>(W + static_cast<size_t>(j) * K) + k4);
   }
-  for (int i = threadIdx.x; i < kCondRows * (Kpad - K); i += blockDim.x) {  // zero tail of every row
-    const int rr = i / (Kpad - K);
-    stage[rr * ld + K + (i - rr * (Kpad - K))] = 0.f;
+}
+
+// W[j0 + t % 8] . in[r0 + t / 8] for the calling thread t (0 when that row is past the group);
+// every thread of the block calls it, and it leaves the partial-sum area free for the next call.
+__device__ __forceinline__ float cond_dot8(const float* __restrict__ in, int K, int r0, int nr, const float* ws,
+                                           float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K4 = K >> 2, per = (K4 + kCondWarps - 1) / kCondWarps;
+  const int c0 = warp * per, c1 = min(c0 + per, K4);
+  float acc[kCondFeat];
+#pragma unroll
+  for (int f = 0; f < kCondFeat; ++f) acc[f] = 0.f;
+  if (lane < nr) {
+    const float4* x = reinterpret_cast<const float4*>(in + static_cast<size_t>(r0 + lane) * K);
+#pragma unroll 4
+    for (int c = c0; c < c1; ++c) {
+      const float4 v = x[c];
+#pragma unroll
+      for (int f = 0; f < kCondFeat; ++f) {
+        const float4 w = reinterpret_cast<const float4*>(ws + f * K)[c];
+        acc[f] = fmaf(v.w, w.w, fmaf(v.z, w.z, fmaf(v.y, w.y, fmaf(v.x, w.x, acc[f]))));
+      }
+    }
   }
-  for (int i = threadIdx.x; i < (kCondRows - nr) * K; i += blockDim.x)  // rows past the group: zero
-    stage[(nr + i / K) * ld + i % K] = 0.f;
+  __syncthreads();  // the previous call's readers of red are done
+#pragma unroll
+  for (int f = 0; f < kCondFeat; ++f) red[(warp * kCondRows + lane) * kCondRedLd + f] = acc[f];
   __syncthreads();
-  // the warp's whole weight row, lane l holding elements l, l + 32, ...: all loads in flight
-  // at once instead of one round trip per 32-wide step
-  constexpr int kMaxW = 1536 / 32;
-  float wreg[kMaxW];
+  const int r = threadIdx.x / kCondFeat, f = threadIdx.x % kCondFeat;
+  float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxW; ++i) wreg[i] = (32 * i < Kpad && 32 * i + lane < K) ? __ldg(w + 32 * i + lane) : 0.f;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const float* srow = stage + lane * ld;
-#pragma unroll
-  for (int i = 0; i < kMaxW; ++i) {
-    if (32 * i >= Kpad) break;
-#pragma unroll
-    for (int q = 0; q < 32; ++q) acc[q & 3] = fmaf(__shfl_sync(0xffffffffu, wreg[i], q), srow[32 * i + q], acc[q & 3]);
-  }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  for (int w = 0; w < kCondWarps; ++w) s += red[(w * kCondRows + r) * kCondRedLd + f];
+  return s;
 }
 
 // hid[r, j] = SiLU(W1[j] . E[r] + b1[j])
@@ -82,14 +95,17 @@ __global__ void __launch_bounds__(256) cond_hidden_kernel(const float* __restric
                                                           int K, int N) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ float stage[];  // [32][K + 1]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * 8 + warp;
-  const int jc = j < N ? j : N - 1;  // every warp takes part in the block's staging barriers
+  extern __shared__ float4 cond_smem4[];
+  float* ws = reinterpret_cast<float*>(cond_smem4);
+  float* red = ws + kCondFeat * K;
+  const int j0 = blockIdx.x * kCondFeat;
+  cond_stage_w(W1, N, K, j0, ws);
+  __syncthreads();
+  const int j = j0 + threadIdx.x % kCondFeat, rl = threadIdx.x / kCondFeat;
   for (int r0 = blockIdx.y * kCondRows; r0 < R; r0 += gridDim.y * kCondRows) {
     const int nr = min(kCondRows, R - r0);
-    const float v = cond_dot(W1 + static_cast<size_t>(jc) * K, E, K, r0, nr, stage, lane);
-    if (j < N && lane < nr) hid[static_cast<size_t>(r0 + lane) * N + j] = silu_f(v + b1[j]);
+    const float v = cond_dot8(E, K, r0, nr, ws, red);
+    if (j < N && rl < nr) hid[static_cast<size_t>(r0 + rl) * N + j] = silu_f(v + b1[j]);
   }
 }
 
@@ -99,15 +115,18 @@ __global__ void __launch_bounds__(256) cond_hidden_kernel(const float* __restric
 __global__ void __launch_bounds__(256) cond_out_kernel(CondArgs a) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ float stage[];  // [32][d + 1]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * 8 + warp;
-  const int jc = j < a.d ? j : a.d - 1;
+  extern __shared__ float4 cond_smem4[];
+  float* ws = reinterpret_cast<float*>(cond_smem4);
+  float* red = ws + kCondFeat * a.d;
+  const int j0 = blockIdx.x * kCondFeat;
+  cond_stage_w(a.w2, a.d, a.d, j0, ws);
+  __syncthreads();
+  const int j = j0 + threadIdx.x % kCondFeat, rl = threadIdx.x / kCondFeat;
   for (int r0 = blockIdx.y * kCondRows; r0 < a.R; r0 += gridDim.y * kCondRows) {
     const int nr = min(kCondRows, a.R - r0);
-    const float acc = cond_dot(a.w2 + static_cast<size_t>(jc) * a.d, a.hid, a.d, r0, nr, stage, lane);
-    if (j >= a.d || lane >= nr) continue;
-    const int r = r0 + lane;
+    const float acc = cond_dot8(a.hid, a.d, r0, nr, ws, red);
+    if (j >= a.d || rl >= nr) continue;
+    const int r = r0 + rl;
     const float et = acc + a.b2[j];  // timestep embedding
     float ey;                        // class embedding / text vector
     if (a.cond_kind == DIT_COND_CLASS) {
@@ -153,13 +172,13 @@ __global__ void __launch_bounds__(256) cond_out_kernel(CondArgs a) {
 
 cudaError_t launch_condition(const CondArgs& a, cudaStream_t st) {
   if ((a.freq % 4) != 0 || (a.d % 4) != 0) return cudaErrorInvalidValue;
-  const size_t smem_h = static_cast<size_t>(kCondRows) * cond_stage_ld(a.freq) * sizeof(float);
-  const size_t smem_o = static_cast<size_t>(kCondRows) * cond_stage_ld(a.d) * sizeof(float);
+  const size_t smem_h = cond_smem_bytes(a.freq);
+  const size_t smem_o = cond_smem_bytes(a.d);
   static bool attr_done[kMaxDevices] = {};
   const int dev = current_device();
   if (dev < 0) return cudaErrorInvalidDevice;
   if (!attr_done[dev]) {  // the largest stage the library's limits allow (d, freq_dim <= 1536)
-    const int mx = static_cast<int>(static_cast<size_t>(kCondRows) * cond_stage_ld(1536) * sizeof(float));
+    const int mx = static_cast<int>(cond_smem_bytes(1536));
     cudaError_t e = cudaFuncSetAttribute(cond_hidden_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(cond_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
     if (e != cudaSuccess) return e;
@@ -171,10 +190,11 @@ cudaError_t launch_condition(const CondArgs& a, cudaStream_t st) {
                                  a.t_scale, a.E);
   if (e != cudaSuccess) return e;
   const int rg = (a.R + kCondRows - 1) / kCondRows;
-  e = launch_kernel(cond_hidden_kernel, dim3((a.d + 7) / 8, rg), dim3(256), smem_h, st, (const float*)a.E, a.w1, a.b1,
-                    a.hid, a.R, a.freq, a.d);
+  const dim3 grid((a.d + kCondFeat - 1) / kCondFeat, rg);
+  e = launch_kernel(cond_hidden_kernel, grid, dim3(kCondWarps * 32), smem_h, st, (const float*)a.E, a.w1, a.b1, a.hid,
+                    a.R, a.freq, a.d);
   if (e != cudaSuccess) return e;
-  return launch_kernel(cond_out_kernel, dim3((a.d + 7) / 8, rg), dim3(256), smem_o, st, a);
+  return launch_kernel(cond_out_kernel, grid, dim3(kCondWarps * 32), smem_o, st, a);
 }
 
 // ============================================================================ patch embed
@@ -343,6 +363,8 @@ cudaError_t launch_patch_embed(const PatchArgs& a, cudaStream_t st) {
 constexpr int kLnMaxVec = 12;   // d <= 1536 (float4 per lane)
 constexpr int kLnRows = 32;     // token rows per block
 constexpr int kLnThreads = 256;
+constexpr int kLnWarpRows = kLnRows / (kLnThreads / 32);  // rows per warp, taken two at a time
+static_assert(kLnWarpRows % 2 == 0, "a warp normalises its rows in pairs");
 
 // Writes the modulated row; the normalised values replace x (the E4M3 output needs them twice).
 template <int OUT, int VEC>
@@ -433,7 +455,7 @@ __global__ void __launch_bounds__(kLnThreads) ln_modulate_kernel(LnArgs a) {
   const int m0 = blockIdx.x * kLnRows;
   float4 xa[VEC], xb[VEC];
   {
-    const int ma = m0 + warp * (kLnRows / 8), mb = ma + 1;
+    const int ma = m0 + warp * kLnWarpRows, mb = ma + 1;
     if (ma < a.M) ln_load_row<VEC>(a.h + static_cast<size_t>(ma) * a.d, lane, nv, xa);
     if (mb < a.M) ln_load_row<VEC>(a.h + static_cast<size_t>(mb) * a.d, lane, nv, xb);
   }
@@ -450,8 +472,8 @@ __global__ void __launch_bounds__(kLnThreads) ln_modulate_kernel(LnArgs a) {
     }
   }
   __syncthreads();
-  for (int pr = 0; pr < kLnRows / 8; pr += 2) {  // each warp: rows m0 + 4 warp + {0, 1}, then {2, 3}
-    const int ma = m0 + warp * (kLnRows / 8) + pr, mb = ma + 1;
+  for (int pr = 0; pr < kLnWarpRows; pr += 2) {  // each warp: rows m0 + kLnWarpRows warp + {0, 1}, {2, 3}, ...
+    const int ma = m0 + warp * kLnWarpRows + pr, mb = ma + 1;
     if (ma >= a.M) break;
     const bool hb = mb < a.M;
     if (pr > 0) {
